@@ -1,0 +1,350 @@
+"""Benchmark of the W8A8 MoE expert-FFN layer forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+A step is one whole forward (router, grouping + quantisation, gate_up GEMM, requantisation,
+down GEMM, combine) over one batch of synthetic tokens. Default workload: the Qwen3-30B-A3B
+shaped decode layer (64 tokens, hidden 2048, 128 experts, top-8, intermediate 768).
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and a device
+synchronisation on both sides, timed with CUDA events on the launching stream; the maximum
+over ranks is reported. Each step streams the touched experts' weights (about 597 MB for the
+decode layer), more than the 126 MB L2, so no step is served from L2 by the previous one.
+
+Multi-GPU (torchrun): replicas. Every rank holds the full layer and runs its own batch of the
+same size; nothing is exchanged on the data path (tokens are independent), so scaling is weak.
+
+--impl reference times the CPU oracle on this host on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W8A8 MoE layer tokens/s on 1 B200; INT8 TOPS and HBM GB/s vs peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="qwen3-30b-a3b-decode")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                break
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle leg
+def cpu_oracle_rate(wl, n_tokens: int, min_seconds: float = 10.0, max_seconds: float = 30.0):
+    """Times the oracle (as it stands) on `n_tokens` tokens of the workload; tokens/s."""
+    from oracle import w8a8_oracle as O
+    from w8a8_int8_quantized_act_b200 import synth
+
+    x = synth.activations(wl.T, wl.H, wl.n_outlier, wl.seed)[:n_tokens]
+    wg = synth.router_weight(wl.E, wl.H, wl.seed)
+    bias = synth.router_bias(wl.E, wl.seed) if wl.skewed else None
+    r = O.route(x, wg, bias, wl.k, wl.renorm)
+    touched = np.unique(r.ids)
+    gq, gs = O.quantize_weight_per_channel(synth.expert_gate_up(wl.E, wl.I, wl.H, wl.seed, experts=touched))
+    dq, ds = O.quantize_weight_per_channel(synth.expert_down(wl.E, wl.H, wl.I, wl.seed, experts=touched))
+    d = lambda a: {int(e): a[i] for i, e in enumerate(touched)}  # noqa: E731
+    wgu_q, s_gu, wd_q, s_d = d(gq), d(gs), d(dq), d(ds)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        O.moe_forward(x, wg, bias, wgu_q, s_gu, wd_q, s_d, wl.k, wl.renorm)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or (reps >= 1 and el * (reps + 1) / reps > max_seconds):
+            break
+    return n_tokens * reps / el, reps, el
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def default_sample_tokens(wl) -> int:
+    return min(wl.T, 16)
+
+
+# ---------------------------------------------------------------------------- algorithmic work
+def algorithmic(wl, counts: np.ndarray):
+    """Algorithmic ops and bytes of one layer forward, and bytes of the gate_up launch."""
+    touched = int((counts > 0).sum())
+    A = wl.T * wl.k
+    ops = 2 * A * (2 * wl.I * wl.H + wl.H * wl.I) + 2 * wl.T * wl.H * wl.E
+    w_bytes = touched * (3 * wl.I * wl.H + 4 * (2 * wl.I + wl.H))
+    io_bytes = 2 * wl.T * wl.H * 2 + 2 * wl.E * wl.H
+    gate_up_bytes = touched * (2 * wl.I * wl.H + 4 * 2 * wl.I) + A * wl.H + A * wl.I * 2
+    down_bytes = touched * (wl.H * wl.I + 4 * wl.H) + A * wl.I + A * wl.H * 2
+    return dict(ops=ops, bytes=w_bytes + io_bytes, touched=touched, gate_up_bytes=gate_up_bytes,
+                down_bytes=down_bytes, gate_up_ops=2 * A * 2 * wl.I * wl.H, down_ops=2 * A * wl.H * wl.I)
+
+
+# ---------------------------------------------------------------------------- native arm
+def run_native(args, wl, rank, world, dist):
+    import torch
+
+    from w8a8_int8_quantized_act_b200 import binding as B
+    from w8a8_int8_quantized_act_b200 import synth
+
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B.lib()
+    # every rank: its own batch of wl.T tokens (seeded by rank), the full layer's weights
+    x_host = synth.activations(wl.T, wl.H, wl.n_outlier, wl.seed + rank)
+    inp = synth.moe_inputs(wl)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
+    x = bf(x_host)
+    wg = bf(inp.wg)
+    bias = torch.from_numpy(inp.bias).to(dev) if inp.bias is not None else None
+    wgu_q, s_gu = B.w8a8_quantize_weight_per_channel(bf(inp.wgu))
+    wd_q, s_d = B.w8a8_quantize_weight_per_channel(bf(inp.wd))
+    del inp
+    torch.cuda.empty_cache()
+    ws = torch.empty(B.w8a8_moe_workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I), dtype=torch.uint8, device=dev)
+    y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        B.w8a8_moe_forward(x, wg, wgu_q, s_gu, wd_q, s_d, wl.k, renorm=wl.renorm, bias=bias, workspace=ws, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    B.w8a8_check_status()
+    counts = np.diff(B.moe_intermediates(ws, wl.T, wl.H, wl.E, wl.k, wl.I)["offsets"].cpu().numpy())
+
+    # ---- timed region: K profiled steps (stage events give the per-kernel durations)
+    nst = 7
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            B.w8a8_moe_forward_profiled(x, wg, wgu_q, s_gu, wd_q, s_d, wl.k, ev[i], renorm=wl.renorm, bias=bias,
+                                        workspace=ws, y=y)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    B.w8a8_check_status()
+    ms = start.elapsed_time(stop)
+    stage_ms = np.zeros(nst - 1)
+    for i in range(args.steps):
+        for s_ in range(nst - 1):
+            stage_ms[s_] += ev[i][s_].elapsed_time(ev[i][s_ + 1])
+    stage_ms /= args.steps
+
+    # ---- end to end through the public API with host buffers (copies inside the timed region)
+    x_pin = torch.from_numpy(x_host).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 500))
+    for _ in range(3):
+        x.copy_(x_pin, non_blocking=True)
+        step()
+        y_pin.copy_(y, non_blocking=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_pin, non_blocking=True)
+        step()
+        y_pin.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms = float(t[0]), float(t[1])
+    return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, stage_ms=stage_ms, counts=counts,
+                clocks=clk.summary(), h2d=wl.T * wl.H * 2, d2h=wl.T * wl.H * 2)
+
+
+def main():
+    args = parse()
+    from w8a8_int8_quantized_act_b200 import synth
+
+    wl = synth.MOE_WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    peaks, peak_kind = load_peaks()
+    sample = args.cpu_sample_tokens or default_sample_tokens(wl)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        rate, reps, el = cpu_oracle_rate(wl, sample, min_seconds=min(30.0, 2.0 * max(1, args.steps)),
+                                         max_seconds=120.0)
+        cores = blas_threads()
+        samp = f"{sample} of the workload's {wl.T} tokens per step, {reps} oracle forwards in {el:.1f} s"
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I},
+            "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": samp},
+            "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_mod
+
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    res = run_native(args, wl, rank, world, dist)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    K = args.steps
+    ms_step = res["ms"] / K
+    value = world * wl.T * K / (res["ms"] / 1e3)
+    e2e_value = world * wl.T * res["e2e_steps"] / (res["e2e_ms"] / 1e3)
+    alg = algorithmic(wl, res["counts"])
+    st = dict(zip(("router", "group_quant", "gate_up", "requant", "down", "combine"), res["stage_ms"].tolist()))
+    # dominant kernel: the gate_up GEMM (largest share of every step)
+    prefill_like = wl.T * wl.k >= 4096
+    gu_s = st["gate_up"] / 1e3
+    if prefill_like:
+        int8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        achieved = alg["gate_up_ops"] / gu_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+                "frac": achieved / int8_peak, "traffic": None,
+                "kernel": "gate_up grouped INT8 GEMM (tcgen05 kind::i8)",
+                "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8:bf16 ratio)"}
+    else:
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        achieved = alg["gate_up_bytes"] / gu_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": None, "kernel": "gate_up grouped INT8 GEMM (tcgen05 kind::i8)",
+                "peak_source": f"{peak_kind} HBM copy GB/s"}
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+                   "tokens_per_step_per_gpu": wl.T, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: each step streams the touched experts' int8 weights"},
+        "roofline": roof,
+        "layer": {"tops": alg["ops"] / (ms_step / 1e3) / 1e12, "gbs": alg["bytes"] / (ms_step / 1e3) / 1e9,
+                  "hbm_frac": alg["bytes"] / (ms_step / 1e3) / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
+                  "alg_bytes": alg["bytes"], "alg_ops": alg["ops"], "touched_experts": alg["touched"]},
+        "stage_ms": st,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": 6 * K,
+        "clocks": res["clocks"],
+    }
+    if not args.no_cpu_baseline:
+        rate, reps, el = cpu_oracle_rate(wl, sample)
+        out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"{sample} tokens of the workload per oracle forward, {reps} forwards "
+                                         f"in {el:.1f} s"}
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,182 @@
+/*
+ * w8a8.h - C ABI of libw8a8, the W8A8 INT8 MoE expert-FFN forward for NVIDIA B200 (sm_100a).
+ *
+ * Method (sources are the pages' titles and sections):
+ *   - "Qwen3-30B-A3B-Instruct-2507-quantized.w8a8" explainer, section 二: weights int8 per
+ *     output channel, symmetric min-max, static; activations int8 per token, dynamic.
+ *     Section 三 3.1: mlp.gate maps the hidden state to one score per expert, softmax, top-8;
+ *     the gate is never quantized (ignore list entry re:.*mlp.gate$).
+ *   - "Qwen3.6-35B-A3B-w8a8量化配置深度解读：config.json与recipe.yaml关键参数解析",
+ *     block config_groups.group_0: the same scheme as explicit fields.
+ *   - "Qwen3-1.7B-W4A8-V1" explainer, section "4bit 权重": int4 two's-complement packed
+ *     weights with one scale per group of 128 along K; section "8bit 激活": dynamic
+ *     per-token int8 activations.
+ *   - "Qwen3-235B-A22B-quantized.w8a8" explainer, model table and shard contents: 128
+ *     experts, 8 per token, gate_proj/up_proj/down_proj in INT8, mlp.gate in bf16.
+ *   - "Qwen3-Next-80B-A3B-Instruct 在 AMCT 中的 MoE 混合注意力量化适配实战", section 二 2.2:
+ *     gate_proj and up_proj of an expert concatenated along the output dimension into
+ *     gate_up_proj; down_proj kept separate.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device memory owned by the caller unless stated otherwise; the library
+ *     never allocates, frees or retains them. bf16 tensors are passed as their raw 16-bit
+ *     patterns (w8a8_bf16). All tensors are row-major and contiguous.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) on the current CUDA device. Calls on different streams are safe when each uses
+ *     its own outputs and workspace.
+ *   - The return value is a status code (W8A8_OK or a negative W8A8_ERR_*). Argument and
+ *     shape checks happen on the host before anything is enqueued; a rejected call enqueues
+ *     nothing. Faults found on the device (a wait that ran out, an out-of-range expert id)
+ *     set a device error word that w8a8_check_status() reports.
+ *   - Shape rules: hidden sizes and reduction lengths are multiples of 128 (the TMA/MMA
+ *     K-block), the expert intermediate size I a multiple of 64, E <= 256, 1 <= k <= 16.
+ */
+#ifndef W8A8_H_
+#define W8A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t w8a8_bf16; /* raw bfloat16 bits */
+typedef void* w8a8_stream;  /* cudaStream_t */
+
+#define W8A8_OK 0
+#define W8A8_ERR_ARG (-1)         /* null pointer, negative or inconsistent size */
+#define W8A8_ERR_UNSUPPORTED (-2) /* shape or alignment outside the supported set */
+#define W8A8_ERR_WORKSPACE (-3)   /* workspace smaller than the size query returned */
+#define W8A8_ERR_LAUNCH (-4)      /* a CUDA call or kernel launch failed */
+#define W8A8_ERR_DEVICE (-5)      /* the device error word was set (see w8a8_check_status) */
+
+#define W8A8_W_INT8_PER_CHANNEL 0 /* w: int8 [N, K], sw: fp32 [N] */
+#define W8A8_W_INT4_PER_GROUP 1   /* w: uint8 [N, K/2] packed int4, sw: fp32 [N, K/group] */
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int w8a8_version(void);
+
+/* Static English text for a status code. */
+const char* w8a8_status_string(int status);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current device.
+ * Returns W8A8_ERR_DEVICE if any kernel since the last check reported a fault, W8A8_ERR_LAUNCH
+ * if the stream itself reports a CUDA error, else W8A8_OK. */
+int w8a8_check_status(w8a8_stream stream);
+
+/* Static per-output-channel int8 weight quantisation (offline weight preparation).
+ *   w      bf16 [G, N, K]   G blocks (experts) of nn.Linear weights [out = N, in = K]
+ *   q      int8 [G, N, K]   codes clamp(rne(w / scale), -127, 127)
+ *   scale  fp32 [G, N]      max |w[g, n, :]| / 127 (0 for an all-zero row)
+ * K must be a multiple of 8. */
+int w8a8_quantize_weight_per_channel(const w8a8_bf16* w, int64_t G, int64_t N, int64_t K, int8_t* q,
+                                     float* scale, w8a8_stream stream);
+
+/* Symmetric int4 weight quantisation with one scale per `group` consecutive K values.
+ *   w       bf16 [N, K]
+ *   packed  uint8 [N, K/2]   byte i = code(2i) & 0xF | (code(2i+1) & 0xF) << 4, codes in [-7, 7]
+ *   scale   fp32 [N, K/group] max |w| over the group / 7
+ * group must be 128 and K a multiple of it. */
+int w8a8_quantize_weight_int4_per_group(const w8a8_bf16* w, int64_t N, int64_t K, int group, uint8_t* packed,
+                                        float* scale, w8a8_stream stream);
+
+/* Dynamic per-token symmetric int8 activation quantisation.
+ *   x      bf16 [T, K]
+ *   q      int8 [T, K]   clamp(rne(x / scale), -127, 127)
+ *   scale  fp32 [T]      max |x[t, :]| / 127 (0 for an all-zero token)
+ * K must be a multiple of 8. T = 0 is a no-op. */
+int w8a8_quant_act_per_token(const w8a8_bf16* x, int64_t T, int64_t K, int8_t* q, float* scale,
+                             w8a8_stream stream);
+
+/* BF16 router (never quantised): logits = x . wg^T (+ bias) accumulated in fp32 on the tensor
+ * cores, softmax over the E experts, top-k by descending probability (equal values: lower
+ * expert first), weights renormalised over the k selected experts when renorm != 0.
+ *   x              bf16 [T, H]
+ *   wg             bf16 [E, H]   (nn.Linear layout)
+ *   bias           fp32 [E] or NULL (added to the logits; for routing stress tests)
+ *   topk_ids       int32 [T, k]  slot j = j-th most probable expert
+ *   topk_w         fp32 [T, k]
+ *   expert_counts  int32 [E] or NULL: number of tokens routed to each expert
+ * H % 128 == 0, 1 <= E <= 256, 1 <= k <= min(16, E). */
+int w8a8_moe_route(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
+                   int k, int renorm, int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
+                   w8a8_stream stream);
+
+/* Byte offsets of the intermediates that w8a8_moe_forward leaves in its workspace (every
+ * region 256-byte aligned). Rows are "sorted rows": the T*k assignments grouped by expert,
+ * ordered by token inside an expert; A_pad = T*k rounded up to a multiple of 128.
+ *   topk_ids int32 [T, k]; topk_w fp32 [T, k]; tile_counts int32 [ceil(T/128), E];
+ *   offsets int32 [E+1] (rows of expert e: offsets[e] .. offsets[e+1]-1);
+ *   perm int32 [T*k] (sorted row -> assignment t*k + j); sx fp32 [T] (token scales);
+ *   sx_sorted fp32 [A_pad]; xq int8 [A_pad, H] (token codes in sorted-row order);
+ *   h bf16 [A_pad, I] (SiLU(gate)*up); s_h fp32 [A_pad]; hq int8 [A_pad, I];
+ *   o bf16 [T*k, H] (expert outputs in slot order t*k + j). */
+typedef struct {
+  size_t topk_ids, topk_w, tile_counts, offsets, perm, sx, sx_sorted, xq, h, s_h, hq, o;
+  size_t total;
+} w8a8_moe_ws_layout;
+
+/* Fills *layout for the given shape. Returns W8A8_ERR_ARG / W8A8_ERR_UNSUPPORTED on bad
+ * shapes. */
+int w8a8_moe_workspace_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_layout* layout);
+
+/* Workspace bytes w8a8_moe_forward needs for this shape (0 if the shape is rejected). */
+size_t w8a8_moe_workspace_size(int64_t T, int64_t H, int64_t E, int k, int64_t I);
+
+/* W8A8 MoE expert-FFN forward of one Qwen3-MoE layer:
+ *   route (bf16) -> per-token int8 x -> grouped int8 gate_up GEMM (int32) -> dequant
+ *   ((acc * s_x) * s_gu), SiLU(gate) * up -> bf16 h -> per-row int8 requantisation of h ->
+ *   grouped int8 down GEMM -> dequant ((acc * s_h) * s_d) -> bf16 o -> y[t] = bf16(sum_j
+ *   w[t,j] * o[t,j]) (fp32 products and sums in slot order).
+ *   x     bf16 [T, H];  wg bf16 [E, H];  bias fp32 [E] or NULL
+ *   wgu   int8 [E, 2I, H]  packed gate_up: rows 0..I-1 gate_proj, rows I..2I-1 up_proj
+ *   s_gu  fp32 [E, 2I]     per-channel scales of wgu
+ *   wd    int8 [E, H, I];  s_d fp32 [E, H]
+ *   workspace  device buffer of at least w8a8_moe_workspace_size() bytes, 256-byte aligned;
+ *              it keeps the intermediates listed in w8a8_moe_ws_layout after the call.
+ *   y     bf16 [T, H]
+ * H % 128 == 0, I % 128 == 0, E <= 256, 1 <= k <= min(16, E). T = 0 is a no-op. */
+int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                     const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E,
+                     int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
+                     w8a8_stream stream);
+
+/* w8a8_moe_forward that also records caller-created CUDA events (cudaEvent_t, may be NULL
+ * entries) on `stream` at the stage boundaries, for per-kernel timing:
+ *   [0] before the router, [1] before grouping + quantisation, [2] before the gate_up GEMM,
+ *   [3] before the requantisation of h, [4] before the down GEMM, [5] before the combine,
+ *   [6] after the combine. stage_events must point to 7 entries. */
+int w8a8_moe_forward_profiled(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                              const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H,
+                              int64_t E, int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes,
+                              w8a8_bf16* y, w8a8_stream stream, void* const* stage_events);
+
+/* Workspace bytes w8a8_linear needs (0 if the shape is rejected). */
+size_t w8a8_linear_workspace_size(int64_t M, int64_t K, int64_t N, int w_format, int group);
+
+/* Dense W8A8 / W4A8 linear: y = x . W^T with per-token dynamic int8 x.
+ *   W8A8_W_INT8_PER_CHANNEL: w int8 [N, K], sw fp32 [N]; y = bf16(((float)acc * s_x) * sw[n]).
+ *   W8A8_W_INT4_PER_GROUP:   w uint8 [N, K/2] (packing as above), sw fp32 [N, K/group];
+ *     y = bf16(acc_f * s_x) with acc_f = sum over groups g in order of (float)acc_g * sw[n, g],
+ *     acc_g the int32 sum of group g (fp32 products and sums).
+ *   x bf16 [M, K]; workspace of w8a8_linear_workspace_size() bytes; y bf16 [M, N].
+ * K % 128 == 0, N % 128 == 0, group == 128 for the int4 format. */
+int w8a8_linear(const w8a8_bf16* x, const void* w, const float* sw, int w_format, int group, int64_t M,
+                int64_t K, int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream);
+
+/* Exact integer GEMM on the tensor cores: c[m, n] = sum_k a[m, k] * b[n, k] in int32.
+ *   a int8 [M, K], b int8 [N, K], c int32 [M, N];  K % 128 == 0, N % 128 == 0. */
+int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
+                      w8a8_stream stream);
+
+/* Test hook for the bounded waits: launches one CTA that waits on an mbarrier phase nothing
+ * completes; after `timeout_ns` the wait gives up and sets the device error word, which the
+ * next w8a8_check_status() reports as W8A8_ERR_DEVICE. The context stays usable. */
+int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W8A8_H_ */

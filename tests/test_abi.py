@@ -1,0 +1,86 @@
+"""The C ABI library loads and exports every entry point include/w8a8.h declares (CPU only:
+no kernel is launched here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from w8a8_int8_quantized_act_b200 import binding as B
+from w8a8_int8_quantized_act_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w8a8.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(w8a8_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    try:
+        build_mod.build()
+    except RuntimeError as e:  # pragma: no cover
+        pytest.skip(f"cannot build: {e}")
+    return B.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(B.SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.w8a8_version() == 100
+    for st in range(-5, 1):
+        assert B.status_string(st) not in ("", "unknown status")
+
+
+def test_workspace_queries_are_host_only(lib):
+    assert B.w8a8_moe_workspace_size(64, 2048, 128, 8, 768) > 64 * 8 * 2048
+    L = B.w8a8_moe_workspace_layout(64, 2048, 128, 8, 768)
+    offs = [L[k] for k in ("topk_ids", "topk_w", "tile_counts", "offsets", "perm", "sx", "sx_sorted", "xq",
+                           "h", "s_h", "hq", "o")]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and L["total"] > offs[-1]
+    assert L["o"] + 64 * 8 * 2048 * 2 <= L["total"]
+    # rejected shapes report size 0
+    assert B.w8a8_moe_workspace_size(64, 2000, 128, 8, 768) == 0  # H % 128
+    assert B.w8a8_moe_workspace_size(64, 2048, 300, 8, 768) == 0  # E > 256
+    assert B.w8a8_moe_workspace_size(64, 2048, 128, 17, 768) == 0  # k > 16
+    assert B.w8a8_moe_workspace_size(64, 2048, 4, 8, 768) == 0  # k > E
+    assert B.w8a8_linear_workspace_size(2048, 2048, 6144, 1, 64) == 0  # group != 128
+    assert B.w8a8_linear_workspace_size(2048, 2048, 6144, 1, 128) > 0
+
+
+def test_argument_checks_reject_before_any_launch(lib):
+    c = ctypes.c_void_p
+    # negative sizes, null pointers, unsupported shapes: all rejected on the host
+    assert lib.w8a8_quant_act_per_token(None, -1, 128, None, None, None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_quant_act_per_token(c(16), 4, 7, c(16), c(16), None) == B.W8A8_ERR_UNSUPPORTED
+    assert lib.w8a8_quant_act_per_token(None, 4, 128, None, None, None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_quant_act_per_token(None, 0, 128, None, None, None) == B.W8A8_OK  # empty
+    assert lib.w8a8_moe_forward(None, None, None, None, None, None, None, 8, 2048, 128, 8, 768, 1, None, 0, None,
+                                None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_moe_forward(None, None, None, None, None, None, None, 0, 2048, 128, 8, 768, 1, None, 0, None,
+                                None) == B.W8A8_OK  # T = 0 is a no-op
+    assert lib.w8a8_moe_forward(c(256), c(256), None, c(256), c(256), c(256), c(256), 8, 2048, 128, 8, 768, 1,
+                                c(256), 10, c(256), None) == B.W8A8_ERR_WORKSPACE
+    assert lib.w8a8_moe_route(None, None, None, 4, 2048, 128, 9, 1, None, None, None, None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_quantize_weight_int4_per_group(None, 4, 256, 64, None, None, None) == B.W8A8_ERR_UNSUPPORTED
+    assert lib.w8a8_gemm_s8s8s32(None, None, None, 4, 100, 128, None) == B.W8A8_ERR_UNSUPPORTED
+    assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
+
+
+def test_package_has_no_oracle_dependency():
+    pkg = os.path.join(ROOT, "w8a8_int8_quantized_act_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", src, re.M), f

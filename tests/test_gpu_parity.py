@@ -1,0 +1,200 @@
+"""GPU parity: every stage of the CUDA path through the C ABI against the CPU oracle.
+
+Integer codes, scales, int32 accumulators, perm/offsets and the bf16 intermediates (h, o)
+and output y are compared bit for bit, the oracle being fed the GPU's routing; the routing
+itself is compared with the oracle's router (identical expert sets wherever the k-th/(k+1)-th
+probability gap exceeds 1e-4, weights within fp32 rounding); y is also checked end to end
+against the oracle's own routing (max abs <= 2e-2, relative L2 <= 5e-3).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import w8a8_oracle as O
+from w8a8_int8_quantized_act_b200 import binding as B
+from w8a8_int8_quantized_act_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from tests import gpu_common as G  # noqa: E402
+else:  # pragma: no cover
+    G = None
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    yield
+    if torch.cuda.is_available():
+        B.w8a8_check_status()
+
+
+# ------------------------------------------------------------------ exact int8 GEMM
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (128, 128, 256), (300, 384, 2048), (1000, 256, 768),
+                                   (77, 6144, 128)])
+def test_gemm_s8s8s32_exact(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    a = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    b = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    c = B.w8a8_gemm_s8s8s32(G.to_dev(a), G.to_dev(b))
+    np.testing.assert_array_equal(c.cpu().numpy(), O.int_gemm(a, b))
+
+
+def test_gemm_s8s8s32_extremes():
+    K = 4096
+    a = np.full((130, K), -127, np.int8)
+    b = np.full((128, K), -127, np.int8)
+    b[::2] = 127
+    c = B.w8a8_gemm_s8s8s32(G.to_dev(a), G.to_dev(b)).cpu().numpy()
+    np.testing.assert_array_equal(c, O.int_gemm(a, b))
+
+
+# ------------------------------------------------------------------ quantisers
+@pytest.mark.parametrize("T,K", [(1, 128), (64, 256), (64, 2048), (300, 2048), (129, 4096), (8192, 2048)])
+def test_quant_act_per_token_exact(T, K):
+    x = synth.activations(T, K, max(1, K // 100), seed=T)
+    x[min(3, T - 1)] = 0  # an all-zero token
+    q, s = B.w8a8_quant_act_per_token(G.bf16_dev(x))
+    oq, os_ = O.quant_act_per_token(x)
+    np.testing.assert_array_equal(q.cpu().numpy(), oq)
+    np.testing.assert_array_equal(s.cpu().numpy(), os_)
+
+
+def test_quant_act_rounding_ties():
+    # rows with amax 127: v/scale lands exactly on .5 for the designed entries
+    v = np.zeros((2, 128), np.float32)
+    v[:, 0] = 127
+    v[0, 1:9] = [0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5, -126.5]
+    v[1, 1:3] = [3.5, -3.5]
+    x = O.f32_to_bf16(v)
+    q, s = B.w8a8_quant_act_per_token(G.bf16_dev(x))
+    np.testing.assert_array_equal(q.cpu().numpy(), O.quant_act_per_token(x)[0])
+    assert q.cpu().numpy()[0, 1:9].tolist() == [0, 2, 2, 0, -2, -2, 126, -126]
+
+
+def test_quant_act_empty():
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    q, s = B.w8a8_quant_act_per_token(x)
+    assert q.shape == (0, 256) and s.shape == (0,)
+
+
+@pytest.mark.parametrize("G_,N,K", [(1, 4, 128), (8, 256, 128), (3, 1536, 2048), (2, 2048, 768)])
+def test_quantize_weight_per_channel_exact(G_, N, K):
+    w = synth.expert_gate_up(G_, N // 2, K, seed=K) if N % 2 == 0 else None
+    w[0, 1] = 0  # an all-zero channel
+    q, s = B.w8a8_quantize_weight_per_channel(G.bf16_dev(w))
+    oq, os_ = O.quantize_weight_per_channel(w)
+    np.testing.assert_array_equal(q.cpu().numpy(), oq)
+    np.testing.assert_array_equal(s.cpu().numpy(), os_)
+
+
+@pytest.mark.parametrize("N,K", [(4, 128), (6144, 2048), (130, 1024)])
+def test_quantize_int4_exact(N, K):
+    w = synth.dense_weight(N, K, seed=N)
+    p, s = B.w8a8_quantize_weight_int4_per_group(G.bf16_dev(w), 128)
+    op, os_ = O.quantize_weight_int4_per_group(w, 128)
+    np.testing.assert_array_equal(p.cpu().numpy(), op)
+    np.testing.assert_array_equal(s.cpu().numpy(), os_)
+
+
+# ------------------------------------------------------------------ router
+@pytest.mark.parametrize("T,H,E,k,renorm,skew", [
+    (64, 256, 8, 2, True, False), (64, 2048, 128, 8, True, False), (1, 2048, 128, 8, True, False),
+    (300, 1024, 100, 6, False, False), (8192, 2048, 128, 8, True, True), (129, 4096, 128, 8, True, False),
+    (50, 512, 16, 16, True, False), (40, 256, 256, 4, False, False), (33, 128, 1, 1, True, False)])
+def test_route(T, H, E, k, renorm, skew):
+    x = synth.activations(T, H, max(1, H // 100), seed=T)
+    wg = synth.router_weight(E, H, seed=E)
+    bias = synth.router_bias(E, 0, n_hot=min(8, E)) if skew else None
+    ids, w, counts = B.w8a8_moe_route(G.bf16_dev(x), G.bf16_dev(wg), k, renorm,
+                                      bias=G.to_dev(bias) if bias is not None else None)
+    ids, w, counts = ids.cpu().numpy(), w.cpu().numpy(), counts.cpu().numpy()
+    r = O.route(x, wg, bias, k, renorm)
+    clear = r.gap > 1e-4
+    np.testing.assert_array_equal(np.sort(ids[clear], 1), np.sort(r.ids[clear], 1))
+    same = np.all(ids == r.ids, axis=1)
+    assert same.mean() > 0.9
+    np.testing.assert_allclose(w[same], r.weights[same], rtol=2e-4, atol=2e-6)
+    np.testing.assert_array_equal(counts, np.bincount(ids.reshape(-1), minlength=E))
+    assert all(len(set(row)) == k for row in ids.tolist())
+
+
+# ------------------------------------------------------------------ whole layer
+def _full_check(run):
+    wl = run.wl
+    m = run.mid
+    G.check_grouping(m["topk_ids"], m["perm"], m["offsets"], wl.E)
+    tokens = np.arange(run.inp.x.shape[0])
+    G.compare_tokens(run, tokens)
+    clear = G.check_routing(run, m["topk_ids"], m["topk_w"])
+    G.y_tolerance_check(run, tokens, clear)
+
+
+def test_moe_tiny_all_stages():
+    _full_check(G.run_moe(synth.MOE_WORKLOADS["tiny"]))
+
+
+def test_moe_decode_all_tokens():
+    _full_check(G.run_moe(synth.MOE_WORKLOADS["qwen3-30b-a3b-decode"]))
+
+
+@pytest.mark.parametrize("T,E,k,I", [(1, 8, 2, 128), (129, 8, 2, 128), (37, 8, 8, 128), (200, 1, 1, 256),
+                                     (70, 16, 4, 384)])
+def test_moe_edge_shapes(T, E, k, I):
+    wl = synth.MoEWorkload("edge", T=T, H=256, E=E, k=k, I=I, n_outlier=2, seed=T)
+    _full_check(G.run_moe(wl))
+
+
+def test_moe_zero_tokens_and_empty_experts():
+    wl = synth.MoEWorkload("empty-experts", T=100, H=256, E=16, k=2, I=128, n_outlier=2)
+    bias = np.zeros(16, np.float32)
+    bias[[2, 9, 11]] = 40.0  # every token picks two of three experts: 13 experts stay empty
+    run = G.run_moe(wl, bias_override=bias)
+    assert (np.diff(run.mid["offsets"]) == 0).sum() == 13
+    _full_check(run)
+    x0 = np.zeros_like(run.inp.x)
+    run0 = G.run_moe(wl, x_override=x0)
+    assert not O.bf16_to_f32(run0.y).any()
+    e = synth.MoEWorkload("empty", T=0, H=256, E=8, k=2, I=128, n_outlier=0)
+    run_e = G.run_moe(e)
+    assert run_e.y.shape == (0, 256)
+
+
+@pytest.mark.parametrize("name", ["qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed", "qwen3-235b-a22b"])
+def test_moe_full_size_sampled_tokens(name):
+    wl = synth.MOE_WORKLOADS[name]
+    run = G.run_moe(wl)
+    m = run.mid
+    G.check_grouping(m["topk_ids"], m["perm"], m["offsets"], wl.E)
+    rng = np.random.default_rng(1)
+    tokens = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(wl.T, 14, replace=False)]))
+    G.compare_tokens(run, tokens)
+    clear = G.check_routing(run, m["topk_ids"], m["topk_w"], tokens)
+    G.y_tolerance_check(run, tokens, clear)
+    if wl.skewed:
+        counts = np.diff(m["offsets"])
+        hot = np.flatnonzero(run.inp.bias)
+        assert counts[hot].min() > 4 * np.median(counts)
+
+
+# ------------------------------------------------------------------ dense linear
+@pytest.mark.parametrize("M,K,N", [(1, 128, 128), (200, 512, 384), (2048, 2048, 6144)])
+def test_linear_w8a8_exact(M, K, N):
+    x = synth.activations(M, K, max(1, K // 100), seed=M)
+    w = synth.dense_weight(N, K, seed=N)
+    q, s = B.w8a8_quantize_weight_per_channel(G.bf16_dev(w))
+    y = B.w8a8_linear(G.bf16_dev(x), q, s, B.W8A8_W_INT8_PER_CHANNEL)
+    oq, os_ = O.quantize_weight_per_channel(w)
+    np.testing.assert_array_equal(G.host(y), O.linear_w8a8(x, oq, os_))
+
+
+# ------------------------------------------------------------------ failure detection
+def test_bounded_wait_reports_timeout_and_context_survives():
+    B.w8a8_debug_wait_timeout(2_000_000)  # 2 ms
+    with pytest.raises(B.W8A8Error) as ei:
+        B.w8a8_check_status()
+    assert ei.value.status == B.W8A8_ERR_DEVICE
+    B.w8a8_check_status()  # cleared
+    x = synth.activations(8, 256, 2)
+    q, s = B.w8a8_quant_act_per_token(G.bf16_dev(x))
+    np.testing.assert_array_equal(q.cpu().numpy(), O.quant_act_per_token(x)[0])

@@ -1,0 +1,280 @@
+"""Python binding of libw8a8 (the C ABI in include/w8a8.h).
+
+Argument marshalling only: each function takes torch CUDA tensors, allocates any output the
+caller did not pass, and calls the C entry point of the same name on the current CUDA stream.
+Every step of the computation runs in the library's kernels. If the library is missing the
+first call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw8a8.so")
+
+W8A8_OK = 0
+W8A8_ERR_ARG = -1
+W8A8_ERR_UNSUPPORTED = -2
+W8A8_ERR_WORKSPACE = -3
+W8A8_ERR_LAUNCH = -4
+W8A8_ERR_DEVICE = -5
+W8A8_W_INT8_PER_CHANNEL = 0
+W8A8_W_INT4_PER_GROUP = 1
+
+_c_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_size = ctypes.c_size_t
+
+
+class W8A8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+        self.status = status
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("topk_ids", "topk_w", "tile_counts", "offsets", "perm", "sx", "sx_sorted", "xq", "h",
+                 "s_h", "hq", "o", "total")]
+
+
+# (name, restype, argtypes) of every exported entry point
+SIGNATURES = {
+    "w8a8_version": (_int, []),
+    "w8a8_status_string": (ctypes.c_char_p, [_int]),
+    "w8a8_check_status": (_int, [_c_p]),
+    "w8a8_quantize_weight_per_channel": (_int, [_c_p, _i64, _i64, _i64, _c_p, _c_p, _c_p]),
+    "w8a8_quantize_weight_int4_per_group": (_int, [_c_p, _i64, _i64, _int, _c_p, _c_p, _c_p]),
+    "w8a8_quant_act_per_token": (_int, [_c_p, _i64, _i64, _c_p, _c_p, _c_p]),
+    "w8a8_moe_route": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _int, _c_p, _c_p, _c_p, _c_p]),
+    "w8a8_moe_workspace_layout": (_int, [_i64, _i64, _i64, _int, _i64, ctypes.POINTER(_Layout)]),
+    "w8a8_moe_workspace_size": (_size, [_i64, _i64, _i64, _int, _i64]),
+    "w8a8_moe_forward": (_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _i64, _int,
+                                _c_p, _size, _c_p, _c_p]),
+    "w8a8_moe_forward_profiled": (_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _i64,
+                                         _int, _c_p, _size, _c_p, _c_p, ctypes.POINTER(_c_p)]),
+    "w8a8_linear_workspace_size": (_size, [_i64, _i64, _i64, _int, _int]),
+    "w8a8_linear": (_int, [_c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _size, _c_p, _c_p]),
+    "w8a8_gemm_s8s8s32": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p]),
+    "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libw8a8.so (built in-tree by build.py); raises if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libw8a8.so not found at {LIB_PATH}; run w8a8_int8_quantized_act_b200/build.py")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().w8a8_status_string(status).decode()
+    except Exception:  # pragma: no cover - library missing
+        return "?"
+
+
+def _check(rc: int, where: str):
+    if rc != W8A8_OK:
+        raise W8A8Error(rc, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _bf16(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected a bfloat16 tensor")
+    return t
+
+
+def w8a8_version() -> int:
+    return lib().w8a8_version()
+
+
+def w8a8_check_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status; raises on error."""
+    rc = lib().w8a8_check_status(_stream(stream))
+    _check(rc, "w8a8_check_status")
+    return rc
+
+
+def w8a8_quantize_weight_per_channel(w: torch.Tensor, q=None, scale=None, stream=None):
+    """w bf16 [..., N, K] -> (q int8 [..., N, K], scale fp32 [..., N])."""
+    _bf16(w)
+    *lead, N, K = w.shape
+    G = 1
+    for d in lead:
+        G *= d
+    q = torch.empty(w.shape, dtype=torch.int8, device=w.device) if q is None else q
+    scale = torch.empty((*lead, N), dtype=torch.float32, device=w.device) if scale is None else scale
+    _check(lib().w8a8_quantize_weight_per_channel(_ptr(w), G, N, K, _ptr(q), _ptr(scale), _stream(stream)),
+           "w8a8_quantize_weight_per_channel")
+    return q, scale
+
+
+def w8a8_quantize_weight_int4_per_group(w: torch.Tensor, group: int = 128, packed=None, scale=None, stream=None):
+    """w bf16 [N, K] -> (packed uint8 [N, K/2], scale fp32 [N, K/group])."""
+    _bf16(w)
+    N, K = w.shape
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device) if packed is None else packed
+    scale = torch.empty((N, K // group), dtype=torch.float32, device=w.device) if scale is None else scale
+    _check(lib().w8a8_quantize_weight_int4_per_group(_ptr(w), N, K, group, _ptr(packed), _ptr(scale),
+                                                     _stream(stream)),
+           "w8a8_quantize_weight_int4_per_group")
+    return packed, scale
+
+
+def w8a8_quant_act_per_token(x: torch.Tensor, q=None, scale=None, stream=None):
+    """x bf16 [T, K] -> (q int8 [T, K], scale fp32 [T])."""
+    _bf16(x)
+    T, K = x.shape
+    q = torch.empty((T, K), dtype=torch.int8, device=x.device) if q is None else q
+    scale = torch.empty((T,), dtype=torch.float32, device=x.device) if scale is None else scale
+    _check(lib().w8a8_quant_act_per_token(_ptr(x), T, K, _ptr(q), _ptr(scale), _stream(stream)),
+           "w8a8_quant_act_per_token")
+    return q, scale
+
+
+def w8a8_moe_route(x: torch.Tensor, wg: torch.Tensor, k: int, renorm: bool = True, bias=None,
+                   topk_ids=None, topk_w=None, expert_counts=None, stream=None):
+    """Router: (topk_ids int32 [T, k], topk_w fp32 [T, k], expert_counts int32 [E])."""
+    _bf16(x), _bf16(wg)
+    T, H = x.shape
+    E = wg.shape[0]
+    dev = x.device
+    topk_ids = torch.empty((T, k), dtype=torch.int32, device=dev) if topk_ids is None else topk_ids
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    expert_counts = torch.empty((E,), dtype=torch.int32, device=dev) if expert_counts is None else expert_counts
+    _check(lib().w8a8_moe_route(_ptr(x), _ptr(wg), _ptr(bias), T, H, E, k, int(renorm), _ptr(topk_ids),
+                                _ptr(topk_w), _ptr(expert_counts), _stream(stream)), "w8a8_moe_route")
+    return topk_ids, topk_w, expert_counts
+
+
+def w8a8_moe_workspace_layout(T: int, H: int, E: int, k: int, I: int) -> dict:
+    L = _Layout()
+    _check(lib().w8a8_moe_workspace_layout(T, H, E, k, I, ctypes.byref(L)), "w8a8_moe_workspace_layout")
+    return {name: getattr(L, name) for name, _ in _Layout._fields_}
+
+
+def w8a8_moe_workspace_size(T: int, H: int, E: int, k: int, I: int) -> int:
+    return lib().w8a8_moe_workspace_size(T, H, E, k, I)
+
+
+def w8a8_moe_forward(x, wg, wgu, s_gu, wd, s_d, k: int, renorm: bool = True, bias=None, workspace=None,
+                     y=None, stream=None):
+    """W8A8 MoE expert-FFN forward; returns y bf16 [T, H] (workspace keeps the intermediates)."""
+    _bf16(x), _bf16(wg)
+    T, H = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    ws_bytes = w8a8_moe_workspace_size(T, H, E, k, I)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(lib().w8a8_moe_forward(_ptr(x), _ptr(wg), _ptr(bias), _ptr(wgu), _ptr(s_gu), _ptr(wd), _ptr(s_d),
+                                  T, H, E, k, I, int(renorm), _ptr(workspace), workspace.numel(), _ptr(y),
+                                  _stream(stream)), "w8a8_moe_forward")
+    return y
+
+
+MOE_STAGES = ("router", "group_quant", "gate_up", "requant", "down", "combine")
+
+
+def w8a8_moe_forward_profiled(x, wg, wgu, s_gu, wd, s_d, k: int, events, renorm: bool = True, bias=None,
+                              workspace=None, y=None, stream=None):
+    """w8a8_moe_forward recording the 7 torch.cuda.Event objects in `events` at stage boundaries."""
+    T, H = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    if workspace is None:
+        workspace = torch.empty(max(w8a8_moe_workspace_size(T, H, E, k, I), 1), dtype=torch.uint8,
+                                device=x.device)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if y is None else y
+    arr = (_c_p * 7)(*[e.cuda_event for e in events])
+    _check(lib().w8a8_moe_forward_profiled(_ptr(x), _ptr(wg), _ptr(bias), _ptr(wgu), _ptr(s_gu), _ptr(wd),
+                                           _ptr(s_d), T, H, E, k, I, int(renorm), _ptr(workspace),
+                                           workspace.numel(), _ptr(y), _stream(stream), arr),
+           "w8a8_moe_forward_profiled")
+    return y
+
+
+def moe_intermediates(workspace: torch.Tensor, T: int, H: int, E: int, k: int, I: int) -> dict:
+    """Views of the intermediates w8a8_moe_forward leaves in its workspace."""
+    L = w8a8_moe_workspace_layout(T, H, E, k, I)
+    A = T * k
+    Ap = max(1, -(-A // 128)) * 128 if A else 128
+    C = -(-T // 128)
+
+    def view(name, dtype, shape):
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return workspace[L[name]:L[name] + nbytes].view(dtype).view(*shape)
+
+    return dict(
+        topk_ids=view("topk_ids", torch.int32, (T, k)), topk_w=view("topk_w", torch.float32, (T, k)),
+        tile_counts=view("tile_counts", torch.int32, (C, E)), offsets=view("offsets", torch.int32, (E + 1,)),
+        perm=view("perm", torch.int32, (A,)), sx=view("sx", torch.float32, (T,)),
+        sx_sorted=view("sx_sorted", torch.float32, (Ap,)), xq=view("xq", torch.int8, (Ap, H)),
+        h=view("h", torch.bfloat16, (Ap, I)), s_h=view("s_h", torch.float32, (Ap,)),
+        hq=view("hq", torch.int8, (Ap, I)), o=view("o", torch.bfloat16, (A, H)))
+
+
+def w8a8_linear_workspace_size(M: int, K: int, N: int, w_format: int, group: int = 128) -> int:
+    return lib().w8a8_linear_workspace_size(M, K, N, w_format, group)
+
+
+def w8a8_linear(x, w, sw, w_format: int = W8A8_W_INT8_PER_CHANNEL, group: int = 128, workspace=None, y=None,
+                stream=None):
+    """Dense W8A8 / W4A8 linear: y bf16 [M, N] = x [M, K] . W^T."""
+    _bf16(x)
+    M, K = x.shape
+    N = w.shape[0]
+    ws_bytes = w8a8_linear_workspace_size(M, K, N, w_format, group)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(lib().w8a8_linear(_ptr(x), _ptr(w), _ptr(sw), w_format, group, M, K, N, _ptr(workspace),
+                             workspace.numel(), _ptr(y), _stream(stream)), "w8a8_linear")
+    return y
+
+
+def w8a8_gemm_s8s8s32(a, b, c=None, stream=None):
+    """Exact int8 GEMM on the tensor cores: c int32 [M, N] = a [M, K] . b [N, K]^T."""
+    M, K = a.shape
+    N = b.shape[0]
+    c = torch.empty((M, N), dtype=torch.int32, device=a.device) if c is None else c
+    _check(lib().w8a8_gemm_s8s8s32(_ptr(a), _ptr(b), _ptr(c), M, N, K, _stream(stream)), "w8a8_gemm_s8s8s32")
+    return c
+
+
+def w8a8_debug_wait_timeout(timeout_ns: int, stream=None):
+    _check(lib().w8a8_debug_wait_timeout(timeout_ns, _stream(stream)), "w8a8_debug_wait_timeout")

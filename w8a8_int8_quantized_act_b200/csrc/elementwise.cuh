@@ -1,0 +1,198 @@
+// Memory-bound kernels of the path: per-row symmetric quantisation (activations per token,
+// weights per output channel, h per assignment row), the int4 per-group weight packer, the
+// grouping of assignments by expert fused with the activation quantisation, and the
+// scatter-free weighted combine. All use 16-byte vector loads and one warp per row.
+#pragma once
+#include "numerics.cuh"
+
+namespace w8a8 {
+
+constexpr int kRowWarps = 8;  // warps per CTA for one-warp-per-row kernels
+
+// q[r, :] = codes of src[r, :], scale[r] = amax / 127, for rows r < R (row length K).
+__global__ void __launch_bounds__(kRowWarps * 32) quant_rows_kernel(const uint16_t* __restrict__ src,
+                                                                    int64_t R, int K, int8_t* __restrict__ q,
+                                                                    float* __restrict__ scale) {
+  const int64_t r = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (r >= R) return;
+  int8_t* dst = q + r * K;
+  const float s = quant_row_warp(src + r * K, K, [&](int i, uint2 v) {
+    *reinterpret_cast<uint2*>(dst + i) = v;
+  });
+  if ((threadIdx.x & 31) == 0) scale[r] = s;
+}
+
+// Symmetric int4 per group of 128 along K: one warp per (row, group), 4 values per lane.
+// Byte i of a row holds code 2i (low nibble) and code 2i+1 (high nibble).
+__global__ void __launch_bounds__(kRowWarps * 32) quant_int4_group128_kernel(
+    const uint16_t* __restrict__ w, int64_t N, int K, uint8_t* __restrict__ packed, float* __restrict__ scale) {
+  const int groups = K / 128;
+  const int64_t item = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (item >= N * groups) return;
+  const int64_t n = item / groups;
+  const int g = int(item - n * groups);
+  const int lane = threadIdx.x & 31;
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(w + n * K + g * 128 + lane * 4));
+  const float f[4] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y)};
+  float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+  amax = warp_max(amax);
+  const float s = sym_scale(amax, kQMaxInt4);
+  uint32_t nib[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) nib[j] = uint32_t(sym_code(f[j], s, 7)) & 0xFu;
+  const uint16_t bytes = uint16_t((nib[0] | (nib[1] << 4)) | ((nib[2] | (nib[3] << 4)) << 8));
+  *reinterpret_cast<uint16_t*>(packed + n * (K / 2) + g * 64 + lane * 2) = bytes;
+  if (lane == 0) scale[n * groups + g] = s;
+}
+
+// Groups the T*k assignments by expert (stable by token) and quantises each token once,
+// writing its codes to every sorted row that it feeds.
+//   tile_counts [C, E]: assignments per (128-token chunk, expert) (from the router)
+//   offsets [E+1], perm [A] (sorted row -> t*k + j), sx [T], sx_sorted [A], xq_sorted [A, H]
+// One CTA per 128-token chunk; each CTA derives its own write positions from tile_counts.
+constexpr int kPermThreads = 256;
+constexpr int kChunk = 128;
+
+__global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
+    const uint16_t* __restrict__ x, const int* __restrict__ ids, const int* __restrict__ tile_counts, int T,
+    int H, int E, int k, int* __restrict__ offsets, int* __restrict__ perm, float* __restrict__ sx,
+    float* __restrict__ sx_sorted, int8_t* __restrict__ xq_sorted) {
+  extern __shared__ int sm[];
+  int* base = sm;                 // [E]  first sorted row of this chunk's rows of expert e
+  int* run = sm + E;              // [E]  running count inside the chunk
+  int* dest = sm + 2 * E;         // [kChunk * k]
+  const int C = (T + kChunk - 1) / kChunk;
+  const int A = T * k;
+  const int chunk = blockIdx.x;
+  const int t0 = chunk * kChunk;
+  const int nt = min(kChunk, T - t0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // per-expert totals and this chunk's prefix over earlier chunks
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int total = 0, before = 0;
+    for (int c = 0; c < C; ++c) {
+      const int v = __ldg(tile_counts + size_t(c) * E + e);
+      total += v;
+      if (c < chunk) before += v;
+    }
+    base[e] = total;  // temporarily: totals
+    run[e] = before;
+  }
+  for (int i = threadIdx.x; i < kChunk * k; i += blockDim.x) dest[i] = -1;
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of totals over experts (one warp)
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = (e < E) ? base[e] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (e < E) {
+        const int excl = carry + incl - v;
+        if (chunk == 0) offsets[e] = excl;
+        base[e] = excl + run[e];
+        run[e] = 0;
+      }
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (chunk == 0 && lane == 0) offsets[E] = carry;
+  }
+  __syncthreads();
+  // stable ranks: warp 0 walks the chunk's assignments in (token, slot) order
+  if (warp == 0) {
+    const int per = 32 / k;  // tokens per step
+    for (int tl0 = 0; tl0 < nt; tl0 += per) {
+      const int tl = tl0 + lane / k;
+      const int j = lane % k;
+      const bool valid = (lane < per * k) && (tl < nt);
+      const unsigned active = __ballot_sync(0xffffffffu, valid);
+      if (valid) {
+        const int a = (t0 + tl) * k + j;
+        int e = __ldg(ids + a);
+        if (e < 0 || e >= E) {
+          atomicOr(&g_error_word, kErrBadIndex);
+          e = 0;
+        }
+        const unsigned peers = __match_any_sync(active, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int b = run[e];
+        __syncwarp(active);
+        if (rank == 0) run[e] = b + __popc(peers);
+        const int d = base[e] + b + rank;
+        if (d >= 0 && d < A) {
+          perm[d] = a;
+          dest[tl * k + j] = d;
+        } else {
+          atomicOr(&g_error_word, kErrBadIndex);  // ids inconsistent with the per-chunk counts
+        }
+      }
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // quantise each token once, write its codes to its k sorted rows
+  for (int tl = warp; tl < nt; tl += kPermThreads / 32) {
+    const int t = t0 + tl;
+    const int* drow = dest + tl * k;
+    const float s = quant_row_warp(x + size_t(t) * H, H, [&](int i, uint2 v) {
+      for (int j = 0; j < k; ++j)
+        if (drow[j] >= 0) *reinterpret_cast<uint2*>(xq_sorted + size_t(drow[j]) * H + i) = v;
+    });
+    if (lane == 0) sx[t] = s;
+    for (int j = lane; j < k; j += 32)
+      if (drow[j] >= 0) sx_sorted[drow[j]] = s;
+  }
+}
+
+// y[t, :] = bf16(sum_j w[t, j] * o[t, j, :]) with fp32 products and sums in slot order.
+// One CTA per token, 8 columns per thread, no atomics: every y element has one writer.
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ o, const float* __restrict__ w,
+                                                      int T, int H, int k, uint16_t* __restrict__ y) {
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const float wj = __ldg(w + size_t(t) * k + j);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(o + (size_t(t) * k + j) * H + c));
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, bf16_lo(u[i])));
+        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, bf16_hi(u[i])));
+      }
+    }
+    uint4 out;
+    out.x = pack_bf16(acc[0], acc[1]);
+    out.y = pack_bf16(acc[2], acc[3]);
+    out.z = pack_bf16(acc[4], acc[5]);
+    out.w = pack_bf16(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(y + size_t(t) * H + c) = out;
+  }
+}
+
+// Host-visible probe of the bounded-wait machinery: waits on an mbarrier phase that nothing
+// completes, so the wait must run out after `timeout_ns` and raise the error word.
+__global__ void wait_timeout_probe_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtx wc{&abort_flag, globaltimer_ns() + timeout_ns};
+    mbar_wait(&bar, 0, wc);
+  }
+}
+
+}  // namespace w8a8

@@ -1,0 +1,520 @@
+// libw8a8: C ABI entry points (declared in include/w8a8.h). Host code only checks arguments,
+// encodes TMA tensor maps and launches the kernels; every step of the path runs on the GPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdlib.h>
+
+#include <mutex>
+
+#include "../../include/w8a8.h"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+
+namespace w8a8 {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+cudaStream_t as_stream(w8a8_stream s) { return static_cast<cudaStream_t>(s); }
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+uint64_t wait_timeout_ns() {
+  static uint64_t ns = [] {
+    const char* env = getenv("W8A8_WAIT_TIMEOUT_MS");
+    const double ms = env ? atof(env) : 2000.0;
+    return uint64_t((ms > 0 ? ms : 2000.0) * 1e6);
+  }();
+  return ns;
+}
+
+// ------------------------------------------------------------------ TMA tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D K-major map over [rows, inner] elements with a (box_rows x 128-byte) box, 128-byte swizzle,
+// zero fill outside the tensor.
+bool make_kmajor_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint64_t rows,
+                     uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || inner == 0) return false;
+  const uint32_t esize = bf16 ? 2 : 1;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * esize};
+  const cuuint32_t box[2] = {128u / esize, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launch helpers
+int launch_status() { return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_LAUNCH; }
+
+template <int BN, int EPI, int KIND>
+int launch_gemm(const GemmParams& p, int max_tiles, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, EPI, KIND>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) !=
+      cudaSuccess)
+    return W8A8_ERR_LAUNCH;
+  const int grid = max(1, min(num_sms(), max_tiles));
+  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(p);
+  return launch_status();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+// Router column tile: the smallest supported MMA N that covers E experts.
+int router_bn(int64_t E) {
+  for (int bn : {16, 32, 64, 128, 256})
+    if (E <= bn) return bn;
+  return 0;
+}
+
+int check_moe_shape(int64_t T, int64_t H, int64_t E, int k, int64_t I) {
+  if (T < 0 || H <= 0 || E <= 0 || I <= 0 || k <= 0) return W8A8_ERR_ARG;
+  if (k > E) return W8A8_ERR_ARG;
+  if (H % 128 || I % 128 || E > 256 || k > kMaxTopK) return W8A8_ERR_UNSUPPORTED;
+  if (T * k >= (int64_t(1) << 31) / 2) return W8A8_ERR_UNSUPPORTED;
+  if (E * 2 * I >= (int64_t(1) << 31) || E * H >= (int64_t(1) << 31)) return W8A8_ERR_UNSUPPORTED;
+  return W8A8_OK;
+}
+
+void fill_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_layout* L) {
+  const int64_t A = T * k;
+  const int64_t Ap = round_up(A > 0 ? A : 1, 128);
+  const int64_t C = (T + kChunk - 1) / kChunk;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L->topk_ids = take(sizeof(int32_t) * A);
+  L->topk_w = take(sizeof(float) * A);
+  L->tile_counts = take(sizeof(int32_t) * C * E);
+  L->offsets = take(sizeof(int32_t) * (E + 1));
+  L->perm = take(sizeof(int32_t) * A);
+  L->sx = take(sizeof(float) * T);
+  L->sx_sorted = take(sizeof(float) * Ap);
+  L->xq = take(size_t(Ap) * H);
+  L->h = take(size_t(Ap) * I * 2);
+  L->s_h = take(sizeof(float) * Ap);
+  L->hq = take(size_t(Ap) * I);
+  L->o = take(size_t(A) * H * 2);
+  L->total = off;
+}
+
+// Router: tcgen05 bf16 GEMM with the softmax / top-k epilogue. tile_counts is zeroed here.
+// counts: expert histogram rows (nullptr: none) with `count_stride` elements between the rows of
+// consecutive 128-token tiles (0: every tile adds into one row of E counters).
+int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t T, int64_t H, int64_t E, int k,
+               int renorm, int* ids, float* w, int* counts, int64_t count_stride, cudaStream_t stream) {
+  const int bn = router_bn(E);
+  GemmParams p{};
+  if (!make_kmajor_map(&p.tmA, x, true, H, T, 128) || !make_kmajor_map(&p.tmB, wg, true, H, E, bn / 2))
+    return W8A8_ERR_UNSUPPORTED;
+  const int64_t C = (T + kChunk - 1) / kChunk;
+  if (counts != nullptr) {
+    const size_t rows = count_stride ? size_t(C) : 1;
+    if (cudaMemsetAsync(counts, 0, sizeof(int) * rows * E, stream) != cudaSuccess) return W8A8_ERR_LAUNCH;
+  }
+  p.num_kb = int(H / 64);
+  p.n_tiles = 1;
+  p.num_groups = 1;
+  p.group_offsets = nullptr;
+  p.M = int(T);
+  p.b_rows_per_group = 0;
+  p.b_n_step = 0;
+  p.b_half_offset = bn / 2;
+  p.timeout_ns = wait_timeout_ns();
+  p.out = ids;
+  p.n_valid = int(E);
+  p.bias = bias;
+  p.topk = k;
+  p.renorm = renorm;
+  p.topk_w = w;
+  p.tile_counts = counts;
+  p.tile_count_stride = int(count_stride);
+  const int tiles = int(C);
+  switch (bn) {
+    case 16: return launch_gemm<16, kEpiRouter, kKindBF16>(p, tiles, stream);
+    case 32: return launch_gemm<32, kEpiRouter, kKindBF16>(p, tiles, stream);
+    case 64: return launch_gemm<64, kEpiRouter, kKindBF16>(p, tiles, stream);
+    case 128: return launch_gemm<128, kEpiRouter, kKindBF16>(p, tiles, stream);
+    default: return launch_gemm<256, kEpiRouter, kKindBF16>(p, tiles, stream);
+  }
+}
+
+// Upper bound of the number of 128-row tiles over all groups: ceil(A/128) + min(E, A).
+int max_m_tiles(int64_t A, int64_t E) { return int((A + kBM - 1) / kBM + (E < A ? E : A)); }
+
+}  // namespace
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" {
+
+int w8a8_version(void) { return kVersion; }
+
+const char* w8a8_status_string(int status) {
+  switch (status) {
+    case W8A8_OK: return "ok";
+    case W8A8_ERR_ARG: return "bad argument (null pointer or inconsistent size)";
+    case W8A8_ERR_UNSUPPORTED: return "unsupported shape or alignment";
+    case W8A8_ERR_WORKSPACE: return "workspace too small";
+    case W8A8_ERR_LAUNCH: return "CUDA launch or runtime error";
+    case W8A8_ERR_DEVICE: return "device error word set (a bounded wait ran out or an index was invalid)";
+    default: return "unknown status";
+  }
+}
+
+int w8a8_check_status(w8a8_stream stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return W8A8_ERR_LAUNCH;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return W8A8_ERR_LAUNCH;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+    return W8A8_ERR_DEVICE;
+  }
+  return W8A8_OK;
+}
+
+int w8a8_quantize_weight_per_channel(const w8a8_bf16* w, int64_t G, int64_t N, int64_t K, int8_t* q, float* scale,
+                                     w8a8_stream stream) {
+  if (G < 0 || N < 0 || K <= 0) return W8A8_ERR_ARG;
+  const int64_t R = G * N;
+  if (R == 0) return W8A8_OK;
+  if (!w || !q || !scale) return W8A8_ERR_ARG;
+  if (K % 8 || !aligned16(w) || (K % 16 && !aligned16(q)) || K > (1 << 30)) return W8A8_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(q) & 7u) return W8A8_ERR_UNSUPPORTED;
+  const int64_t blocks = (R + kRowWarps - 1) / kRowWarps;
+  quant_rows_kernel<<<unsigned(blocks), kRowWarps * 32, 0, as_stream(stream)>>>(w, R, int(K), q, scale);
+  return launch_status();
+}
+
+int w8a8_quantize_weight_int4_per_group(const w8a8_bf16* w, int64_t N, int64_t K, int group, uint8_t* packed,
+                                        float* scale, w8a8_stream stream) {
+  if (N < 0 || K <= 0 || group <= 0) return W8A8_ERR_ARG;
+  if (group != 128 || K % group) return W8A8_ERR_UNSUPPORTED;
+  if (N == 0) return W8A8_OK;
+  if (!w || !packed || !scale) return W8A8_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(w) & 7u) || (reinterpret_cast<uintptr_t>(packed) & 1u))
+    return W8A8_ERR_UNSUPPORTED;
+  const int64_t items = N * (K / group);
+  const int64_t blocks = (items + kRowWarps - 1) / kRowWarps;
+  quant_int4_group128_kernel<<<unsigned(blocks), kRowWarps * 32, 0, as_stream(stream)>>>(w, N, int(K), packed,
+                                                                                        scale);
+  return launch_status();
+}
+
+int w8a8_quant_act_per_token(const w8a8_bf16* x, int64_t T, int64_t K, int8_t* q, float* scale,
+                             w8a8_stream stream) {
+  if (T < 0 || K <= 0) return W8A8_ERR_ARG;
+  if (T == 0) return W8A8_OK;
+  if (!x || !q || !scale) return W8A8_ERR_ARG;
+  if (K % 8 || !aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7u) || K > (1 << 30))
+    return W8A8_ERR_UNSUPPORTED;
+  const int64_t blocks = (T + kRowWarps - 1) / kRowWarps;
+  quant_rows_kernel<<<unsigned(blocks), kRowWarps * 32, 0, as_stream(stream)>>>(x, T, int(K), q, scale);
+  return launch_status();
+}
+
+int w8a8_moe_route(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
+                   int k, int renorm, int32_t* topk_ids, float* topk_w, int32_t* expert_counts,
+                   w8a8_stream stream) {
+  if (T < 0 || H <= 0 || E <= 0 || k <= 0 || k > E) return W8A8_ERR_ARG;
+  if (H % 128 || E > 256 || k > kMaxTopK) return W8A8_ERR_UNSUPPORTED;
+  if (T == 0) {
+    if (expert_counts) return cudaMemsetAsync(expert_counts, 0, sizeof(int) * E, as_stream(stream)) == cudaSuccess
+                                  ? W8A8_OK : W8A8_ERR_LAUNCH;
+    return W8A8_OK;
+  }
+  if (!x || !wg || !topk_ids || !topk_w) return W8A8_ERR_ARG;
+  if (!aligned16(x) || !aligned16(wg)) return W8A8_ERR_UNSUPPORTED;
+  // every tile adds its tokens' experts into the single row expert_counts[E]
+  return run_router(x, wg, bias, T, H, E, k, renorm, topk_ids, topk_w, expert_counts, 0, as_stream(stream));
+}
+
+int w8a8_moe_workspace_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_layout* layout) {
+  if (!layout) return W8A8_ERR_ARG;
+  const int st = check_moe_shape(T, H, E, k, I);
+  if (st != W8A8_OK) return st;
+  fill_layout(T, H, E, k, I, layout);
+  return W8A8_OK;
+}
+
+size_t w8a8_moe_workspace_size(int64_t T, int64_t H, int64_t E, int k, int64_t I) {
+  w8a8_moe_ws_layout L;
+  return w8a8_moe_workspace_layout(T, H, E, k, I, &L) == W8A8_OK ? L.total : 0;
+}
+
+}  // extern "C"
+
+namespace w8a8 {
+namespace {
+
+// Records stage event `i` (if events were supplied) on the stream.
+inline void mark(void* const* events, int i, cudaStream_t s) {
+  if (events != nullptr && events[i] != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+}
+
+int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                     const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E, int k,
+                     int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
+                     w8a8_stream stream, void* const* ev) {
+  const int st = check_moe_shape(T, H, E, k, I);
+  if (st != W8A8_OK) return st;
+  if (T == 0) return W8A8_OK;
+  if (!x || !wg || !wgu || !s_gu || !wd || !s_d || !workspace || !y) return W8A8_ERR_ARG;
+  if (!aligned16(x) || !aligned16(wg) || !aligned16(wgu) || !aligned16(wd) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return W8A8_ERR_UNSUPPORTED;
+  w8a8_moe_ws_layout L;
+  fill_layout(T, H, E, k, I, &L);
+  if (workspace_bytes < L.total) return W8A8_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* ids = reinterpret_cast<int*>(ws + L.topk_ids);
+  float* w = reinterpret_cast<float*>(ws + L.topk_w);
+  int* tile_counts = reinterpret_cast<int*>(ws + L.tile_counts);
+  int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+  int* perm = reinterpret_cast<int*>(ws + L.perm);
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
+  float* sx_sorted = reinterpret_cast<float*>(ws + L.sx_sorted);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  float* s_h = reinterpret_cast<float*>(ws + L.s_h);
+  int8_t* hq = reinterpret_cast<int8_t*>(ws + L.hq);
+  uint16_t* o = reinterpret_cast<uint16_t*>(ws + L.o);
+  cudaStream_t s = as_stream(stream);
+  const int64_t A = T * k;
+  const int64_t Ap = round_up(A, 128);
+  const int C = int((T + kChunk - 1) / kChunk);
+  int rc;
+
+  // 1. router (bf16 tcgen05 GEMM + softmax / top-k epilogue, per-chunk expert histogram)
+  mark(ev, 0, s);
+  rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E, s);
+  if (rc != W8A8_OK) return rc;
+
+  // 2. group assignments by expert and quantise every token once into its sorted rows
+  const size_t gq_smem = sizeof(int) * (2 * E + kChunk * k);
+  mark(ev, 1, s);
+  group_quant_kernel<<<C, kPermThreads, gq_smem, s>>>(x, ids, tile_counts, int(T), int(H), int(E), k, offsets,
+                                                      perm, sx, sx_sorted, xq);
+  if ((rc = launch_status()) != W8A8_OK) return rc;
+
+  // 3. grouped gate_up GEMM with the dequant + SiLU(gate)*up epilogue -> h
+  const bool wide = A >= 4096;  // prefill-sized batches use 256-wide tiles
+  {
+    GemmParams p{};
+    const int bn = wide ? 256 : 128;
+    if (I % (bn / 2)) return W8A8_ERR_UNSUPPORTED;
+    if (!make_kmajor_map(&p.tmA, xq, false, H, Ap, 128) ||
+        !make_kmajor_map(&p.tmB, wgu, false, H, uint64_t(E) * 2 * I, bn / 2))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(H / 128);
+    p.n_tiles = int(I / (bn / 2));
+    p.num_groups = int(E);
+    p.group_offsets = offsets;
+    p.b_rows_per_group = int(2 * I);
+    p.b_n_step = bn / 2;
+    p.b_half_offset = int(I);
+    p.timeout_ns = wait_timeout_ns();
+    p.out = h;
+    p.ldo = int(I);
+    p.row_scale = sx_sorted;
+    p.col_scale = s_gu;
+    p.col_scale_stride = int(2 * I);
+    p.up_offset = int(I);
+    const int tiles = max_m_tiles(A, E) * p.n_tiles;
+    mark(ev, 2, s);
+    rc = wide ? launch_gemm<256, kEpiGateUp, kKindI8>(p, tiles, s) : launch_gemm<128, kEpiGateUp, kKindI8>(p, tiles, s);
+    if (rc != W8A8_OK) return rc;
+  }
+
+  // 4. per-row requantisation of h
+  {
+    const int64_t blocks = (A + kRowWarps - 1) / kRowWarps;
+    mark(ev, 3, s);
+    quant_rows_kernel<<<unsigned(blocks), kRowWarps * 32, 0, s>>>(h, A, int(I), hq, s_h);
+    if ((rc = launch_status()) != W8A8_OK) return rc;
+  }
+
+  // 5. grouped down GEMM with the dequant epilogue -> o in slot order
+  {
+    GemmParams p{};
+    const int bn = wide ? 256 : 128;
+    if (H % bn) return W8A8_ERR_UNSUPPORTED;
+    if (!make_kmajor_map(&p.tmA, hq, false, I, Ap, 128) ||
+        !make_kmajor_map(&p.tmB, wd, false, I, uint64_t(E) * H, bn / 2))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(I / 128);
+    p.n_tiles = int(H / bn);
+    p.num_groups = int(E);
+    p.group_offsets = offsets;
+    p.b_rows_per_group = int(H);
+    p.b_n_step = bn;
+    p.b_half_offset = bn / 2;
+    p.timeout_ns = wait_timeout_ns();
+    p.out = o;
+    p.ldo = int(H);
+    p.out_col_step = bn;
+    p.row_scale = s_h;
+    p.col_scale = s_d;
+    p.col_scale_stride = int(H);
+    p.row_map = perm;
+    const int tiles = max_m_tiles(A, E) * p.n_tiles;
+    mark(ev, 4, s);
+    rc = wide ? launch_gemm<256, kEpiDown, kKindI8>(p, tiles, s) : launch_gemm<128, kEpiDown, kKindI8>(p, tiles, s);
+    if (rc != W8A8_OK) return rc;
+  }
+
+  // 6. scatter-free weighted combine
+  mark(ev, 5, s);
+  combine_kernel<<<unsigned(T), 256, 0, s>>>(o, w, int(T), int(H), k, y);
+  rc = launch_status();
+  mark(ev, 6, s);
+  return rc;
+}
+
+}  // namespace
+}  // namespace w8a8
+
+extern "C" {
+
+int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                     const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E, int k,
+                     int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
+                     w8a8_stream stream) {
+  return moe_forward_impl(x, wg, bias, wgu, s_gu, wd, s_d, T, H, E, k, I, renorm, workspace, workspace_bytes, y,
+                          stream, nullptr);
+}
+
+int w8a8_moe_forward_profiled(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                              const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H,
+                              int64_t E, int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes,
+                              w8a8_bf16* y, w8a8_stream stream, void* const* stage_events) {
+  return moe_forward_impl(x, wg, bias, wgu, s_gu, wd, s_d, T, H, E, k, I, renorm, workspace, workspace_bytes, y,
+                          stream, stage_events);
+}
+
+size_t w8a8_linear_workspace_size(int64_t M, int64_t K, int64_t N, int w_format, int group) {
+  if (M < 0 || K <= 0 || N <= 0) return 0;
+  if (K % 128 || N % 128) return 0;
+  if (w_format == W8A8_W_INT4_PER_GROUP && group != 128) return 0;
+  if (w_format != W8A8_W_INT8_PER_CHANNEL && w_format != W8A8_W_INT4_PER_GROUP) return 0;
+  const int64_t Mp = round_up(M > 0 ? M : 1, 128);
+  return align256(size_t(Mp) * K) + align256(sizeof(float) * Mp) + 256;
+}
+
+int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_format, int group, int64_t M, int64_t K,
+                int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream) {
+  if (M < 0 || K <= 0 || N <= 0) return W8A8_ERR_ARG;
+  const size_t need = w8a8_linear_workspace_size(M, K, N, w_format, group);
+  if (need == 0) return W8A8_ERR_UNSUPPORTED;
+  if (M == 0) return W8A8_OK;
+  if (!x || !wq || !sw || !workspace || !y) return W8A8_ERR_ARG;
+  if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return W8A8_ERR_UNSUPPORTED;
+  if (M >= (int64_t(1) << 30) || N * K >= (int64_t(1) << 40)) return W8A8_ERR_UNSUPPORTED;
+  if (w_format != W8A8_W_INT8_PER_CHANNEL) return W8A8_ERR_UNSUPPORTED;  // int4 path: not yet built
+  const int64_t Mp = round_up(M, 128);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(ws + align256(size_t(Mp) * K));
+  cudaStream_t s = as_stream(stream);
+  int rc = w8a8_quant_act_per_token(x, M, K, xq, sx, stream);
+  if (rc != W8A8_OK) return rc;
+  GemmParams p{};
+  if (!make_kmajor_map(&p.tmA, xq, false, K, Mp, 128) || !make_kmajor_map(&p.tmB, wq, false, K, N, 128))
+    return W8A8_ERR_UNSUPPORTED;
+  p.num_kb = int(K / 128);
+  p.n_tiles = int(N / 256);
+  p.num_groups = 1;
+  p.M = int(M);
+  p.b_n_step = 256;
+  p.b_half_offset = 128;
+  p.timeout_ns = wait_timeout_ns();
+  p.out = y;
+  p.ldo = int(N);
+  p.out_col_step = 256;
+  p.row_scale = sx;
+  p.col_scale = sw;
+  if (N % 256 == 0) {
+    const int tiles = int((M + 127) / 128) * p.n_tiles;
+    return launch_gemm<256, kEpiDense, kKindI8>(p, tiles, s);
+  }
+  // N % 128 == 0: 128-wide tiles
+  if (!make_kmajor_map(&p.tmB, wq, false, K, N, 64)) return W8A8_ERR_UNSUPPORTED;
+  p.n_tiles = int(N / 128);
+  p.b_n_step = 128;
+  p.b_half_offset = 64;
+  p.out_col_step = 128;
+  const int tiles = int((M + 127) / 128) * p.n_tiles;
+  return launch_gemm<128, kEpiDense, kKindI8>(p, tiles, s);
+}
+
+int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
+                      w8a8_stream stream) {
+  if (M < 0 || N <= 0 || K <= 0) return W8A8_ERR_ARG;
+  if (K % 128 || N % 128) return W8A8_ERR_UNSUPPORTED;
+  if (M == 0) return W8A8_OK;
+  if (!a || !b || !c) return W8A8_ERR_ARG;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c) || M >= (int64_t(1) << 30)) return W8A8_ERR_UNSUPPORTED;
+  GemmParams p{};
+  if (!make_kmajor_map(&p.tmA, a, false, K, M, 128) || !make_kmajor_map(&p.tmB, b, false, K, N, 64))
+    return W8A8_ERR_UNSUPPORTED;
+  p.num_kb = int(K / 128);
+  p.n_tiles = int(N / 128);
+  p.num_groups = 1;
+  p.M = int(M);
+  p.b_n_step = 128;
+  p.b_half_offset = 64;
+  p.timeout_ns = wait_timeout_ns();
+  p.out = c;
+  p.ldo = int(N);
+  p.out_col_step = 128;
+  const int tiles = int((M + 127) / 128) * p.n_tiles;
+  return launch_gemm<128, kEpiRawS32, kKindI8>(p, tiles, as_stream(stream));
+}
+
+int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {
+  if (timeout_ns == 0 || timeout_ns > 10ull * 1000 * 1000 * 1000) return W8A8_ERR_ARG;
+  wait_timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns);
+  return launch_status();
+}
+
+}  // extern "C"
