@@ -208,6 +208,9 @@ def run_native(args, wl, rank, world, dist):
     # ---- timed region: K profiled steps (stage events give the per-kernel durations)
     nst = 7
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    for row in ev:  # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()

@@ -160,5 +160,10 @@ def y_tolerance_check(run: MoERun, tokens: np.ndarray, clear: np.ndarray):
     yg = O.bf16_to_f32(run.y[sel]).astype(np.float64)
     err = np.abs(yg - yr)
     rel = np.linalg.norm(yg - yr) / max(np.linalg.norm(yr), 1e-30)
-    assert err.max() <= 2e-2, err.max()
+    # 2e-2 wherever a bf16 ulp is finer than that (|y| < 4); above, one rounding flip of
+    # the bf16 output is one ulp (2**-5 at |y| in [4, 8)), so exactly one ulp is allowed there
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(yr), 2.0 ** -126))) - 7)
+    tol = np.maximum(2e-2, ulp)
+    assert np.all(err <= tol), (err.max(), yr.flat[np.argmax(err - tol)])
+    assert (err > 2e-2).mean() <= 1e-4, (err > 2e-2).sum()
     assert rel <= 5e-3, rel
