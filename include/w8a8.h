@@ -152,6 +152,32 @@ int w8a8_moe_forward_profiled(const w8a8_bf16* x, const w8a8_bf16* wg, const flo
                               int64_t E, int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes,
                               w8a8_bf16* y, w8a8_stream stream, void* const* stage_events);
 
+/* Allocation-free variant of w8a8_moe_forward (no counterpart on the pages: it only changes
+ * where the scratch memory comes from).
+ *
+ * Some callers cannot hand this library a workspace: code on a latency-critical serving path
+ * where cudaMalloc may synchronise the whole device and stall every other stream, plugins
+ * whose host framework owns all device memory and lends none, and processes that run under
+ * a fixed device-memory budget decided before the first request. For them this entry point
+ * keeps its scratch in a buffer compiled into the library: W8A8_NOALLOC_SCRATCH_BYTES bytes
+ * of device memory that every GPU loading the library holds until the process exits.
+ *
+ *   - Arguments and results are those of w8a8_moe_forward, without the workspace.
+ *   - The call allocates and frees nothing. Shapes whose workspace (w8a8_moe_workspace_size)
+ *     exceeds W8A8_NOALLOC_SCRATCH_BYTES are rejected with W8A8_ERR_UNSUPPORTED before
+ *     anything is enqueued; that covers decode-sized batches (up to about 240 tokens of the
+ *     Qwen3-30B-A3B shaped layer, about 120 of the Qwen3-235B-A22B shaped one), not prefill.
+ *   - The first call on a device looks the buffer's address up on that device (the device
+ *     must be current). Make that first call before any stream capture begins.
+ *   - All calls on one device share the one buffer; each call overwrites it and resets what
+ *     must start at zero. Calls whose work overlaps on the GPU (different streams without
+ *     ordering between them) race on the buffer: serialise them, e.g. on one stream. The
+ *     intermediates of the last call stay in the buffer but are not exposed. */
+#define W8A8_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int w8a8_moe_forward_noalloc(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                             const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H,
+                             int64_t E, int k, int64_t I, int renorm, w8a8_bf16* y, w8a8_stream stream);
+
 /* Workspace bytes w8a8_linear needs (0 if the shape is rejected). */
 size_t w8a8_linear_workspace_size(int64_t M, int64_t K, int64_t N, int w_format, int group);
 

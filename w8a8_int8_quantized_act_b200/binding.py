@@ -57,6 +57,8 @@ SIGNATURES = {
                                 _c_p, _size, _c_p, _c_p]),
     "w8a8_moe_forward_profiled": (_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _i64,
                                          _int, _c_p, _size, _c_p, _c_p, ctypes.POINTER(_c_p)]),
+    "w8a8_moe_forward_noalloc": (_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _i64,
+                                        _int, _c_p, _c_p]),
     "w8a8_linear_workspace_size": (_size, [_i64, _i64, _i64, _int, _int]),
     "w8a8_linear": (_int, [_c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _size, _c_p, _c_p]),
     "w8a8_gemm_s8s8s32": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p]),
@@ -201,6 +203,24 @@ def w8a8_moe_forward(x, wg, wgu, s_gu, wd, s_d, k: int, renorm: bool = True, bia
     _check(lib().w8a8_moe_forward(_ptr(x), _ptr(wg), _ptr(bias), _ptr(wgu), _ptr(s_gu), _ptr(wd), _ptr(s_d),
                                   T, H, E, k, I, int(renorm), _ptr(workspace), workspace.numel(), _ptr(y),
                                   _stream(stream)), "w8a8_moe_forward")
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def w8a8_moe_forward_noalloc(x, wg, wgu, s_gu, wd, s_d, k: int, renorm: bool = True, bias=None, y=None,
+                             stream=None):
+    """The MoE forward with scratch in the library's own device buffer: for callers that can
+    not allocate (see include/w8a8.h). Only y is allocated here, and only when not passed."""
+    _bf16(x), _bf16(wg)
+    T, H = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(lib().w8a8_moe_forward_noalloc(_ptr(x), _ptr(wg), _ptr(bias), _ptr(wgu), _ptr(s_gu), _ptr(wd),
+                                          _ptr(s_d), T, H, E, k, I, int(renorm), _ptr(y), _stream(stream)),
+           "w8a8_moe_forward_noalloc")
     return y
 
 

@@ -422,6 +422,56 @@ int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
                           stream, nullptr);
 }
 
+// ------------------------------------------------------------------ allocation-free variant
+}  // extern "C"
+
+namespace w8a8 {
+namespace {
+
+// Device scratch for w8a8_moe_forward_noalloc. It lives in the library's module, so every GPU
+// that loads the library holds these bytes until the process exits. Host code must not pass
+// the symbol itself to a kernel (on the host it only names a stand-in object); the device
+// address comes from cudaGetSymbolAddress, fetched once per device below.
+constexpr size_t kNoallocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (first call per device looks it
+// up with that device current); nullptr if the lookup fails.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace w8a8
+
+extern "C" {
+
+int w8a8_moe_forward_noalloc(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                             const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H,
+                             int64_t E, int k, int64_t I, int renorm, w8a8_bf16* y, w8a8_stream stream) {
+  const int st = check_moe_shape(T, H, E, k, I);
+  if (st != W8A8_OK) return st;
+  if (T == 0) return W8A8_OK;
+  w8a8_moe_ws_layout L;
+  fill_layout(T, H, E, k, I, &L);
+  if (L.total > kNoallocScratchBytes) return W8A8_ERR_UNSUPPORTED;
+  void* scratch = noalloc_scratch();
+  if (scratch == nullptr) return W8A8_ERR_LAUNCH;
+  return moe_forward_impl(x, wg, bias, wgu, s_gu, wd, s_d, T, H, E, k, I, renorm, scratch, kNoallocScratchBytes, y,
+                          stream, nullptr);
+}
+
 int w8a8_moe_forward_profiled(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
                               const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H,
                               int64_t E, int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes,
