@@ -39,7 +39,7 @@ class W8A8Error(RuntimeError):
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "tile_counts", "offsets", "perm", "sx", "sx_sorted", "xq", "h",
-                 "s_h", "hq", "o", "total")]
+                 "s_h", "hq", "o", "logits", "total")]
 
 
 # (name, restype, argtypes) of every exported entry point
@@ -265,7 +265,8 @@ def moe_intermediates(workspace: torch.Tensor, T: int, H: int, E: int, k: int, I
         perm=view("perm", torch.int32, (A,)), sx=view("sx", torch.float32, (T,)),
         sx_sorted=view("sx_sorted", torch.float32, (Ap,)), xq=view("xq", torch.int8, (Ap, H)),
         h=view("h", torch.bfloat16, (Ap, I)), s_h=view("s_h", torch.float32, (Ap,)),
-        hq=view("hq", torch.int8, (Ap, I)), o=view("o", torch.bfloat16, (A, H)))
+        hq=view("hq", torch.int8, (Ap, I)), o=view("o", torch.bfloat16, (A, H)),
+        logits=view("logits", torch.float32, (T, E)))
 
 
 def w8a8_linear_workspace_size(M: int, K: int, N: int, w_format: int, group: int = 128) -> int:

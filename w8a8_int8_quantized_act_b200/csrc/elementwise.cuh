@@ -10,13 +10,14 @@ namespace w8a8 {
 constexpr int kRowWarps = 8;  // warps per CTA for one-warp-per-row kernels
 
 // q[r, :] = codes of src[r, :], scale[r] = amax / 127, for rows r < R (row length K).
+template <int U>
 __global__ void __launch_bounds__(kRowWarps * 32) quant_rows_kernel(const uint16_t* __restrict__ src,
                                                                     int64_t R, int K, int8_t* __restrict__ q,
                                                                     float* __restrict__ scale) {
   const int64_t r = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
   if (r >= R) return;
   int8_t* dst = q + r * K;
-  const float s = quant_row_warp(src + r * K, K, [&](int i, uint2 v) {
+  const float s = quant_row_warp<U>(src + r * K, K, [&](int i, uint2 v) {
     *reinterpret_cast<uint2*>(dst + i) = v;
   });
   if ((threadIdx.x & 31) == 0) scale[r] = s;
@@ -49,37 +50,54 @@ __global__ void __launch_bounds__(kRowWarps * 32) quant_int4_group128_kernel(
 // writing its codes to every sorted row that it feeds.
 //   tile_counts [C, E]: assignments per (128-token chunk, expert) (from the router)
 //   offsets [E+1], perm [A] (sorted row -> t*k + j), sx [T], sx_sorted [A], xq_sorted [A, H]
-// One CTA per 128-token chunk; each CTA derives its own write positions from tile_counts.
+// Grid (chunk, split): the CTAs of one 128-token chunk each derive the chunk's write positions
+// (only split 0 stores perm/offsets) and quantise every split-th token. Inside a chunk, the
+// rank of assignment (t, e) among the chunk's rows of expert e is the number of earlier tokens
+// of the chunk that chose e: a popcount over a 128-bit token mask per expert.
 constexpr int kPermThreads = 256;
 constexpr int kChunk = 128;
 
+template <int U>
 __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
     const uint16_t* __restrict__ x, const int* __restrict__ ids, const int* __restrict__ tile_counts, int T,
     int H, int E, int k, int* __restrict__ offsets, int* __restrict__ perm, float* __restrict__ sx,
     float* __restrict__ sx_sorted, int8_t* __restrict__ xq_sorted) {
   extern __shared__ int sm[];
-  int* base = sm;                 // [E]  first sorted row of this chunk's rows of expert e
-  int* run = sm + E;              // [E]  running count inside the chunk
-  int* dest = sm + 2 * E;         // [kChunk * k]
+  int* base = sm;                                   // [E]  first sorted row of the chunk's rows of e
+  int* before = sm + E;                             // [E]  rows of e in earlier chunks
+  int* dest = sm + 2 * E;                           // [kChunk * k]
+  int* cid = dest + kChunk * k;                     // [kChunk * k] the chunk's expert ids
+  uint32_t* mask = reinterpret_cast<uint32_t*>(cid + kChunk * k);  // [E][4] token masks
   const int C = (T + kChunk - 1) / kChunk;
   const int A = T * k;
   const int chunk = blockIdx.x;
+  const int split = blockIdx.y, nsplit = gridDim.y;
   const int t0 = chunk * kChunk;
   const int nt = min(kChunk, T - t0);
+  const int na = nt * k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  // per-expert totals and this chunk's prefix over earlier chunks
+  // per-expert totals and this chunk's prefix over earlier chunks; the chunk's ids; clear masks
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int total = 0, before = 0;
+    int total = 0, prior = 0;
     for (int c = 0; c < C; ++c) {
       const int v = __ldg(tile_counts + size_t(c) * E + e);
       total += v;
-      if (c < chunk) before += v;
+      if (c < chunk) prior += v;
     }
     base[e] = total;  // temporarily: totals
-    run[e] = before;
+    before[e] = prior;
   }
-  for (int i = threadIdx.x; i < kChunk * k; i += blockDim.x) dest[i] = -1;
+  for (int i = threadIdx.x; i < 4 * E; i += blockDim.x) mask[i] = 0u;
+  for (int i = threadIdx.x; i < kChunk * k; i += blockDim.x) {
+    dest[i] = -1;
+    int e = (i < na) ? __ldg(ids + size_t(t0) * k + i) : -1;
+    if (i < na && (e < 0 || e >= E)) {
+      if (split == 0) atomicOr(&g_error_word, kErrBadIndex);
+      e = -1;  // an invalid id gets no row
+    }
+    cid[i] = e;
+  }
   __syncthreads();
   if (warp == 0) {  // exclusive scan of totals over experts (one warp)
     int carry = 0;
@@ -94,52 +112,42 @@ __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
       }
       if (e < E) {
         const int excl = carry + incl - v;
-        if (chunk == 0) offsets[e] = excl;
-        base[e] = excl + run[e];
-        run[e] = 0;
+        if (chunk == 0 && split == 0) offsets[e] = excl;
+        base[e] = excl + before[e];
       }
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (chunk == 0 && lane == 0) offsets[E] = carry;
+    if (chunk == 0 && split == 0 && lane == 0) offsets[E] = carry;
+  } else {
+    for (int i = threadIdx.x - 32; i < na; i += blockDim.x - 32) {
+      const int e = cid[i];
+      const int tl = i / k;
+      if (e >= 0) atomicOr(mask + 4 * e + (tl >> 5), 1u << (tl & 31));
+    }
   }
   __syncthreads();
-  // stable ranks: warp 0 walks the chunk's assignments in (token, slot) order
-  if (warp == 0) {
-    const int per = 32 / k;  // tokens per step
-    for (int tl0 = 0; tl0 < nt; tl0 += per) {
-      const int tl = tl0 + lane / k;
-      const int j = lane % k;
-      const bool valid = (lane < per * k) && (tl < nt);
-      const unsigned active = __ballot_sync(0xffffffffu, valid);
-      if (valid) {
-        const int a = (t0 + tl) * k + j;
-        int e = __ldg(ids + a);
-        if (e < 0 || e >= E) {
-          atomicOr(&g_error_word, kErrBadIndex);
-          e = 0;
-        }
-        const unsigned peers = __match_any_sync(active, e);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        const int b = run[e];
-        __syncwarp(active);
-        if (rank == 0) run[e] = b + __popc(peers);
-        const int d = base[e] + b + rank;
-        if (d >= 0 && d < A) {
-          perm[d] = a;
-          dest[tl * k + j] = d;
-        } else {
-          atomicOr(&g_error_word, kErrBadIndex);  // ids inconsistent with the per-chunk counts
-        }
-      }
-      __syncwarp();
+  // every assignment's sorted row, in parallel
+  for (int i = threadIdx.x; i < na; i += blockDim.x) {
+    const int e = cid[i];
+    if (e < 0) continue;
+    const int tl = i / k;
+    const uint32_t* mk = mask + 4 * e;
+    int rank = __popc(mk[tl >> 5] & ((1u << (tl & 31)) - 1u));
+    for (int w = 0; w < (tl >> 5); ++w) rank += __popc(mk[w]);
+    const int d = base[e] + rank;
+    if (d >= 0 && d < A) {
+      if (split == 0) perm[d] = t0 * k + i;
+      dest[i] = d;
+    } else if (split == 0) {
+      atomicOr(&g_error_word, kErrBadIndex);  // ids inconsistent with the per-chunk counts
     }
   }
   __syncthreads();
   // quantise each token once, write its codes to its k sorted rows
-  for (int tl = warp; tl < nt; tl += kPermThreads / 32) {
+  for (int tl = split + nsplit * warp; tl < nt; tl += nsplit * (kPermThreads / 32)) {
     const int t = t0 + tl;
     const int* drow = dest + tl * k;
-    const float s = quant_row_warp(x + size_t(t) * H, H, [&](int i, uint2 v) {
+    const float s = quant_row_warp<U>(x + size_t(t) * H, H, [&](int i, uint2 v) {
       for (int j = 0; j < k; ++j)
         if (drow[j] >= 0) *reinterpret_cast<uint2*>(xq_sorted + size_t(drow[j]) * H + i) = v;
     });

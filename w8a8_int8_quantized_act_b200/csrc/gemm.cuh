@@ -1,58 +1,65 @@
 // Persistent, warp-specialised grouped GEMM on the 5th-generation tensor cores (sm_100a).
 //
-//   D[r, n] = sum_k A[r, k] * B[n, k]      (A and B K-major; D accumulated in TMEM)
+//   D[m, n] = sum_k A[m, k] * B[n, k]      (A and B K-major; D accumulated in TMEM)
 //
-// A holds activation rows, grouped: rows offsets[g] .. offsets[g+1]-1 belong to group g
-// (an expert). B holds one weight block per group. Each CTA owns one SM and walks a static
-// list of 128 x BN output tiles; per CTA:
-//   warp 0      TMA producer: 128-byte-swizzled K-blocks of A (128 rows) and B (BN rows)
-//               into a STAGES-deep shared-memory ring (mbarrier full/empty pairs);
-//   warp 1      TMEM allocator and MMA issuer: one thread issues tcgen05.mma
-//               (kind::i8 -> s32, or kind::f16 bf16 -> f32) into one of two TMEM
-//               accumulators, so the epilogue of tile i overlaps the MMAs of tile i+1;
-//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes (one output row per thread),
-//               fused dequantisation / activation / routing, stores to global memory.
+// The MMA's M side (128 TMEM lanes) holds A rows, its N side holds up to NB B rows.
+//   * Expert GEMMs (kind::i8) put weight channels on M and token rows on N ("swap-AB"): a tile
+//     is (expert g, token block of at most NB sorted rows, block of 128 channels), and the MMA
+//     N is the token count of the block rounded up to 16, so decode tiles with a handful of
+//     tokens stream their weights without dragging 128 activation rows along. gate_up loads
+//     two A blocks per stage (128 gate rows and the matching 128 up rows) into two
+//     accumulators, so one thread holds gate and up of the same channel.
+//   * The router (kind::f16) puts 128 token rows on M and the E experts on N, so one thread
+//     owns all logits of its token.
+// Roles per CTA (one CTA per SM, 10 warps):
+//   warp 0      TMA producer: 128-byte-swizzled K-blocks (128 bytes of K) into a ring of
+//               STAGES shared-memory slots guarded by mbarrier full/empty pairs;
+//   warp 1      TMEM allocator and MMA issuer (one thread): tcgen05.mma into one of two
+//               accumulator sets, so the epilogue of a tile overlaps the next tile's MMAs;
+//   warps 2-9   epilogue: tcgen05.ld of their TMEM lane quarter, fused dequantisation,
+//               activation, routing, stores. Two warps share a quarter and split columns.
 // Every mbarrier wait is bounded; a timeout aborts the CTA cleanly (see ptx.cuh).
 #pragma once
-#include "numerics.cuh"
+#include "routing.cuh"
 
 namespace w8a8 {
 
 enum EpiKind : int {
   kEpiRawS32 = 0,   // int32 accumulators stored as they are (exact integer GEMM)
-  kEpiRouter = 1,   // fp32 logits -> (+bias) softmax, top-k, weights, per-tile expert histogram
+  kEpiRouter = 1,   // fp32 logits -> (+bias) softmax, top-k, weights, expert histogram
   kEpiGateUp = 2,   // int32 gate|up -> dequant, SiLU(gate)*up -> bf16 h
   kEpiDown = 3,     // int32 -> dequant -> bf16 o written to the assignment's slot row
   kEpiDense = 4,    // int32 -> dequant -> bf16 y (dense W8A8 linear)
 };
 
-constexpr int kBM = 128;            // output rows per tile (tcgen05 M)
-constexpr int kKBlockBytes = 128;   // K bytes per pipeline stage (one swizzle atom row)
-constexpr int kGemmThreads = 192;   // 6 warps
+constexpr int kBM = 128;            // MMA M (TMEM lanes)
+constexpr int kKBlockBytes = 128;   // K bytes per pipeline stage (one swizzle row)
+constexpr int kBBoxRows = 16;       // rows per TMA box on the N side
+constexpr int kEpiWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kMaxGroups = 1024;
-constexpr int kMaxTopK = 16;
 
 struct GemmParams {
-  CUtensorMap tmA;  // A: [rowsA, K] K-major, box 128 rows x 128 bytes
-  CUtensorMap tmB;  // B: [G * b_rows_per_group, K] K-major, box BN/2 rows x 128 bytes
+  CUtensorMap tmA;   // M side: boxes of 128 rows x 128 bytes
+  CUtensorMap tmB;   // N side: boxes of 16 rows x 128 bytes (ragged tiles)
+  CUtensorMap tmB2;  // N side: boxes of NB rows x 128 bytes (full tiles: one copy per stage)
   int num_kb;                  // K-blocks of 128 bytes
-  int n_tiles;                 // tiles along N per group
+  int n_cb;                    // 128-channel blocks per group (router: 1)
   int num_groups;              // G
-  const int* group_offsets;    // [G+1] row offsets into A (device); nullptr: one group of M rows
-  int M;                       // rows of A when group_offsets is null
-  int b_rows_per_group;        // rows of B per group
-  int b_n_step;                // B row advance per N tile
-  int b_half_offset;           // B row offset of the second half-box of a tile
+  const int* group_offsets;    // [G+1] token-row offsets (device); nullptr: one group of M rows
+  int M;                       // token rows when group_offsets is null
+  int a_rows_per_group;        // weight rows per group (gate_up: 2I, down: H, dense: 0)
+  int a_second_offset;         // gate_up: row offset of the up block (I)
+  int nb_fixed;                // router: N side rows (E rounded up to 16); else 0
   uint64_t timeout_ns;         // bound on every mbarrier wait
   // epilogue operands
   void* out;                   // see EpiKind
   int ldo;                     // output row stride, elements
-  int out_col_step;            // output column advance per N tile
-  int n_valid;                 // valid output columns (router: E)
-  const float* row_scale;      // per A-row scale (x scale, or the requantisation scale of h)
-  const float* col_scale;      // per output channel scale, group-major
+  int n_valid;                 // router: E
+  const float* row_scale;      // per token-row scale (sx, or the requantisation scale of h)
+  const float* col_scale;      // per channel scale, group-major
   int col_scale_stride;        // per group
-  int up_offset;               // gate_up: column offset of the up half inside col_scale
+  int up_offset;               // gate_up: offset of the up scales inside a group's scales
   const int* row_map;          // down: sorted row -> slot row (t*k + j)
   // router
   const float* bias;
@@ -60,19 +67,31 @@ struct GemmParams {
   int renorm;
   float* topk_w;
   int* tile_counts;            // expert histogram rows (nullptr: none); zeroed before the launch
-  int tile_count_stride;       // elements between the rows of consecutive m-tiles (0: one shared row)
+  int tile_count_stride;       // elements between the rows of consecutive token tiles (0: one row)
 };
 
-template <int BN>
+template <int NA, int NB, int EPI>
 struct GemmCfg {
   static constexpr int kABytes = kBM * kKBlockBytes;
-  static constexpr int kBBytes = BN * kKBlockBytes;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
-  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
-  static constexpr int kBarBytes = 256;
+  static constexpr int kBBytes = NB * kKBlockBytes;
+  static constexpr int kStageBytes = NA * kABytes + kBBytes;
+  // router: logits of one tile transposed to [expert][token] (row pitch 129 floats, so both the
+  // per-token writes and the per-expert reads are free of bank conflicts)
+  static constexpr int kXBytes = (EPI == kEpiRouter) ? NB * 129 * 4 : 0;
+  static constexpr int kStagesRaw = (196 * 1024 - kXBytes) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+  static constexpr int kAccCols = NA * NB;  // TMEM columns of one accumulator set
+  static constexpr int kTmemCols =
+      (2 * kAccCols <= 32)
+          ? 32
+          : (2 * kAccCols <= 64 ? 64 : (2 * kAccCols <= 128 ? 128 : (2 * kAccCols <= 256 ? 256 : 512)));
+  static constexpr int kBarBytes = 512;
+  // after the barriers: token-block prefix [G+1], cached group offsets [G+1], router exchange
   static constexpr size_t kSmemBytes =
-      1024 + size_t(kStages) * kStageBytes + kBarBytes + sizeof(int) * (kMaxGroups + 1);
+      1024 + size_t(kStages) * kStageBytes + kBarBytes + 2 * sizeof(int) * (kMaxGroups + 1) + kXBytes;
+  static_assert(2 * kAccCols <= 512, "two accumulator sets must fit in TMEM");
+  // (the router with 128 < E <= 256 keeps one stage: its transposed logits fill the rest)
+  static_assert(kStages >= 2 || (EPI == kEpiRouter && kStages >= 1), "pipeline too shallow");
 };
 
 // Largest g with prefix[g] <= mt (prefix is non-decreasing, prefix[0] = 0).
@@ -85,198 +104,191 @@ __device__ __forceinline__ int find_group(const int* prefix, int G, int mt) {
   return lo;
 }
 
-struct TileCoord {
-  int g, m0, nt, row0, rows;
+struct Tile {
+  int g;       // group (expert)
+  int cb;      // channel block (router: 0)
+  int tok0;    // first token row of the tile
+  int rows;    // valid token rows
+  int a_row;   // first A row (weights, or router tokens)
+  int b_row;   // first B row (tokens, or router experts)
+  int nb;      // B rows loaded (multiple of 16) = MMA N
+  int tt;      // token-tile index (router histogram row)
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const GemmParams& p, const int* mt_prefix, int tile) {
-  TileCoord c;
-  const int mt = tile / p.n_tiles;
-  c.nt = tile - mt * p.n_tiles;
-  if (p.group_offsets == nullptr) {
+template <int EPI, int NB>
+__device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* mt_prefix, const int* goff, int tile) {
+  Tile c;
+  if constexpr (EPI == kEpiRouter) {
     c.g = 0;
-    c.m0 = mt * kBM;
-    c.row0 = c.m0;
-    c.rows = min(kBM, p.M - c.m0);
+    c.cb = 0;
+    c.tt = tile;
+    c.tok0 = tile * kBM;
+    c.rows = min(kBM, p.M - c.tok0);
+    c.a_row = c.tok0;
+    c.b_row = 0;
+    c.nb = p.nb_fixed;
   } else {
-    c.g = find_group(mt_prefix, p.num_groups, mt);
-    c.m0 = (mt - mt_prefix[c.g]) * kBM;
-    const int off = __ldg(p.group_offsets + c.g);
-    const int cnt = __ldg(p.group_offsets + c.g + 1) - off;
-    c.row0 = off + c.m0;
-    c.rows = min(kBM, cnt - c.m0);
+    const int mt = tile / p.n_cb;
+    c.cb = tile - mt * p.n_cb;
+    c.tt = mt;
+    int off, cnt, blk;
+    if (p.group_offsets == nullptr) {
+      c.g = 0;
+      off = 0;
+      cnt = p.M;
+      blk = mt;
+    } else {
+      c.g = find_group(mt_prefix, p.num_groups, mt);
+      off = goff[c.g];
+      cnt = goff[c.g + 1] - off;
+      blk = mt - mt_prefix[c.g];
+    }
+    c.tok0 = off + blk * NB;
+    c.rows = min(NB, cnt - blk * NB);
+    c.a_row = c.g * p.a_rows_per_group + c.cb * kBM;
+    c.b_row = c.tok0;
+    c.nb = (c.rows + 15) & ~15;
   }
   return c;
 }
 
+// 16 consecutive 32-bit TMEM columns of the warp's 32 lanes (wait included). TMEM is not
+// addressable memory, so the statement carries no memory clobber: values already loaded from
+// global or shared memory stay in registers across it.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // ---------------------------------------------------------------------------- epilogues
-// Each runs on the 128 epilogue threads; thread (quarter q, lane l) owns tile row 32q + l.
-template <int BN, int EPI>
-__device__ __forceinline__ void run_epilogue(const GemmParams& p, const TileCoord& c, uint32_t taddr,
-                                             int row_local, int mt) {
-  const bool valid = row_local < c.rows;
-  const int row = c.row0 + row_local;
-  uint32_t r[32];
-  if constexpr (EPI == kEpiRawS32) {
-    int32_t* out = static_cast<int32_t*>(p.out) + size_t(row) * p.ldo + size_t(c.nt) * p.out_col_step;
+// Expert GEMM epilogues: thread = one channel (TMEM lane), columns = the tile's token rows.
+// The two epilogue warps of a lane quarter take alternate 16-column chunks.
+template <int EPI, int NB>
+__device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Tile& c, uint32_t t_lane, int lane_ch,
+                                                  int half) {
+  const int ch = c.cb * kBM + lane_ch;  // channel within the group
+  const size_t ldo = size_t(p.ldo);
+  const float* __restrict__ row_scale = p.row_scale;
+  uint32_t r[16];
+  if constexpr (EPI == kEpiGateUp) {
+    const float sg = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+    const float su = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + p.up_offset + ch);
+    uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
+    uint32_t ru[16];
 #pragma unroll 1
-    for (int col = 0; col < BN; col += 32) {
-      tmem_ld32(taddr + col, r);
-      if (valid) {
-        int4* dst = reinterpret_cast<int4*>(out + col);
+    for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
+      tmem_ld16(t_lane + j0, r);        // gate accumulators
+      tmem_ld16(t_lane + NB + j0, ru);  // up accumulators
 #pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-      }
-    }
-  } else if constexpr (EPI == kEpiGateUp) {
-    // TMEM columns [0, BN/2) are gate channels, [BN/2, BN) the matching up channels.
-    constexpr int HALF = BN / 2;
-    const int hc0 = c.nt * HALF;  // first h column of this tile
-    const float sx = valid ? __ldg(p.row_scale + row) : 0.0f;
-    const float* sg = p.col_scale + size_t(c.g) * p.col_scale_stride + hc0;
-    const float* su = sg + p.up_offset;
-    uint16_t* out = static_cast<uint16_t*>(p.out) + size_t(row) * p.ldo + hc0;
-    uint32_t ru[32];
-#pragma unroll 1
-    for (int col = 0; col < HALF; col += 32) {
-      tmem_ld32(taddr + col, r);
-      tmem_ld32(taddr + HALF + col, ru);
-      uint32_t packed[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float h2[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float g = dequant(int32_t(r[i + j]), sx, __ldg(sg + col + i + j));
-          const float u = dequant(int32_t(ru[i + j]), sx, __ldg(su + col + i + j));
-          h2[j] = __fmul_rn(silu_exact(g), u);
+      for (int j = 0; j < 16; ++j) {
+        if (j0 + j < c.rows) {
+          const int row = c.tok0 + j0 + j;
+          const float sx = __ldg(row_scale + row);
+          const float g = dequant(int32_t(r[j]), sx, sg);
+          const float u = dequant(int32_t(ru[j]), sx, su);
+          out[size_t(row) * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu_exact(g), u)));
         }
-        packed[i / 2] = pack_bf16(h2[0], h2[1]);
-      }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(out + col);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
       }
     }
   } else if constexpr (EPI == kEpiDown || EPI == kEpiDense) {
-    const int n0 = c.nt * p.out_col_step;
-    const float srow = valid ? __ldg(p.row_scale + row) : 0.0f;
-    const float* sc = p.col_scale + size_t(c.g) * p.col_scale_stride + n0;
-    int orow = row;
-    if constexpr (EPI == kEpiDown) orow = valid ? __ldg(p.row_map + row) : 0;
-    uint16_t* out = static_cast<uint16_t*>(p.out) + size_t(orow) * p.ldo + n0;
+    const float sc = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+    const int* __restrict__ row_map = p.row_map;
+    uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
 #pragma unroll 1
-    for (int col = 0; col < BN; col += 32) {
-      tmem_ld32(taddr + col, r);
-      uint32_t packed[16];
+    for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
+      tmem_ld16(t_lane + j0, r);
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float a = dequant(int32_t(r[i]), srow, __ldg(sc + col + i));
-        const float b = dequant(int32_t(r[i + 1]), srow, __ldg(sc + col + i + 1));
-        packed[i / 2] = pack_bf16(a, b);
-      }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(out + col);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-      }
-    }
-  } else if constexpr (EPI == kEpiRouter) {
-    // One token per thread: logits of experts 0..E-1 in TMEM columns 0..E-1 (fp32).
-    const int E = p.n_valid;
-    const int k = p.topk;
-    float tv[kMaxTopK];
-    int ti[kMaxTopK];
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) { tv[j] = -INFINITY; ti[j] = 0x7fffffff; }
-#pragma unroll 1
-    for (int col = 0; col < BN; col += 32) {
-      tmem_ld32(taddr + col, r);
-#pragma unroll 1
-      for (int i = 0; i < 32; ++i) {
-        const int e = col + i;
-        if (e >= E) break;
-        float l = __uint_as_float(r[i]);
-        if (p.bias) l += __ldg(p.bias + e);
-        // insert keeping descending values; equal values keep the lower expert first
-        if (l > tv[k - 1]) {
-          int pos = k - 1;
-          while (pos > 0 && l > tv[pos - 1]) { tv[pos] = tv[pos - 1]; ti[pos] = ti[pos - 1]; --pos; }
-          tv[pos] = l;
-          ti[pos] = e;
+      for (int j = 0; j < 16; ++j) {
+        if (j0 + j < c.rows) {
+          const int row = c.tok0 + j0 + j;
+          const int orow = (EPI == kEpiDown) ? __ldg(row_map + row) : row;
+          const float v = dequant(int32_t(r[j]), __ldg(row_scale + row), sc);
+          out[size_t(orow) * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
         }
       }
     }
-    // a slot left unfilled (only possible with non-finite logits) is reported, never used
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k && (ti[j] < 0 || ti[j] >= E)) {
-        atomicOr(&g_error_word, kErrBadIndex);
-        ti[j] = j;
-        tv[j] = tv[0];
-      }
-    }
-    const float m = tv[0];
-    float sel_sum = 0.0f;
-    float ev[kMaxTopK];
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      ev[j] = (j < k) ? expf(tv[j] - m) : 0.0f;
-      sel_sum += ev[j];
-    }
-    float denom = sel_sum;
-    if (!p.renorm) {
-      denom = 0.0f;
+  } else if constexpr (EPI == kEpiRawS32) {
+    int32_t* out = static_cast<int32_t*>(p.out) + ch;
 #pragma unroll 1
-      for (int col = 0; col < BN; col += 32) {
-        tmem_ld32(taddr + col, r);
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i) {
-          const int e = col + i;
-          if (e >= E) break;
-          float l = __uint_as_float(r[i]);
-          if (p.bias) l += __ldg(p.bias + e);
-          denom += expf(l - m);
-        }
-      }
-    }
-    if (valid) {
-      int* ids = static_cast<int*>(p.out) + size_t(row) * k;
-      float* w = p.topk_w + size_t(row) * k;
-      for (int j = 0; j < k; ++j) {
-        ids[j] = ti[j];
-        w[j] = ev[j] / denom;
-      }
-      if (p.tile_counts != nullptr) {
-        int* counts = p.tile_counts + size_t(mt) * p.tile_count_stride;
-        for (int j = 0; j < k; ++j) atomicAdd(counts + ti[j], 1);
-      }
+    for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
+      tmem_ld16(t_lane + j0, r);
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j0 + j < c.rows) out[size_t(c.tok0 + j0 + j) * ldo] = int32_t(r[j]);
     }
   }
 }
 
-template <int BN, int EPI, int KIND>
+// Router epilogue. The logits of a 128-token tile arrive one token per thread (TMEM lane);
+// the two epilogue warps of each lane quarter copy half the experts each into shared memory,
+// transposed to [expert][token]. After all 256 epilogue threads have written (bounded mbarrier),
+// each warp takes whole tokens: lane l holds experts l, l+32, ... as order-preserving integer
+// keys, and each of the k rounds is two warp reductions: the largest key, then the lowest
+// expert holding it (equal values go to the lower expert). The winner's lane drops the entry.
+// Lanes 0..k-1 end up holding pick j = lane, normalise and store them; a second barrier phase
+// marks the buffer free for the CTA's next tile.
+template <int NB>
+__device__ __forceinline__ void epilogue_router(const GemmParams& p, const Tile& c, uint32_t t_lane, int lane_row,
+                                                int half, int ew, float* xs, uint64_t* xbar, uint32_t& xphase,
+                                                const WaitCtx& wc) {
+  constexpr int SPAN = NB >= 32 ? NB / 2 : NB;  // experts each warp of a quarter copies
+  constexpr int PER = (NB + 31) / 32;  // experts per lane in the per-token phase
+  const int E = p.n_valid;
+  const int k = p.topk;
+  const float* __restrict__ bias = p.bias;
+  // 1. TMEM -> shared memory, transposed (with 16 experts the lower warp copies them all)
+  if (NB >= 32 || half == 0) {
+    const int c0 = NB >= 32 ? half * SPAN : 0;
+#pragma unroll
+    for (int c16 = 0; c16 < SPAN; c16 += 16) {
+      uint32_t r[16];
+      tmem_ld16(t_lane + c0 + c16, r);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xs[(c0 + c16 + i) * 129 + lane_row] = __uint_as_float(r[i]);
+    }
+  }
+  mbar_arrive(xbar);
+  if (!mbar_wait(xbar, xphase, wc)) return;
+  xphase ^= 1u;
+  // 2. one warp per token
+  int* counts = p.tile_counts != nullptr ? p.tile_counts + size_t(c.tt) * p.tile_count_stride : nullptr;
+#pragma unroll 1
+  for (int tl = ew; tl < c.rows; tl += kEpiWarps) {
+    const int row = c.tok0 + tl;
+    warp_topk_token<PER>([&](int e) { return xs[e * 129 + tl]; }, E, k, p.renorm != 0, bias,
+                         static_cast<int*>(p.out) + size_t(row) * k, p.topk_w + size_t(row) * k, counts);
+  }
+  // 3. buffer free for the next tile once every epilogue thread is past step 2
+  mbar_arrive(xbar);
+  mbar_wait(xbar, xphase, wc);
+  xphase ^= 1u;
+}
+
+template <int NA, int NB, int EPI, int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<NA, NB, EPI>;
   constexpr int STAGES = Cfg::kStages;
-  constexpr uint32_t IDESC = (KIND == kKindI8) ? idesc_s8s8s32(BN) : idesc_bf16f32(BN);
   constexpr int KB_ELEMS = (KIND == kKindI8) ? 128 : 64;
+  constexpr uint32_t IDESC0 = (KIND == kKindI8) ? idesc_s8s8s32(0) : idesc_bf16f32(0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * Cfg::kABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::kBBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1 + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* mt_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + Cfg::kBarBytes);
+  int* goff = mt_prefix + (kMaxGroups + 1);
+  float* xs = reinterpret_cast<float*>(goff + (kMaxGroups + 1));  // router: [NB][129] logits
+  uint64_t* xbar = drain + 1;  // router: all epilogue threads, two phases per tile
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -284,36 +296,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, 4 * 32); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, kEpiWarps * 32); }
     mbar_init(drain, 1);
+    mbar_init(xbar, 32 * kEpiWarps);
     fence_mbar_init();
     *abort_flag = 0;
-    // m-tile prefix over groups
-    if (p.group_offsets != nullptr) {
-      int acc = 0;
-      mt_prefix[0] = 0;
-      for (int g = 0; g < p.num_groups; ++g) {
-        const int cnt = __ldg(p.group_offsets + g + 1) - __ldg(p.group_offsets + g);
-        acc += (cnt + kBM - 1) / kBM;
-        mt_prefix[g + 1] = acc;
-      }
-    } else {
-      mt_prefix[0] = 0;
-      mt_prefix[1] = (p.M + kBM - 1) / kBM;
-    }
+    mt_prefix[0] = 0;
+    if (!(EPI != kEpiRouter && p.group_offsets != nullptr))
+      mt_prefix[1] = (EPI == kEpiRouter) ? (p.M + kBM - 1) / kBM : (p.M + NB - 1) / NB;
     tma_prefetch_map(&p.tmA);
     tma_prefetch_map(&p.tmB);
+    tma_prefetch_map(&p.tmB2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  if (EPI != kEpiRouter && p.group_offsets != nullptr && warp >= 2) {
+    // cache the group offsets and build the token-block prefix: one warp-wide scan per 32 groups
+    for (int g = threadIdx.x - 64; g <= p.num_groups; g += 32 * kEpiWarps) goff[g] = __ldg(p.group_offsets + g);
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kEpiWarps) : "memory");
+    if (warp == 2) {
+      int carry = 0;
+      for (int g0 = 0; g0 < p.num_groups; g0 += 32) {
+        const int g = g0 + lane;
+        const int v = (g < p.num_groups) ? (goff[g + 1] - goff[g] + NB - 1) / NB : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        if (g < p.num_groups) mt_prefix[g + 1] = carry + incl;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int groups_for_prefix = (p.group_offsets != nullptr) ? p.num_groups : 1;
-  const int total_tiles = mt_prefix[groups_for_prefix] * p.n_tiles;
+  const int groups_for_prefix = (EPI != kEpiRouter && p.group_offsets != nullptr) ? p.num_groups : 1;
+  const int total_tiles = mt_prefix[groups_for_prefix] * p.n_cb;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -322,17 +346,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
-        const TileCoord c = decode_tile(p, mt_prefix, tile);
-        const int b_row0 = c.g * p.b_rows_per_group + c.nt * p.b_n_step;
-        const int b_row1 = b_row0 + p.b_half_offset;
+        const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
+        const uint32_t bytes = uint32_t(NA * Cfg::kABytes + c.nb * kKBlockBytes);
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
-          mbar_arrive_expect_tx(full + stage, Cfg::kStageBytes);
+          uint8_t* st = smem + stage * Cfg::kStageBytes;
+          mbar_arrive_expect_tx(full + stage, bytes);
           const int x = kb * KB_ELEMS;
-          tma_load_2d(sA + stage * Cfg::kABytes, &p.tmA, full + stage, x, c.row0);
-          tma_load_2d(sB + stage * Cfg::kBBytes, &p.tmB, full + stage, x, b_row0);
-          tma_load_2d(sB + stage * Cfg::kBBytes + Cfg::kBBytes / 2, &p.tmB, full + stage, x, b_row1);
+          tma_load_2d(st, &p.tmA, full + stage, x, c.a_row);
+          if (NA == 2) tma_load_2d(st + Cfg::kABytes, &p.tmA, full + stage, x, c.a_row + p.a_second_offset);
+          uint8_t* sb = st + NA * Cfg::kABytes;
+          if (c.nb == NB) {
+            tma_load_2d(sb, &p.tmB2, full + stage, x, c.b_row);
+          } else {
+            for (int b = 0; b < c.nb; b += kBBoxRows)
+              tma_load_2d(sb + b * kKBlockBytes, &p.tmB, full + stage, x, c.b_row + b);
+          }
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -357,19 +387,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       uint32_t acc_phase = 0;
       bool issued_any = false;
       for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+        const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
+        const uint32_t idesc = IDESC0 | (uint32_t(c.nb >> 3) << 17);
         if (!mbar_wait(tempty + acc, acc_phase ^ 1u, wc)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        const uint32_t d0 = tmem_base + uint32_t(acc * Cfg::kAccCols);
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(full + stage, phase, wc)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_addr(sA + stage * Cfg::kABytes);
-          const uint32_t b0 = smem_addr(sB + stage * Cfg::kBBytes);
+          const uint32_t s0 = smem_addr(smem + stage * Cfg::kStageBytes);
+          const uint32_t sb = s0 + NA * Cfg::kABytes;
 #pragma unroll
-          for (int kk = 0; kk < kKBlockBytes / 32; ++kk)
-            tc_mma<KIND>(d_tmem, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), IDESC,
-                         (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kKBlockBytes / 32; ++kk) {
+            const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            tc_mma<KIND>(d0, sw128_kmajor_desc(s0 + kk * 32), bdesc, idesc, accum);
+            if (NA == 2)
+              tc_mma<KIND>(d0 + NB, sw128_kmajor_desc(s0 + Cfg::kABytes + kk * 32), bdesc, idesc, accum);
+          }
           issued_any = true;
           tc_commit(empty + stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -388,17 +424,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row_local = q * 32 + lane;
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;   // which of the quarter's two warps
+    const int lane_idx = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t xphase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      const TileCoord c = decode_tile(p, mt_prefix, tile);
+      const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
       if (!mbar_wait(tfull + acc, acc_phase, wc)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN);
-      run_epilogue<BN, EPI>(p, c, taddr, row_local, tile / p.n_tiles);
+      const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * Cfg::kAccCols);
+      if constexpr (EPI == kEpiRouter) {
+        epilogue_router<NB>(p, c, t_lane, lane_idx, half, warp - 2, xs, xbar, xphase, wc);
+      } else {
+        epilogue_channels<EPI, NB>(p, c, t_lane, lane_idx, half);
+      }
       tc_fence_before();
       mbar_arrive(tempty + acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }

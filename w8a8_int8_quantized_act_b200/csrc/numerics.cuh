@@ -22,6 +22,24 @@ __device__ __forceinline__ int sym_code(float v, float scale, int qmax) {
   return max(-qmax, min(qmax, q));
 }
 
+// The same code, with the divide replaced by a multiply where that cannot change the result:
+// y = v * rcp_rn(scale) is within 2.3e-5 of fl(v / scale) when |v / scale| <= 127 (two
+// round-to-nearest steps, 2^-24 relative each, plus fl(v/scale)'s own half ulp), so if y lies
+// more than 3e-5 from every half-integer both round to the same integer; the few values that
+// land closer take the true divide. inv = __frcp_rn(scale), computed once per row.
+__device__ __forceinline__ int sym_code_fast(float v, float scale, float inv, int qmax) {
+  if (scale == 0.0f) return 0;
+  const float y = __fmul_rn(v, inv);
+  const float f = y - floorf(y);
+  int q;
+  if (fabsf(f - 0.5f) > 3e-5f) {
+    q = __float2int_rn(y);
+  } else {
+    q = __float2int_rn(__fdiv_rn(v, scale));
+  }
+  return max(-qmax, min(qmax, q));
+}
+
 // exp(x) by Cody-Waite range reduction (ln 2 split into a 15-significant-bit high part and a
 // low part) and a degree-7 Taylor polynomial evaluated by Horner's rule, every product and
 // sum rounded to fp32, then an exact scaling by 2^n. x > 88 -> +inf, x < -87 -> 0.
@@ -53,34 +71,71 @@ __device__ __forceinline__ float dequant(int32_t acc, float s_row, float s_col) 
   return __fmul_rn(__fmul_rn(__int2float_rn(acc), s_row), s_col);
 }
 
+// Codes of 8 bf16 values (one 16-byte vector) packed into 8 bytes; inv = __frcp_rn(s).
+__device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t a = uint32_t(sym_code_fast(bf16_lo(w[j]), s, inv, 127)) & 0xFFu;
+    const uint32_t b = uint32_t(sym_code_fast(bf16_hi(w[j]), s, inv, 127)) & 0xFFu;
+    const uint32_t pair = a | (b << 8);
+    if (j < 2) lo |= pair << (16 * j); else hi |= pair << (16 * (j - 2));
+  }
+  return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float amax8(const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+  return m;
+}
+
 // Quantises one row of K bf16 values with one warp (K a multiple of 8, row 16-byte aligned):
-// returns the scale; `emit(i, packed8)` receives the 8 codes of elements i..i+7.
-template <typename Emit>
+// returns the scale; `emit(i, packed8)` receives the 8 codes of elements i..i+7. With U > 0 the
+// row (at most 256 * U values) is read once into registers, every load in flight together;
+// U = 0 reads rows of any length twice.
+template <int U, typename Emit>
 __device__ __forceinline__ float quant_row_warp(const uint16_t* __restrict__ src, int K, Emit emit) {
   const int lane = threadIdx.x & 31;
-  float amax = 0.0f;
-  for (int i = lane * 8; i < K; i += 256) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + i));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if constexpr (U > 0) {
+    uint4 v[U];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
-  }
-  amax = warp_max(amax);
-  const float s = sym_scale(amax, kQMaxInt8);
-  for (int i = lane * 8; i < K; i += 256) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + i));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t lo = 0, hi = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t a = uint32_t(sym_code(bf16_lo(w[j]), s, 127)) & 0xFFu;
-      const uint32_t b = uint32_t(sym_code(bf16_hi(w[j]), s, 127)) & 0xFFu;
-      const uint32_t pair = a | (b << 8);
-      if (j < 2) lo |= pair << (16 * j); else hi |= pair << (16 * (j - 2));
+    for (int u = 0; u < U; ++u) {
+      const int i = lane * 8 + u * 256;
+      v[u] = (i < K) ? __ldg(reinterpret_cast<const uint4*>(src + i)) : make_uint4(0, 0, 0, 0);
     }
-    emit(i, make_uint2(lo, hi));
+    float amax = 0.0f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) amax = fmaxf(amax, amax8(v[u]));
+    amax = warp_max(amax);
+    const float s = sym_scale(amax, kQMaxInt8);
+    const float inv = __frcp_rn(s);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = lane * 8 + u * 256;
+      if (i < K) emit(i, quant8(v[u], s, inv));
+    }
+    return s;
+  } else {
+    float amax = 0.0f;
+    for (int i = lane * 8; i < K; i += 256)
+      amax = fmaxf(amax, amax8(__ldg(reinterpret_cast<const uint4*>(src + i))));
+    amax = warp_max(amax);
+    const float s = sym_scale(amax, kQMaxInt8);
+    const float inv = __frcp_rn(s);
+    for (int i = lane * 8; i < K; i += 256)
+      emit(i, quant8(__ldg(reinterpret_cast<const uint4*>(src + i)), s, inv));
+    return s;
   }
-  return s;
+}
+
+// Registers-per-lane choice for a row of K values: 0 (two passes) beyond 4096.
+inline int row_units(int K) {
+  const int u = (K + 255) / 256;
+  return u <= 1 ? 1 : u <= 2 ? 2 : u <= 4 ? 4 : u <= 8 ? 8 : u <= 16 ? 16 : 0;
 }
 
 }  // namespace w8a8

@@ -1,0 +1,156 @@
+// Routing pieces shared by the tensor-core router epilogue and the small-batch router:
+// the warp-per-token top-k selection, the CUDA-core logits kernel for short batches and the
+// top-k kernel that consumes its output.
+#pragma once
+#include "numerics.cuh"
+
+namespace w8a8 {
+
+constexpr int kMaxTopK = 16;
+
+// Top-k routing of one token by one warp. Lane l holds experts l, l+32, ..., as order-preserving
+// integer keys of their logits (+ bias); each of the k rounds is two warp reductions: the
+// largest key, then the lowest expert holding it (equal logits go to the lower expert), and
+// the winner's lane drops that entry. Softmax over the picks (renorm) or over all E experts,
+// in fp32; lanes 0..k-1 store ids[j], w[j] and add to counts[e] when counts is given.
+// logit(e) returns the fp32 logit of expert e < PER * 32 (only called for e < E).
+template <int PER, typename Logit>
+__device__ __forceinline__ void warp_topk_token(Logit logit, int E, int k, bool renorm, const float* __restrict__ bias,
+                                                int* ids, float* w, int* counts) {
+  const int lane = threadIdx.x & 31;
+  float lv[PER];
+  uint32_t key[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    float l = 0.0f;
+    if (e < E) {
+      l = logit(e);
+      if (bias != nullptr) l += __ldg(bias + e);
+    }
+    lv[i] = l;
+    key[i] = (e < E) ? ordered_key(l) : 0u;  // 0: below every real logit, never picked
+  }
+  float pick_v = 0.0f, m = 0.0f;
+  int pick_e = -1;
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    uint32_t lbest = 0;
+    int li = 0;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i)  // downward, so the lowest expert wins among equals
+      if (key[i] >= lbest) { lbest = key[i]; li = i; }
+    const uint32_t wbest = warp_max_u32(lbest);
+    const uint32_t cand = (wbest != 0u && lbest == wbest) ? uint32_t(lane + 32 * li) : 0xFFFFFFFFu;
+    const uint32_t ebest = warp_min_u32(cand);
+    if (ebest != 0xFFFFFFFFu && int(ebest & 31u) == lane) {
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (i == int(ebest >> 5)) key[i] = 0u;
+    }
+    const float v = from_ordered_key(wbest);
+    if (j == 0) m = v;
+    if (lane == j) {
+      pick_v = v;
+      pick_e = (ebest == 0xFFFFFFFFu) ? -1 : int(ebest);
+    }
+  }
+  const float ev = (lane < k && pick_e >= 0) ? expf(pick_v - m) : 0.0f;
+  float denom = ev;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+  if (!renorm) {
+    float sall = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (lane + 32 * i < E) sall += expf(lv[i] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sall += __shfl_xor_sync(0xffffffffu, sall, o);
+    denom = sall;
+  }
+  if (lane < k) {
+    int e = pick_e;
+    if (e < 0) {  // only non-finite logits can leave a slot unfilled; report, never index
+      atomicOr(&g_error_word, kErrBadIndex);
+      e = lane;
+    }
+    ids[lane] = e;
+    w[lane] = ev / denom;
+    if (counts != nullptr) atomicAdd(counts + e, 1);
+  }
+}
+
+// Router logits on the CUDA cores for short batches: logits[t, e] = sum_h x[t, h] * wg[e, h] in
+// fp32 (bf16 inputs). Block = 8 warps; warp w takes expert blockIdx.x * 8 + w and the
+// kSmallRouterTokens tokens of blockIdx.y together (all their loads in flight at once, one
+// accumulator per token and vector slot); each lane holds its 1/32 of the expert's row
+// (H <= 256 * RU) in registers.
+constexpr int kSmallRouterTokens = 4;
+template <int RU>
+__global__ void __launch_bounds__(256) router_logits_small_kernel(const uint16_t* __restrict__ x,
+                                                                  const uint16_t* __restrict__ wg, int T, int H,
+                                                                  int E, float* __restrict__ logits) {
+  constexpr int TT = kSmallRouterTokens;
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (e >= E) return;
+  const int t0 = blockIdx.y * TT;
+  uint4 wv[RU];
+  uint4 xv[TT][RU];
+#pragma unroll
+  for (int u = 0; u < RU; ++u) {
+    const int i = lane * 8 + u * 256;
+    wv[u] = (i < H) ? __ldg(reinterpret_cast<const uint4*>(wg + size_t(e) * H + i)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      xv[t][u] = (i < H && t0 + t < T) ? __ldg(reinterpret_cast<const uint4*>(x + size_t(t0 + t) * H + i))
+                                       : make_uint4(0, 0, 0, 0);
+  }
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    float part[RU];
+#pragma unroll
+    for (int u = 0; u < RU; ++u) {
+      const uint32_t a[4] = {xv[t][u].x, xv[t][u].y, xv[t][u].z, xv[t][u].w};
+      const uint32_t b[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+      float s2 = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s2 = fmaf(bf16_lo(a[j]), bf16_lo(b[j]), s2);
+        s2 = fmaf(bf16_hi(a[j]), bf16_hi(b[j]), s2);
+      }
+      part[u] = s2;
+    }
+    float sum = 0.0f;
+#pragma unroll
+    for (int u = 0; u < RU; ++u) sum += part[u];
+    acc[t] = sum;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+  if (lane < TT && t0 + lane < T) {
+    float v = acc[0];
+#pragma unroll
+    for (int t = 1; t < TT; ++t) v = (lane == t) ? acc[t] : v;
+    logits[size_t(t0 + lane) * E + e] = v;
+  }
+}
+
+// Top-k over precomputed logits [T, E]: one warp per token. counts has one row of E per
+// 128-token chunk (count_stride = E) or a single row (count_stride = 0).
+template <int PER>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, const float* bias, int T,
+                                                          int E, int k, int renorm, int* ids, float* w, int* counts,
+                                                          int count_stride) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + size_t(t) * E;
+  int* crow = counts != nullptr ? counts + size_t(t / 128) * count_stride : nullptr;
+  warp_topk_token<PER>([&](int e) { return __ldg(row + e); }, E, k, renorm != 0, bias, ids + size_t(t) * k,
+                       w + size_t(t) * k, crow);
+}
+
+}  // namespace w8a8

@@ -75,10 +75,10 @@ bool make_kmajor_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner
 // ------------------------------------------------------------------ launch helpers
 int launch_status() { return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_LAUNCH; }
 
-template <int BN, int EPI, int KIND>
+template <int NA, int NB, int EPI, int KIND>
 int launch_gemm(const GemmParams& p, int max_tiles, cudaStream_t stream) {
-  using Cfg = GemmCfg<BN>;
-  auto kern = gemm_tc_kernel<BN, EPI, KIND>;
+  using Cfg = GemmCfg<NA, NB, EPI>;
+  auto kern = gemm_tc_kernel<NA, NB, EPI, KIND>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) !=
       cudaSuccess)
     return W8A8_ERR_LAUNCH;
@@ -131,31 +131,65 @@ void fill_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_
   L->s_h = take(sizeof(float) * Ap);
   L->hq = take(size_t(Ap) * I);
   L->o = take(size_t(A) * H * 2);
+  L->logits = take(sizeof(float) * T * E);
   L->total = off;
 }
 
 // Router: tcgen05 bf16 GEMM with the softmax / top-k epilogue. tile_counts is zeroed here.
 // counts: expert histogram rows (nullptr: none) with `count_stride` elements between the rows of
 // consecutive 128-token tiles (0: every tile adds into one row of E counters).
+// Short batches (T <= kSmallRouterMaxT): fp32 logits on the CUDA cores spread over many CTAs,
+// then a warp-per-token top-k; `logits` is T*E floats of scratch. Longer batches: the
+// tensor-core router with the top-k in its epilogue (logits unused).
+constexpr int64_t kSmallRouterMaxT = 512;
+
+int run_router_small(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t T, int64_t H, int64_t E,
+                     int k, int renorm, int* ids, float* w, int* counts, int64_t count_stride, float* logits,
+                     cudaStream_t stream) {
+  const dim3 grid1(unsigned((E + 7) / 8), unsigned((T + kSmallRouterTokens - 1) / kSmallRouterTokens));
+  switch (row_units(int(H))) {
+    case 1: router_logits_small_kernel<1><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
+    case 2: router_logits_small_kernel<2><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
+    case 4: router_logits_small_kernel<4><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
+    case 8: router_logits_small_kernel<8><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
+    case 16: router_logits_small_kernel<16><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
+    default: return W8A8_ERR_UNSUPPORTED;
+  }
+  int rc = launch_status();
+  if (rc != W8A8_OK) return rc;
+  const unsigned grid2 = unsigned((T + 7) / 8);
+  const int cs = int(count_stride);
+  switch ((E + 31) / 32) {
+    case 1: router_topk_kernel<1><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
+    case 2: router_topk_kernel<2><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
+    case 3:
+    case 4: router_topk_kernel<4><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
+    default: router_topk_kernel<8><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
+  }
+  return launch_status();
+}
+
 int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t T, int64_t H, int64_t E, int k,
-               int renorm, int* ids, float* w, int* counts, int64_t count_stride, cudaStream_t stream) {
-  const int bn = router_bn(E);
+               int renorm, int* ids, float* w, int* counts, int64_t count_stride, float* logits,
+               cudaStream_t stream) {
+  const int nb = router_bn(E);
   GemmParams p{};
-  if (!make_kmajor_map(&p.tmA, x, true, H, T, 128) || !make_kmajor_map(&p.tmB, wg, true, H, E, bn / 2))
+  if (!make_kmajor_map(&p.tmA, x, true, H, T, 128) || !make_kmajor_map(&p.tmB, wg, true, H, E, kBBoxRows) ||
+      !make_kmajor_map(&p.tmB2, wg, true, H, E, uint32_t(nb)))
     return W8A8_ERR_UNSUPPORTED;
   const int64_t C = (T + kChunk - 1) / kChunk;
   if (counts != nullptr) {
     const size_t rows = count_stride ? size_t(C) : 1;
     if (cudaMemsetAsync(counts, 0, sizeof(int) * rows * E, stream) != cudaSuccess) return W8A8_ERR_LAUNCH;
   }
+  if (logits != nullptr && T <= kSmallRouterMaxT && H <= 4096)
+    return run_router_small(x, wg, bias, T, H, E, k, renorm, ids, w, counts, count_stride, logits, stream);
   p.num_kb = int(H / 64);
-  p.n_tiles = 1;
+  p.n_cb = 1;
   p.num_groups = 1;
   p.group_offsets = nullptr;
   p.M = int(T);
-  p.b_rows_per_group = 0;
-  p.b_n_step = 0;
-  p.b_half_offset = bn / 2;
+  p.nb_fixed = nb;
   p.timeout_ns = wait_timeout_ns();
   p.out = ids;
   p.n_valid = int(E);
@@ -166,17 +200,53 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
   p.tile_counts = counts;
   p.tile_count_stride = int(count_stride);
   const int tiles = int(C);
-  switch (bn) {
-    case 16: return launch_gemm<16, kEpiRouter, kKindBF16>(p, tiles, stream);
-    case 32: return launch_gemm<32, kEpiRouter, kKindBF16>(p, tiles, stream);
-    case 64: return launch_gemm<64, kEpiRouter, kKindBF16>(p, tiles, stream);
-    case 128: return launch_gemm<128, kEpiRouter, kKindBF16>(p, tiles, stream);
-    default: return launch_gemm<256, kEpiRouter, kKindBF16>(p, tiles, stream);
+  switch (nb) {
+    case 16: return launch_gemm<1, 16, kEpiRouter, kKindBF16>(p, tiles, stream);
+    case 32: return launch_gemm<1, 32, kEpiRouter, kKindBF16>(p, tiles, stream);
+    case 64: return launch_gemm<1, 64, kEpiRouter, kKindBF16>(p, tiles, stream);
+    case 128: return launch_gemm<1, 128, kEpiRouter, kKindBF16>(p, tiles, stream);
+    default: return launch_gemm<1, 256, kEpiRouter, kKindBF16>(p, tiles, stream);
   }
 }
 
-// Upper bound of the number of 128-row tiles over all groups: ceil(A/128) + min(E, A).
-int max_m_tiles(int64_t A, int64_t E) { return int((A + kBM - 1) / kBM + (E < A ? E : A)); }
+// Launches quant_rows_kernel with the register depth that fits rows of K values.
+int launch_quant_rows(const uint16_t* src, int64_t R, int K, int8_t* q, float* scale, cudaStream_t s) {
+  const unsigned blocks = unsigned((R + kRowWarps - 1) / kRowWarps);
+  switch (row_units(K)) {
+    case 1: quant_rows_kernel<1><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+    case 2: quant_rows_kernel<2><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+    case 4: quant_rows_kernel<4><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+    case 8: quant_rows_kernel<8><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+    case 16: quant_rows_kernel<16><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+    default: quant_rows_kernel<0><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+  }
+  return launch_status();
+}
+
+int launch_group_quant(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* x, const int* ids,
+                       const int* tile_counts, int T, int H, int E, int k, int* offsets, int* perm, float* sx,
+                       float* sx_sorted, int8_t* xq) {
+  switch (row_units(H)) {
+#define W8A8_GQ(U_)                                                                                        \
+  case U_:                                                                                                 \
+    group_quant_kernel<U_><<<grid, kPermThreads, smem, s>>>(x, ids, tile_counts, T, H, E, k, offsets, perm, \
+                                                            sx, sx_sorted, xq);                            \
+    break;
+    W8A8_GQ(1) W8A8_GQ(2) W8A8_GQ(4) W8A8_GQ(8) W8A8_GQ(16) W8A8_GQ(0)
+#undef W8A8_GQ
+  }
+  return launch_status();
+}
+
+// Upper bound of the number of token blocks of `nb` rows over all groups: ceil(A/nb) + min(E, A).
+int max_token_blocks(int64_t A, int64_t E, int nb) { return int((A + nb - 1) / nb + (E < A ? E : A)); }
+
+// Token block of the expert GEMMs: 32 rows when experts see few tokens (decode), else 128.
+bool small_token_blocks(int64_t A, int64_t E) { return A <= 32 * E; }
+
+// CTAs per 128-token chunk of the grouping kernel: enough warps for every token of a small
+// batch, fewer for long ones (each CTA re-derives its chunk's positions).
+int group_quant_splits(int64_t T) { return T <= 1024 ? 8 : (T <= 4096 ? 4 : 2); }
 
 }  // namespace
 }  // namespace w8a8
@@ -219,9 +289,7 @@ int w8a8_quantize_weight_per_channel(const w8a8_bf16* w, int64_t G, int64_t N, i
   if (!w || !q || !scale) return W8A8_ERR_ARG;
   if (K % 8 || !aligned16(w) || (K % 16 && !aligned16(q)) || K > (1 << 30)) return W8A8_ERR_UNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(q) & 7u) return W8A8_ERR_UNSUPPORTED;
-  const int64_t blocks = (R + kRowWarps - 1) / kRowWarps;
-  quant_rows_kernel<<<unsigned(blocks), kRowWarps * 32, 0, as_stream(stream)>>>(w, R, int(K), q, scale);
-  return launch_status();
+  return launch_quant_rows(w, R, int(K), q, scale, as_stream(stream));
 }
 
 int w8a8_quantize_weight_int4_per_group(const w8a8_bf16* w, int64_t N, int64_t K, int group, uint8_t* packed,
@@ -246,9 +314,7 @@ int w8a8_quant_act_per_token(const w8a8_bf16* x, int64_t T, int64_t K, int8_t* q
   if (!x || !q || !scale) return W8A8_ERR_ARG;
   if (K % 8 || !aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 7u) || K > (1 << 30))
     return W8A8_ERR_UNSUPPORTED;
-  const int64_t blocks = (T + kRowWarps - 1) / kRowWarps;
-  quant_rows_kernel<<<unsigned(blocks), kRowWarps * 32, 0, as_stream(stream)>>>(x, T, int(K), q, scale);
-  return launch_status();
+  return launch_quant_rows(x, T, int(K), q, scale, as_stream(stream));
 }
 
 int w8a8_moe_route(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
@@ -264,7 +330,7 @@ int w8a8_moe_route(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, i
   if (!x || !wg || !topk_ids || !topk_w) return W8A8_ERR_ARG;
   if (!aligned16(x) || !aligned16(wg)) return W8A8_ERR_UNSUPPORTED;
   // every tile adds its tokens' experts into the single row expert_counts[E]
-  return run_router(x, wg, bias, T, H, E, k, renorm, topk_ids, topk_w, expert_counts, 0, as_stream(stream));
+  return run_router(x, wg, bias, T, H, E, k, renorm, topk_ids, topk_w, expert_counts, 0, nullptr, as_stream(stream));
 }
 
 int w8a8_moe_workspace_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_layout* layout) {
@@ -325,32 +391,32 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
 
   // 1. router (bf16 tcgen05 GEMM + softmax / top-k epilogue, per-chunk expert histogram)
   mark(ev, 0, s);
-  rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E, s);
+  rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E,
+                  reinterpret_cast<float*>(ws + L.logits), s);
   if (rc != W8A8_OK) return rc;
 
   // 2. group assignments by expert and quantise every token once into its sorted rows
-  const size_t gq_smem = sizeof(int) * (2 * E + kChunk * k);
+  const size_t gq_smem = sizeof(int) * (2 * E + 2 * kChunk * k + 4 * E);
   mark(ev, 1, s);
-  group_quant_kernel<<<C, kPermThreads, gq_smem, s>>>(x, ids, tile_counts, int(T), int(H), int(E), k, offsets,
-                                                      perm, sx, sx_sorted, xq);
-  if ((rc = launch_status()) != W8A8_OK) return rc;
+  rc = launch_group_quant(dim3(C, group_quant_splits(T)), gq_smem, s, x, ids, tile_counts, int(T), int(H), int(E),
+                          k, offsets, perm, sx, sx_sorted, xq);
+  if (rc != W8A8_OK) return rc;
 
-  // 3. grouped gate_up GEMM with the dequant + SiLU(gate)*up epilogue -> h
-  const bool wide = A >= 4096;  // prefill-sized batches use 256-wide tiles
+  // 3. grouped gate_up GEMM (weights on M, tokens on N) with the dequant + SiLU(gate)*up
+  //    epilogue -> h
+  const bool small = small_token_blocks(A, E);
+  const int nbt = small ? 32 : 128;
   {
     GemmParams p{};
-    const int bn = wide ? 256 : 128;
-    if (I % (bn / 2)) return W8A8_ERR_UNSUPPORTED;
-    if (!make_kmajor_map(&p.tmA, xq, false, H, Ap, 128) ||
-        !make_kmajor_map(&p.tmB, wgu, false, H, uint64_t(E) * 2 * I, bn / 2))
+    if (!make_kmajor_map(&p.tmA, wgu, false, H, uint64_t(E) * 2 * I, 128) ||
+        !make_kmajor_map(&p.tmB, xq, false, H, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, xq, false, H, Ap, nbt))
       return W8A8_ERR_UNSUPPORTED;
     p.num_kb = int(H / 128);
-    p.n_tiles = int(I / (bn / 2));
+    p.n_cb = int(I / 128);
     p.num_groups = int(E);
     p.group_offsets = offsets;
-    p.b_rows_per_group = int(2 * I);
-    p.b_n_step = bn / 2;
-    p.b_half_offset = int(I);
+    p.a_rows_per_group = int(2 * I);
+    p.a_second_offset = int(I);
     p.timeout_ns = wait_timeout_ns();
     p.out = h;
     p.ldo = int(I);
@@ -358,46 +424,41 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     p.col_scale = s_gu;
     p.col_scale_stride = int(2 * I);
     p.up_offset = int(I);
-    const int tiles = max_m_tiles(A, E) * p.n_tiles;
+    const int tiles = max_token_blocks(A, E, nbt) * p.n_cb;
     mark(ev, 2, s);
-    rc = wide ? launch_gemm<256, kEpiGateUp, kKindI8>(p, tiles, s) : launch_gemm<128, kEpiGateUp, kKindI8>(p, tiles, s);
+    rc = small ? launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, tiles, s)
+               : launch_gemm<2, 128, kEpiGateUp, kKindI8>(p, tiles, s);
     if (rc != W8A8_OK) return rc;
   }
 
   // 4. per-row requantisation of h
   {
-    const int64_t blocks = (A + kRowWarps - 1) / kRowWarps;
     mark(ev, 3, s);
-    quant_rows_kernel<<<unsigned(blocks), kRowWarps * 32, 0, s>>>(h, A, int(I), hq, s_h);
-    if ((rc = launch_status()) != W8A8_OK) return rc;
+    if ((rc = launch_quant_rows(h, A, int(I), hq, s_h, s)) != W8A8_OK) return rc;
   }
 
   // 5. grouped down GEMM with the dequant epilogue -> o in slot order
   {
     GemmParams p{};
-    const int bn = wide ? 256 : 128;
-    if (H % bn) return W8A8_ERR_UNSUPPORTED;
-    if (!make_kmajor_map(&p.tmA, hq, false, I, Ap, 128) ||
-        !make_kmajor_map(&p.tmB, wd, false, I, uint64_t(E) * H, bn / 2))
+    if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(E) * H, 128) ||
+        !make_kmajor_map(&p.tmB, hq, false, I, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, hq, false, I, Ap, nbt))
       return W8A8_ERR_UNSUPPORTED;
     p.num_kb = int(I / 128);
-    p.n_tiles = int(H / bn);
+    p.n_cb = int(H / 128);
     p.num_groups = int(E);
     p.group_offsets = offsets;
-    p.b_rows_per_group = int(H);
-    p.b_n_step = bn;
-    p.b_half_offset = bn / 2;
+    p.a_rows_per_group = int(H);
     p.timeout_ns = wait_timeout_ns();
     p.out = o;
     p.ldo = int(H);
-    p.out_col_step = bn;
     p.row_scale = s_h;
     p.col_scale = s_d;
     p.col_scale_stride = int(H);
     p.row_map = perm;
-    const int tiles = max_m_tiles(A, E) * p.n_tiles;
+    const int tiles = max_token_blocks(A, E, nbt) * p.n_cb;
     mark(ev, 4, s);
-    rc = wide ? launch_gemm<256, kEpiDown, kKindI8>(p, tiles, s) : launch_gemm<128, kEpiDown, kKindI8>(p, tiles, s);
+    rc = small ? launch_gemm<1, 32, kEpiDown, kKindI8>(p, tiles, s)
+               : launch_gemm<1, 128, kEpiDown, kKindI8>(p, tiles, s);
     if (rc != W8A8_OK) return rc;
   }
 
@@ -509,32 +570,20 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
   int rc = w8a8_quant_act_per_token(x, M, K, xq, sx, stream);
   if (rc != W8A8_OK) return rc;
   GemmParams p{};
-  if (!make_kmajor_map(&p.tmA, xq, false, K, Mp, 128) || !make_kmajor_map(&p.tmB, wq, false, K, N, 128))
+  if (!make_kmajor_map(&p.tmA, wq, false, K, N, 128) || !make_kmajor_map(&p.tmB, xq, false, K, Mp, kBBoxRows) ||
+      !make_kmajor_map(&p.tmB2, xq, false, K, Mp, 128))
     return W8A8_ERR_UNSUPPORTED;
   p.num_kb = int(K / 128);
-  p.n_tiles = int(N / 256);
+  p.n_cb = int(N / 128);
   p.num_groups = 1;
   p.M = int(M);
-  p.b_n_step = 256;
-  p.b_half_offset = 128;
   p.timeout_ns = wait_timeout_ns();
   p.out = y;
   p.ldo = int(N);
-  p.out_col_step = 256;
   p.row_scale = sx;
   p.col_scale = sw;
-  if (N % 256 == 0) {
-    const int tiles = int((M + 127) / 128) * p.n_tiles;
-    return launch_gemm<256, kEpiDense, kKindI8>(p, tiles, s);
-  }
-  // N % 128 == 0: 128-wide tiles
-  if (!make_kmajor_map(&p.tmB, wq, false, K, N, 64)) return W8A8_ERR_UNSUPPORTED;
-  p.n_tiles = int(N / 128);
-  p.b_n_step = 128;
-  p.b_half_offset = 64;
-  p.out_col_step = 128;
-  const int tiles = int((M + 127) / 128) * p.n_tiles;
-  return launch_gemm<128, kEpiDense, kKindI8>(p, tiles, s);
+  const int tiles = int((M + 127) / 128) * p.n_cb;
+  return launch_gemm<1, 128, kEpiDense, kKindI8>(p, tiles, s);
 }
 
 int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
@@ -544,21 +593,20 @@ int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, i
   if (M == 0) return W8A8_OK;
   if (!a || !b || !c) return W8A8_ERR_ARG;
   if (!aligned16(a) || !aligned16(b) || !aligned16(c) || M >= (int64_t(1) << 30)) return W8A8_ERR_UNSUPPORTED;
+  // channels (rows of b) on the MMA M side, rows of a on N
   GemmParams p{};
-  if (!make_kmajor_map(&p.tmA, a, false, K, M, 128) || !make_kmajor_map(&p.tmB, b, false, K, N, 64))
+  if (!make_kmajor_map(&p.tmA, b, false, K, N, 128) || !make_kmajor_map(&p.tmB, a, false, K, M, kBBoxRows) ||
+      !make_kmajor_map(&p.tmB2, a, false, K, M, 128))
     return W8A8_ERR_UNSUPPORTED;
   p.num_kb = int(K / 128);
-  p.n_tiles = int(N / 128);
+  p.n_cb = int(N / 128);
   p.num_groups = 1;
   p.M = int(M);
-  p.b_n_step = 128;
-  p.b_half_offset = 64;
   p.timeout_ns = wait_timeout_ns();
   p.out = c;
   p.ldo = int(N);
-  p.out_col_step = 128;
-  const int tiles = int((M + 127) / 128) * p.n_tiles;
-  return launch_gemm<128, kEpiRawS32, kKindI8>(p, tiles, as_stream(stream));
+  const int tiles = int((M + 127) / 128) * p.n_cb;
+  return launch_gemm<1, 128, kEpiRawS32, kKindI8>(p, tiles, as_stream(stream));
 }
 
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {
