@@ -188,6 +188,29 @@ def test_linear_w8a8_exact(M, K, N):
     np.testing.assert_array_equal(G.host(y), O.linear_w8a8(x, oq, os_))
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 128, 128), (200, 512, 384), (77, 1024, 256), (2048, 2048, 6144)])
+def test_linear_w4a8_exact(M, K, N):
+    x = synth.activations(M, K, max(1, K // 100), seed=M + 1)
+    w = synth.dense_weight(N, K, seed=N + 1)
+    packed, s = B.w8a8_quantize_weight_int4_per_group(G.bf16_dev(w), 128)
+    y = B.w8a8_linear(G.bf16_dev(x), packed, s, B.W8A8_W_INT4_PER_GROUP, 128)
+    op, os_ = O.quantize_weight_int4_per_group(w, 128)
+    np.testing.assert_array_equal(packed.cpu().numpy(), op)
+    np.testing.assert_array_equal(G.host(y), O.linear_w4a8(x, op, os_, 128))
+
+
+def test_linear_w4a8_extreme_codes():
+    # every nibble pattern the quantiser can produce, including -7 and +7 everywhere
+    M, K, N = 130, 256, 128
+    x = O.f32_to_bf16(np.where(np.arange(M * K).reshape(M, K) % 3 == 0, -127.0, 127.0).astype(np.float32))
+    wv = np.tile(np.array([7, -7, 1, -1, 0, 3, -3, 5], np.float32), (N, K // 8))
+    w = O.f32_to_bf16(wv * np.float32(0.01))
+    packed, s = B.w8a8_quantize_weight_int4_per_group(G.bf16_dev(w), 128)
+    y = B.w8a8_linear(G.bf16_dev(x), packed, s, B.W8A8_W_INT4_PER_GROUP, 128)
+    op, os_ = O.quantize_weight_int4_per_group(w, 128)
+    np.testing.assert_array_equal(G.host(y), O.linear_w4a8(x, op, os_, 128))
+
+
 # ------------------------------------------------------------------ failure detection
 def test_bounded_wait_reports_timeout_and_context_survives():
     B.w8a8_debug_wait_timeout(2_000_000)  # 2 ms

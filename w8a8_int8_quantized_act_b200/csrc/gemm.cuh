@@ -49,7 +49,9 @@ struct GemmParams {
   const int* group_offsets;    // [G+1] token-row offsets (device); nullptr: one group of M rows
   int M;                       // token rows when group_offsets is null
   int a_rows_per_group;        // weight rows per group (gate_up: 2I, down: H, dense: 0)
-  int a_second_offset;         // gate_up: row offset of the up block (I)
+  int a_second_offset;         // row offset of the second A block (gate_up: I; wide tiles: 128)
+  int a_cb_step;               // A rows per channel block (128, or 256 with two 128-row blocks)
+  int n_channels;              // valid output channels per group (second blocks past it are skipped)
   int nb_fixed;                // router: N side rows (E rounded up to 16); else 0
   uint64_t timeout_ns;         // bound on every mbarrier wait
   // epilogue operands
@@ -145,7 +147,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* mt_p
     }
     c.tok0 = off + blk * NB;
     c.rows = min(NB, cnt - blk * NB);
-    c.a_row = c.g * p.a_rows_per_group + c.cb * kBM;
+    c.a_row = c.g * p.a_rows_per_group + c.cb * p.a_cb_step;
     c.b_row = c.tok0;
     c.nb = (c.rows + 15) & ~15;
   }
@@ -171,7 +173,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 template <int EPI, int NB>
 __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Tile& c, uint32_t t_lane, int lane_ch,
                                                   int half) {
-  const int ch = c.cb * kBM + lane_ch;  // channel within the group
+  const int ch = c.cb * p.a_cb_step + lane_ch;  // channel within the group
   const size_t ldo = size_t(p.ldo);
   const float* __restrict__ row_scale = p.row_scale;
   uint32_t r[16];
@@ -196,30 +198,45 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
       }
     }
   } else if constexpr (EPI == kEpiDown || EPI == kEpiDense) {
-    const float sc = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+    // two 128-channel blocks: accumulator columns [0, NB) and [NB, 2NB)
+    const bool second = ch + kBM < p.n_channels;
+    const float sc0 = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+    const float sc1 = second ? __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch + kBM) : 0.0f;
     const int* __restrict__ row_map = p.row_map;
     uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
+    uint32_t r1[16];
 #pragma unroll 1
     for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
       tmem_ld16(t_lane + j0, r);
+      tmem_ld16(t_lane + NB + j0, r1);
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         if (j0 + j < c.rows) {
           const int row = c.tok0 + j0 + j;
           const int orow = (EPI == kEpiDown) ? __ldg(row_map + row) : row;
-          const float v = dequant(int32_t(r[j]), __ldg(row_scale + row), sc);
-          out[size_t(orow) * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+          const float srow = __ldg(row_scale + row);
+          uint16_t* o = out + size_t(orow) * ldo;
+          o[0] = __bfloat16_as_ushort(__float2bfloat16_rn(dequant(int32_t(r[j]), srow, sc0)));
+          if (second) o[kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(dequant(int32_t(r1[j]), srow, sc1)));
         }
       }
     }
   } else if constexpr (EPI == kEpiRawS32) {
     int32_t* out = static_cast<int32_t*>(p.out) + ch;
+    const bool second = ch + kBM < p.n_channels;
+    uint32_t r1[16];
 #pragma unroll 1
     for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
       tmem_ld16(t_lane + j0, r);
+      tmem_ld16(t_lane + NB + j0, r1);
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (j0 + j < c.rows) out[size_t(c.tok0 + j0 + j) * ldo] = int32_t(r[j]);
+      for (int j = 0; j < 16; ++j) {
+        if (j0 + j < c.rows) {
+          int32_t* o = out + size_t(c.tok0 + j0 + j) * ldo;
+          o[0] = int32_t(r[j]);
+          if (second) o[kBM] = int32_t(r1[j]);
+        }
+      }
     }
   }
 }

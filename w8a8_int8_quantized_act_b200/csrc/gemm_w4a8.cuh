@@ -1,0 +1,281 @@
+// Dense W4A8 linear on the 5th-generation tensor cores (sm_100a):
+//
+//   y[t, n] = bf16( s_x[t] * sum_g (float)acc_g[t, n] * s_w[n, g] )
+//   acc_g[t, n] = sum over the g-th group of 128 K values of xq[t, k] * w[n, k]   (int32)
+//
+// The weights arrive as 4-bit two's-complement codes, two per byte (even k in the low nibble),
+// with one fp32 scale per (output channel, group of 128 along K) ("4bit 权重" section of the
+// Qwen3-1.7B-W4A8 page). One 128-byte K-block of int8 is exactly one scale group, so the int32
+// partial of each group is read out of TMEM and scaled on its own.
+// Roles per CTA (one CTA per SM, 14 warps), tile = 128 channels (MMA M) x NB tokens (MMA N):
+//   warp 0      TMA producer: packed weight tile (128 rows x 64 bytes, no swizzle) into a
+//               staging slot, token rows (128-byte swizzled, like the int8 GEMMs);
+//   warp 1      TMEM allocator and MMA issuer: one tcgen05.mma kind::i8 group per K-block into
+//               alternating TMEM buffers;
+//   warps 2-5   converters: sign-extend the nibbles to int8 and write them in the 128-byte
+//               swizzled K-major layout the MMA reads, then fence the async proxy;
+//   warps 6-13  epilogue: per K-block, add (float)acc_g * s_w[n, g] (fp32, product and sum each
+//               rounded) into registers; at the tile's end store bf16(acc * s_x[t]).
+#pragma once
+#include "gemm.cuh"
+
+namespace w8a8 {
+
+constexpr int kW4Threads = 64 + 128 + 32 * kEpiWarps;
+
+struct W4A8Params {
+  CUtensorMap tmW;   // packed weights [N, K/2] bytes, box 128 rows x 64 bytes, no swizzle
+  CUtensorMap tmX;   // xq [Mp, K] int8, box 16 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap tmX2;  // xq, box NB rows (full token tiles)
+  int num_kb;        // K / 128 (= number of scale groups)
+  int n_cb;          // N / 128
+  int M;             // tokens
+  int N;
+  const float* sw;   // [N, num_kb]
+  const float* sx;   // [M]
+  uint16_t* y;       // [M, N] bf16
+  uint64_t timeout_ns;
+};
+
+template <int NB>
+struct W4Cfg {
+  static constexpr int kPackedBytes = kBM * 64;
+  static constexpr int kABytes = kBM * kKBlockBytes;
+  static constexpr int kBBytes = NB * kKBlockBytes;
+  static constexpr int kStageBytes = kPackedBytes + kABytes + kBBytes;
+  static constexpr int kStages = (192 * 1024) / kStageBytes > 8 ? 8 : (192 * 1024) / kStageBytes;
+  static constexpr int kTmemCols = (2 * NB <= 64) ? 64 : (2 * NB <= 128 ? 128 : (2 * NB <= 256 ? 256 : 512));
+  static constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + 512;
+  static_assert(kStages >= 2, "pipeline too shallow");
+};
+
+// 8 packed bytes (16 int4 codes) -> 16 sign-extended int8 codes in k order.
+__device__ __forceinline__ uint4 unpack_int4x16(uint2 pk) {
+  const uint32_t w[2] = {pk.x, pk.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t lo = __vsub4((w[i] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);         // even k
+    const uint32_t hi = __vsub4(((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);  // odd k
+    o[2 * i] = __byte_perm(lo, hi, 0x5140);      // l0 h0 l1 h1
+    o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);  // l2 h2 l3 h3
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_constant__ W4A8Params p) {
+  using Cfg = W4Cfg<NB>;
+  constexpr int STAGES = Cfg::kStages;
+  constexpr uint32_t IDESC0 = idesc_s8s8s32(0);
+  constexpr int HALFC = NB / 2;  // token columns per epilogue warp
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes);
+  uint64_t* conv = full + STAGES;
+  uint64_t* empty = conv + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const WaitCtx wc{abort_flag, globaltimer_ns() + p.timeout_ns};
+  auto packed_of = [&](int s) { return smem + s * Cfg::kStageBytes; };
+  auto a_of = [&](int s) { return smem + s * Cfg::kStageBytes + Cfg::kPackedBytes; };
+  auto b_of = [&](int s) { return smem + s * Cfg::kStageBytes + Cfg::kPackedBytes + Cfg::kABytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(conv + s, 128);
+      mbar_init(empty + s, 1);
+    }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, kEpiWarps * 32); }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+    tma_prefetch_map(&p.tmW);
+    tma_prefetch_map(&p.tmX);
+    tma_prefetch_map(&p.tmX2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int m_tiles = (p.M + NB - 1) / NB;
+  const int total_tiles = m_tiles * p.n_cb;
+  const int nkb = p.num_kb;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
+        const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+        const int tok0 = mt * NB, rows = min(NB, p.M - tok0), nb = (rows + 15) & ~15;
+        const uint32_t bytes = uint32_t(Cfg::kPackedBytes + nb * kKBlockBytes);
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+          mbar_arrive_expect_tx(full + stage, bytes);
+          tma_load_2d(packed_of(stage), &p.tmW, full + stage, kb * 64, cb * kBM);
+          if (nb == NB) {
+            tma_load_2d(b_of(stage), &p.tmX2, full + stage, kb * 128, tok0);
+          } else {
+            for (int b = 0; b < nb; b += kBBoxRows)
+              tma_load_2d(b_of(stage) + b * kKBlockBytes, &p.tmX, full + stage, kb * 128, tok0 + b);
+          }
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        volatile int no_abort = 0;
+        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+        const int mt = tile / p.n_cb;
+        const int rows = min(NB, p.M - mt * NB), nb = (rows + 15) & ~15;
+        const uint32_t idesc = IDESC0 | (uint32_t(nb >> 3) << 17);
+        bool ok = true;
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+          // one scale group per K-block: a fresh accumulator in the free TMEM buffer
+          if (!mbar_wait(tempty + acc, acc_phase ^ 1u, wc)) { ok = false; break; }
+          if (!mbar_wait(conv + stage, phase, wc)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + uint32_t(acc * NB);
+          const uint32_t a0 = smem_addr(a_of(stage));
+          const uint32_t b0 = smem_addr(b_of(stage));
+#pragma unroll
+          for (int kk = 0; kk < kKBlockBytes / 32; ++kk)
+            tc_mma<kKindI8>(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
+                            kk != 0 ? 1u : 0u);
+          issued_any = true;
+          tc_commit(empty + stage);
+          tc_commit(tfull + acc);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag && issued_any) {
+        tc_commit(drain);
+        volatile int no_abort = 0;
+        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+        mbar_wait(drain, 0, dw);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ converters (warps 2..5)
+    const int ct = threadIdx.x - 64;  // 0..127
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(full + stage, phase, wc)) { ok = false; break; }
+        const uint8_t* src = packed_of(stage);
+        uint8_t* dst = a_of(stage);
+        // 128 rows x 64 packed bytes: item = (row, 16-byte packed chunk) -> two 16-byte int8 chunks
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int item = ct + 128 * q;
+          const int r = item >> 2, pch = item & 3;
+          const uint4 pk = *reinterpret_cast<const uint4*>(src + r * 64 + pch * 16);
+          const uint4 o0 = unpack_int4x16(make_uint2(pk.x, pk.y));
+          const uint4 o1 = unpack_int4x16(make_uint2(pk.z, pk.w));
+          const int c0 = 2 * pch, c1 = 2 * pch + 1;  // logical 16-byte chunks of the int8 row
+          *reinterpret_cast<uint4*>(dst + r * 128 + ((c0 ^ (r & 7)) << 4)) = o0;
+          *reinterpret_cast<uint4*>(dst + r * 128 + ((c1 ^ (r & 7)) << 4)) = o1;
+        }
+        fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
+        mbar_arrive(conv + stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 6..13)
+    const int q = warp & 3;
+    const int half = (warp - 6) >> 2;
+    const int ch = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      const int tok0 = mt * NB, rows = min(NB, p.M - tok0);
+      const int n = cb * kBM + ch;
+      const int j0 = half * HALFC;  // this warp's token columns [j0, j0 + HALFC)
+      float accf[HALFC];
+#pragma unroll
+      for (int j = 0; j < HALFC; ++j) accf[j] = 0.0f;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const float s = __ldg(p.sw + size_t(n) * nkb + kb);
+        if (!mbar_wait(tfull + acc, acc_phase, wc)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * NB);
+        if (j0 < rows) {
+#pragma unroll
+          for (int c16 = 0; c16 < HALFC; c16 += 16) {
+            uint32_t r[16];
+            tmem_ld16(t_lane + j0 + c16, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              accf[c16 + i] = __fadd_rn(accf[c16 + i], __fmul_rn(__int2float_rn(int32_t(r[i])), s));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty + acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) break;
+      uint16_t* out = p.y + n;
+#pragma unroll
+      for (int j = 0; j < HALFC; ++j) {
+        const int t = j0 + j;
+        if (t < rows)
+          out[size_t(tok0 + t) * p.N] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(accf[j], __ldg(p.sx + tok0 + t))));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace w8a8

@@ -9,6 +9,7 @@
 #include "../../include/w8a8.h"
 #include "elementwise.cuh"
 #include "gemm.cuh"
+#include "gemm_w4a8.cuh"
 
 namespace w8a8 {
 namespace {
@@ -70,6 +71,20 @@ bool make_kmajor_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over [rows, inner_bytes] bytes with an unswizzled (box_rows x box_bytes) box.
+bool make_plain_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint32_t box_bytes,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || inner_bytes == 0) return false;
+  const cuuint64_t dims[2] = {inner_bytes, rows};
+  const cuuint64_t strides[1] = {inner_bytes};
+  const cuuint32_t box[2] = {box_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------------ launch helpers
@@ -417,6 +432,7 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     p.group_offsets = offsets;
     p.a_rows_per_group = int(2 * I);
     p.a_second_offset = int(I);
+    p.a_cb_step = 128;
     p.timeout_ns = wait_timeout_ns();
     p.out = h;
     p.ldo = int(I);
@@ -444,10 +460,13 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
         !make_kmajor_map(&p.tmB, hq, false, I, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, hq, false, I, Ap, nbt))
       return W8A8_ERR_UNSUPPORTED;
     p.num_kb = int(I / 128);
-    p.n_cb = int(H / 128);
+    p.n_cb = int((H + 255) / 256);
+    p.n_channels = int(H);
     p.num_groups = int(E);
     p.group_offsets = offsets;
     p.a_rows_per_group = int(H);
+    p.a_second_offset = 128;
+    p.a_cb_step = 256;
     p.timeout_ns = wait_timeout_ns();
     p.out = o;
     p.ldo = int(H);
@@ -457,8 +476,8 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     p.row_map = perm;
     const int tiles = max_token_blocks(A, E, nbt) * p.n_cb;
     mark(ev, 4, s);
-    rc = small ? launch_gemm<1, 32, kEpiDown, kKindI8>(p, tiles, s)
-               : launch_gemm<1, 128, kEpiDown, kKindI8>(p, tiles, s);
+    rc = small ? launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s)
+               : launch_gemm<2, 128, kEpiDown, kKindI8>(p, tiles, s);
     if (rc != W8A8_OK) return rc;
   }
 
@@ -560,8 +579,8 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
   if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
   if (!aligned16(x) || !aligned16(wq) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return W8A8_ERR_UNSUPPORTED;
+  if (w_format == W8A8_W_INT4_PER_GROUP && (K / 128) > (int64_t(1) << 20)) return W8A8_ERR_UNSUPPORTED;
   if (M >= (int64_t(1) << 30) || N * K >= (int64_t(1) << 40)) return W8A8_ERR_UNSUPPORTED;
-  if (w_format != W8A8_W_INT8_PER_CHANNEL) return W8A8_ERR_UNSUPPORTED;  // int4 path: not yet built
   const int64_t Mp = round_up(M, 128);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int8_t* xq = reinterpret_cast<int8_t*>(ws);
@@ -569,21 +588,45 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
   cudaStream_t s = as_stream(stream);
   int rc = w8a8_quant_act_per_token(x, M, K, xq, sx, stream);
   if (rc != W8A8_OK) return rc;
+  if (w_format == W8A8_W_INT4_PER_GROUP) {
+    W4A8Params q{};
+    if (!make_plain_map(&q.tmW, wq, uint64_t(K / 2), uint64_t(N), 64, 128) ||
+        !make_kmajor_map(&q.tmX, xq, false, K, Mp, kBBoxRows) || !make_kmajor_map(&q.tmX2, xq, false, K, Mp, 128))
+      return W8A8_ERR_UNSUPPORTED;
+    q.num_kb = int(K / 128);
+    q.n_cb = int(N / 128);
+    q.M = int(M);
+    q.N = int(N);
+    q.sw = sw;
+    q.sx = sx;
+    q.y = y;
+    q.timeout_ns = wait_timeout_ns();
+    using Cfg = W4Cfg<128>;
+    auto kern = w4a8_gemm_kernel<128>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) != cudaSuccess)
+      return W8A8_ERR_LAUNCH;
+    const int tiles = int((M + 127) / 128) * q.n_cb;
+    kern<<<max(1, min(num_sms(), tiles)), kW4Threads, Cfg::kSmemBytes, s>>>(q);
+    return launch_status();
+  }
   GemmParams p{};
   if (!make_kmajor_map(&p.tmA, wq, false, K, N, 128) || !make_kmajor_map(&p.tmB, xq, false, K, Mp, kBBoxRows) ||
       !make_kmajor_map(&p.tmB2, xq, false, K, Mp, 128))
     return W8A8_ERR_UNSUPPORTED;
   p.num_kb = int(K / 128);
-  p.n_cb = int(N / 128);
+  p.n_cb = int((N + 255) / 256);
+  p.n_channels = int(N);
   p.num_groups = 1;
   p.M = int(M);
+  p.a_second_offset = 128;
+  p.a_cb_step = 256;
   p.timeout_ns = wait_timeout_ns();
   p.out = y;
   p.ldo = int(N);
   p.row_scale = sx;
   p.col_scale = sw;
   const int tiles = int((M + 127) / 128) * p.n_cb;
-  return launch_gemm<1, 128, kEpiDense, kKindI8>(p, tiles, s);
+  return launch_gemm<2, 128, kEpiDense, kKindI8>(p, tiles, s);
 }
 
 int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
@@ -599,14 +642,17 @@ int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, i
       !make_kmajor_map(&p.tmB2, a, false, K, M, 128))
     return W8A8_ERR_UNSUPPORTED;
   p.num_kb = int(K / 128);
-  p.n_cb = int(N / 128);
+  p.n_cb = int((N + 255) / 256);
+  p.n_channels = int(N);
   p.num_groups = 1;
   p.M = int(M);
+  p.a_second_offset = 128;
+  p.a_cb_step = 256;
   p.timeout_ns = wait_timeout_ns();
   p.out = c;
   p.ldo = int(N);
   const int tiles = int((M + 127) / 128) * p.n_cb;
-  return launch_gemm<1, 128, kEpiRawS32, kKindI8>(p, tiles, as_stream(stream));
+  return launch_gemm<2, 128, kEpiRawS32, kKindI8>(p, tiles, as_stream(stream));
 }
 
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {
