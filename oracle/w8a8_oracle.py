@@ -35,13 +35,15 @@ Readings where the pages are silent (each one is fixed identically on the GPU si
   the k weights are renormalised to sum to 1 when ``renorm`` is set (Qwen3-MoE default).
 * The gated activation is SiLU(gate) * up (the pages name gate/up/down projections but not
   the function). SiLU uses ``spec_exp``, an exponential defined below step by step so that
-  both sides produce the same bits.
+  both sides produce the same bits; its polynomial is evaluated with fused multiply-adds.
 * Dequantisation is ((float)acc * s_token) * s_channel, two fp32 round-to-nearest products.
 * h is rounded to bf16 before its per-row requantisation; o is rounded to bf16.
-* Combine: acc = 0; for j in 0..k-1: acc = acc + (w[t,j] * o[t,j,n]), each product and
-  each sum rounded to fp32; y = bf16(acc).
-* W4A8: y = bf16(acc_f * s_token) where acc_f = sum over K-groups g, in order, of
-  (float)acc_g * s_w[n, g], each product and sum rounded to fp32.
+* Combine: acc = 0; for j in 0..k-1: acc = fma(w[t,j], o[t,j,n], acc) (one fp32 rounding
+  per step); y = bf16(acc).
+* W4A8: y = bf16(acc_f * s_token) where acc_f = fma((float)acc_g, s_w[n, g], acc_f) over the
+  K-groups g in order.
+* fma(a, b, c) is the fp32 fused multiply-add: a*b + c rounded once. numpy has none, so
+  ``fma32`` computes it exactly from float64 arithmetic (see there).
 """
 from __future__ import annotations
 
@@ -70,6 +72,28 @@ def f32_to_bf16(v: np.ndarray) -> np.ndarray:
     b = np.asarray(v, dtype=np.float32).view(np.uint32).astype(np.uint64)
     b = b + np.uint64(0x7FFF) + ((b >> np.uint64(16)) & np.uint64(1))
     return (b >> np.uint64(16)).astype(np.uint16)
+
+
+def fma32(a, b, c) -> np.ndarray:
+    """fp32 fused multiply-add round(a*b + c), computed exactly from float64 arithmetic.
+
+    a*b of two fp32 values is exact in float64. The sum with c is taken in float64 and then
+    made "round to odd" (Boldo & Melquiond, 2008): when the float64 sum s is inexact (its
+    TwoSum error is non-zero) and its last bit is even, s moves one ulp toward the error.
+    Rounding that round-to-odd float64 to fp32 gives the correctly rounded result, because
+    float64's 53 bits exceed fp32's 24 by more than the 2 bits the theorem needs.
+    """
+    a = np.asarray(a, np.float32).astype(np.float64)
+    b = np.asarray(b, np.float32).astype(np.float64)
+    c = np.asarray(c, np.float32).astype(np.float64)
+    p = a * b
+    s = p + c
+    bb = s - p
+    err = (p - (s - bb)) + (c - bb)
+    even = (np.asarray(s).view(np.int64) & 1) == 0
+    toward = np.where(err > 0, np.inf, -np.inf)
+    s = np.where((err != 0) & even, np.nextafter(s, toward), s)
+    return np.asarray(s).astype(np.float32)
 
 
 # --------------------------------------------------------------------------------------
@@ -178,18 +202,18 @@ EXP_LO = np.float32(-87.0)
 def spec_exp(x: np.ndarray) -> np.ndarray:
     """exp(x) in fp32 by Cody-Waite range reduction and a degree-7 Taylor polynomial.
 
-    n = rint(x * log2(e)); r = (x - n*LN2_HI) - n*LN2_LO; p = sum_{i<=7} r^i / i! by Horner
-    (each product and each sum rounded to fp32); result = p * 2^n (exact scaling).
-    x > 88 gives +inf, x < -87 gives 0. Error is within a few ulp of the true exponential.
+    n = rint(x * log2(e)) (fp32 product); r = fma(-n, LN2_LO, fma(-n, LN2_HI, x));
+    p = sum_{i<=7} r^i / i! by Horner with fused multiply-adds, p = fma(p, r, 1/i!);
+    result = p * 2^n (exact scaling). x > 88 gives +inf, x < -87 gives 0. Error is within a
+    few ulp of the true exponential.
     """
     x = np.asarray(x, dtype=np.float32)
     xc = np.clip(x, EXP_LO, EXP_HI)
     n = np.rint(xc * LOG2E).astype(np.float32)
-    r = (xc - n * LN2_HI) - n * LN2_LO
-    p = TAYLOR[7]
+    r = fma32(-n, LN2_LO, fma32(-n, LN2_HI, xc))
+    p = np.full(x.shape, TAYLOR[7], np.float32)
     for c in TAYLOR[6::-1]:
-        p = p * r + c
-    p = np.asarray(p, dtype=np.float32)
+        p = fma32(p, r, c)
     two_n = ((n.astype(np.int32) + 127).astype(np.uint32) << np.uint32(23)).view(np.float32)
     out = p * two_n
     out = np.where(x > EXP_HI, np.float32(np.inf), out)
@@ -286,13 +310,13 @@ def gated_activation(acc_gu: np.ndarray, s_row: np.ndarray, s_gu: np.ndarray) ->
 
 
 def combine(o_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
-    """y[t] = bf16(sum_j w[t, j] * o[t, j]) with fp32 products and sums in slot order."""
+    """y[t] = bf16(sum_j w[t, j] * o[t, j]): fp32 fused multiply-adds in slot order from 0."""
     o = bf16_to_f32(o_bits)
     T, k, H = o.shape
     acc = np.zeros((T, H), np.float32)
     w = np.asarray(w, np.float32)
     for j in range(k):
-        acc = acc + w[:, j:j + 1] * o[:, j, :]
+        acc = fma32(np.broadcast_to(w[:, j:j + 1], (T, H)), o[:, j, :], acc)
     return f32_to_bf16(acc)
 
 
@@ -408,8 +432,8 @@ def linear_w8a8(x_bits, w_q, s_w) -> np.ndarray:
 def linear_w4a8(x_bits, packed, s_w, group: int = 128) -> np.ndarray:
     """Dense W4A8 linear: per-token int8 x, int4 per-group w.
 
-    acc_g = int32 sum over the g-th group of K; acc_f = sum_g (float)acc_g * s_w[n, g]
-    (fp32, groups in order); y = bf16(acc_f * s_x[t]).
+    acc_g = int32 sum over the g-th group of K; acc_f = fma((float)acc_g, s_w[n, g], acc_f)
+    over the groups in order, from 0; y = bf16(acc_f * s_x[t]).
     """
     xq, sx = quant_act_per_token(x_bits)
     wq = unpack_int4(packed)
@@ -420,5 +444,5 @@ def linear_w4a8(x_bits, packed, s_w, group: int = 128) -> np.ndarray:
     for g in range(K // group):
         ks = slice(g * group, (g + 1) * group)
         acc_g = int_gemm(xq[:, ks], wq[:, ks]).astype(np.float32)
-        acc_f = acc_f + acc_g * s_w[None, :, g]
+        acc_f = fma32(acc_g, np.broadcast_to(s_w[None, :, g], acc_g.shape), acc_f)
     return f32_to_bf16(acc_f * sx[:, None])

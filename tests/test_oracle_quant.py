@@ -186,3 +186,51 @@ def test_bf16_rounding():
     v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1.0 + 2 ** -8 + 2 ** -20], np.float32)
     back = O.bf16_to_f32(O.f32_to_bf16(v))
     np.testing.assert_array_equal(back, [1.0, 1.0, 1.0 + 2 ** -6, -2.5, 1.0 + 2 ** -7])
+
+
+# ------------------------------------------------------------------ fused multiply-add
+def round_f32_exact(fr):
+    """Nearest fp32 (ties to even) of an exact rational, by integer arithmetic (normal range)."""
+    from fractions import Fraction
+    if fr == 0:
+        return 0.0
+    sign = -1.0 if fr < 0 else 1.0
+    fr = abs(Fraction(fr))
+    e = fr.numerator.bit_length() - fr.denominator.bit_length()
+    if Fraction(2) ** e > fr:
+        e -= 1
+    if Fraction(2) ** (e + 1) <= fr:
+        e += 1
+    scaled = fr / Fraction(2) ** (e - 23)  # in [2^23, 2^24)
+    q, rem = divmod(scaled.numerator, scaled.denominator)
+    twice = 2 * rem
+    if twice > scaled.denominator or (twice == scaled.denominator and q % 2 == 1):
+        q += 1
+    return sign * float(q) * 2.0 ** (e - 23)
+
+
+def _fma_exact(a, b, c):
+    from fractions import Fraction
+    return round_f32_exact(Fraction(float(a)) * Fraction(float(b)) + Fraction(float(c)))
+
+
+def test_fma32_matches_exact_rational_rounding():
+    rng = np.random.default_rng(21)
+    n = 3000
+    a = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32)
+    b = (rng.standard_normal(n) * np.exp2(rng.integers(-20, 20, n))).astype(np.float32)
+    c = (rng.standard_normal(n) * np.exp2(rng.integers(-40, 40, n))).astype(np.float32)
+    # designed hard cases: c cancels a*b to within an ulp, and products landing on fp32 ties
+    # and double-rounding traps: a*b + c lies 2^-40 below an fp32 midpoint whose lower
+    # neighbour is odd, so rounding to float64 first lands on the midpoint and ties-to-even
+    # would pick the wrong neighbour
+    a2 = np.array([1 + 2 ** -23, 1 + 2 ** -12, 3.0, 1 + 2 ** -23, 0.1, 8 + 2 ** -20, -(8 + 2 ** -20)], np.float32)
+    b2 = np.array([1 - 2 ** -23, 1 + 2 ** -12, 1 / 3, 1 + 2 ** -23, 10.0, 8 - 2 ** -20, 8 - 2 ** -20], np.float32)
+    c2 = np.array([-1.0, -1.0, -1.0, 2 ** -47, -1.0, 2 ** 30 + 128, -(2 ** 30 + 128)], np.float32)
+    a, b, c = np.concatenate([a, a2]), np.concatenate([b, b2]), np.concatenate([c, c2])
+    got = O.fma32(a, b, c)
+    want = np.array([_fma_exact(x, y, z) for x, y, z in zip(a, b, c)], np.float32)
+    np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+    # it is genuinely fused: differs from the two-rounding result on the cancellation cases
+    two_step = (a2 * b2).astype(np.float32) + c2
+    assert np.any(O.fma32(a2, b2, c2) != two_step)

@@ -298,15 +298,20 @@ def test_w4a8_brute_force_tiny():
     w = bf16(rng.standard_normal((N, K)) * 0.02)
     p, s = O.quantize_weight_int4_per_group(w, G)
     y = O.linear_w4a8(x, p, s, G)
+    from fractions import Fraction
+
+    from tests.test_oracle_quant import round_f32_exact
+
     xq, sx = O.quant_act_per_token(x)
     codes = O.unpack_int4(p)
     for m in range(M):
         for n in range(N):
-            acc = np.float32(0)
+            acc = 0.0
             for g in range(K // G):
                 part = sum(int(xq[m, c]) * int(codes[n, c]) for c in range(g * G, (g + 1) * G))
-                acc = np.float32(acc + np.float32(np.float32(part) * s[n, g]))
-            assert O.f32_to_bf16(np.float32(acc * sx[m])) == y[m, n]
+                # one rounding per step: fp32(part), then fused part * s + acc
+                acc = round_f32_exact(Fraction(float(np.float32(part))) * Fraction(float(s[n, g])) + Fraction(acc))
+            assert O.f32_to_bf16(np.float32(acc) * sx[m]) == y[m, n]
 
 
 def test_oracle_is_independent_of_the_library():

@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
   }
 }
 
-// y[t, :] = bf16(sum_j w[t, j] * o[t, j, :]) with fp32 products and sums in slot order.
+// y[t, :] = bf16(sum_j w[t, j] * o[t, j, :]): fp32 fused multiply-adds in slot order from 0.
 // One CTA per token, 8 columns per thread, no atomics: every y element has one writer.
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ o, const float* __restrict__ w,
                                                       int T, int H, int k, uint16_t* __restrict__ y) {
@@ -173,8 +173,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, bf16_lo(u[i])));
-        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, bf16_hi(u[i])));
+        acc[2 * i] = __fmaf_rn(wj, bf16_lo(u[i]), acc[2 * i]);
+        acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(u[i]), acc[2 * i + 1]);
       }
     }
     uint4 out;

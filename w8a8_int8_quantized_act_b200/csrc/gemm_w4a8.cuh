@@ -1,6 +1,6 @@
 // Dense W4A8 linear on the 5th-generation tensor cores (sm_100a):
 //
-//   y[t, n] = bf16( s_x[t] * sum_g (float)acc_g[t, n] * s_w[n, g] )
+//   y[t, n] = bf16( s_x[t] * acc_f ),  acc_f = fma((float)acc_g, s_w[n, g], acc_f) over g in order
 //   acc_g[t, n] = sum over the g-th group of 128 K values of xq[t, k] * w[n, k]   (int32)
 //
 // The weights arrive as 4-bit two's-complement codes, two per byte (even k in the low nibble),
@@ -14,8 +14,9 @@
 //               alternating TMEM buffers;
 //   warps 2-5   converters: sign-extend the nibbles to int8 and write them in the 128-byte
 //               swizzled K-major layout the MMA reads, then fence the async proxy;
-//   warps 6-13  epilogue: per K-block, add (float)acc_g * s_w[n, g] (fp32, product and sum each
-//               rounded) into registers; at the tile's end store bf16(acc * s_x[t]).
+//   warps 6-13  epilogue: per K-block, acc = fma((float)acc_g, s_w[n, g], acc) in fp32 registers;
+//               at the tile's end store bf16(acc * s_x[t]).
+// Four TMEM buffers let the MMA run up to three K-blocks ahead of the epilogue.
 #pragma once
 #include "gemm.cuh"
 
@@ -44,7 +45,9 @@ struct W4Cfg {
   static constexpr int kBBytes = NB * kKBlockBytes;
   static constexpr int kStageBytes = kPackedBytes + kABytes + kBBytes;
   static constexpr int kStages = (192 * 1024) / kStageBytes > 8 ? 8 : (192 * 1024) / kStageBytes;
-  static constexpr int kTmemCols = (2 * NB <= 64) ? 64 : (2 * NB <= 128 ? 128 : (2 * NB <= 256 ? 256 : 512));
+  static constexpr int kAccBufs = 4;
+  static constexpr int kTmemCols = (kAccBufs * NB <= 128) ? 128 : (kAccBufs * NB <= 256 ? 256 : 512);
+  static_assert(kAccBufs * NB <= 512, "accumulator buffers must fit in TMEM");
   static constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + 512;
   static_assert(kStages >= 2, "pipeline too shallow");
 };
@@ -80,8 +83,8 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
   uint64_t* conv = full + STAGES;
   uint64_t* empty = conv + STAGES;
   uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tempty = tfull + Cfg::kAccBufs;
+  uint64_t* drain = tempty + Cfg::kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
       mbar_init(conv + s, 128);
       mbar_init(empty + s, 1);
     }
-    for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, kEpiWarps * 32); }
+    for (int a = 0; a < Cfg::kAccBufs; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, kEpiWarps * 32); }
     mbar_init(drain, 1);
     fence_mbar_init();
     *abort_flag = 0;
@@ -182,7 +185,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
           tc_commit(empty + stage);
           tc_commit(tfull + acc);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+          if (++acc == Cfg::kAccBufs) { acc = 0; acc_phase ^= 1u; }
         }
         if (!ok) break;
       }
@@ -235,12 +238,15 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
       const int tok0 = mt * NB, rows = min(NB, p.M - tok0);
       const int n = cb * kBM + ch;
       const int j0 = half * HALFC;  // this warp's token columns [j0, j0 + HALFC)
+      const float* __restrict__ swr = p.sw + size_t(n) * nkb;
       float accf[HALFC];
 #pragma unroll
       for (int j = 0; j < HALFC; ++j) accf[j] = 0.0f;
       bool ok = true;
+      float s_next = __ldg(swr);
       for (int kb = 0; kb < nkb; ++kb) {
-        const float s = __ldg(p.sw + size_t(n) * nkb + kb);
+        const float s = s_next;
+        if (kb + 1 < nkb) s_next = __ldg(swr + kb + 1);  // next group's scale, loaded early
         if (!mbar_wait(tfull + acc, acc_phase, wc)) { ok = false; break; }
         tc_fence_after();
         const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * NB);
@@ -251,12 +257,12 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
             tmem_ld16(t_lane + j0 + c16, r);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              accf[c16 + i] = __fadd_rn(accf[c16 + i], __fmul_rn(__int2float_rn(int32_t(r[i])), s));
+              accf[c16 + i] = __fmaf_rn(__int2float_rn(int32_t(r[i])), s, accf[c16 + i]);
           }
         }
         tc_fence_before();
         mbar_arrive(tempty + acc);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == Cfg::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) break;
       uint16_t* out = p.y + n;

@@ -41,8 +41,9 @@ __device__ __forceinline__ int sym_code_fast(float v, float scale, float inv, in
 }
 
 // exp(x) by Cody-Waite range reduction (ln 2 split into a 15-significant-bit high part and a
-// low part) and a degree-7 Taylor polynomial evaluated by Horner's rule, every product and
-// sum rounded to fp32, then an exact scaling by 2^n. x > 88 -> +inf, x < -87 -> 0.
+// low part) and a degree-7 Taylor polynomial evaluated by Horner's rule with fused
+// multiply-adds, then an exact scaling by 2^n. x > 88 -> +inf, x < -87 -> 0.
+//   n = rint(x * log2 e); r = fma(-n, ln2_lo, fma(-n, ln2_hi, x)); p = fma(p, r, 1/i!)
 __device__ __forceinline__ float exp_cw(float x) {
   if (x > 88.0f) return __int_as_float(0x7f800000);
   if (x < -87.0f) return 0.0f;
@@ -50,15 +51,15 @@ __device__ __forceinline__ float exp_cw(float x) {
   const float ln2_hi = (float)0.693145751953125;
   const float ln2_lo = (float)(0.6931471805599453 - 0.693145751953125);
   const float n = rintf(__fmul_rn(x, log2e));
-  const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(n, ln2_hi)), __fmul_rn(n, ln2_lo));
+  const float r = __fmaf_rn(-n, ln2_lo, __fmaf_rn(-n, ln2_hi, x));
   float p = (float)(1.0 / 5040.0);
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 720.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 120.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 24.0));
-  p = __fadd_rn(__fmul_rn(p, r), (float)(1.0 / 6.0));
-  p = __fadd_rn(__fmul_rn(p, r), 0.5f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 24.0));
+  p = __fmaf_rn(p, r, (float)(1.0 / 6.0));
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
   const float two_n = __int_as_float((static_cast<int>(n) + 127) << 23);
   return __fmul_rn(p, two_n);
 }
