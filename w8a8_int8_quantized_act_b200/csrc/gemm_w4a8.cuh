@@ -52,18 +52,32 @@ struct W4Cfg {
   static_assert(kStages >= 2, "pipeline too shallow");
 };
 
+// Four 4-bit two's-complement codes (one per byte, low nibbles) sign-extended to int8 lanes:
+// bit 3 set means negative, and (bit 3) * 30 = 0xF0 fills the high nibble of that byte alone
+// (8 * 30 = 240 < 256, so no product carries into the next byte).
+__device__ __forceinline__ uint32_t sext_nibbles(uint32_t v) {
+  return (v & 0x0F0F0F0Fu) | ((v & 0x08080808u) * 30u);
+}
+
 // 8 packed bytes (16 int4 codes) -> 16 sign-extended int8 codes in k order.
 __device__ __forceinline__ uint4 unpack_int4x16(uint2 pk) {
   const uint32_t w[2] = {pk.x, pk.y};
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const uint32_t lo = __vsub4((w[i] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);         // even k
-    const uint32_t hi = __vsub4(((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);  // odd k
+    const uint32_t lo = sext_nibbles(w[i]);       // even k
+    const uint32_t hi = sext_nibbles(w[i] >> 4);  // odd k
     o[2 * i] = __byte_perm(lo, hi, 0x5140);      // l0 h0 l1 h1
     o[2 * i + 1] = __byte_perm(lo, hi, 0x7362);  // l2 h2 l3 h3
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Exact int -> fp32 for |x| < 2^22 without the conversion pipe: 1.5 * 2^23 + x is an fp32
+// with x in its low mantissa bits, and subtracting 1.5 * 2^23 is exact. A group partial is
+// at most 127 * 7 * 128 < 2^22 in magnitude.
+__device__ __forceinline__ float small_int_to_float(int32_t x) {
+  return __fsub_rn(__int_as_float(x + 0x4B400000), 12582912.0f);
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -257,7 +271,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
             tmem_ld16(t_lane + j0 + c16, r);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              accf[c16 + i] = __fmaf_rn(__int2float_rn(int32_t(r[i])), s, accf[c16 + i]);
+              accf[c16 + i] = __fmaf_rn(small_int_to_float(int32_t(r[i])), s, accf[c16 + i]);
           }
         }
         tc_fence_before();

@@ -53,6 +53,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Like mbar_test, but a thread whose phase is not complete is suspended (not spinning) until the
+// phase completes or `hint_ns` elapses, so waiting warps leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait context: the CTA-wide abort flag (shared memory) and the absolute deadline.
 struct WaitCtx {
   volatile int* abort;
@@ -65,7 +79,7 @@ struct WaitCtx {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_test(bar, parity)) return true;
   while (true) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_test_sleep(bar, parity, 20000u)) return true;
     if (*w.abort) return false;
     if (globaltimer_ns() > w.deadline) {
       *w.abort = 1;
