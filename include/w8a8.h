@@ -29,7 +29,7 @@
  *     nothing. Faults found on the device (a wait that ran out, an out-of-range expert id)
  *     set a device error word that w8a8_check_status() reports.
  *   - Shape rules: hidden sizes and reduction lengths are multiples of 128 (the TMA/MMA
- *     K-block), the expert intermediate size I a multiple of 64, E <= 256, 1 <= k <= 16.
+ *     K-block), the expert intermediate size I a multiple of 128, E <= 256, 1 <= k <= 16.
  */
 #ifndef W8A8_H_
 #define W8A8_H_
