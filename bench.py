@@ -172,6 +172,26 @@ def algorithmic(wl, counts: np.ndarray):
 
 
 # ---------------------------------------------------------------------------- native arm
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's own token batch: the replicas run independent batches of the same layer."""
+    return seed + rank
+
+
+def max_over_ranks(dist, values, device=None):
+    """Element-wise maximum over ranks of per-rank timings: the slowest rank sets the job's time."""
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist is not None and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(world: int, units_per_rank_step: int, steps: int, ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (ms / 1e3)
+
+
 def run_native(args, wl, rank, world, dist):
     import torch
 
@@ -183,7 +203,7 @@ def run_native(args, wl, rank, world, dist):
     dev = torch.device("cuda", local)
     B.lib()
     # every rank: its own batch of wl.T tokens (seeded by rank), the full layer's weights
-    x_host = synth.activations(wl.T, wl.H, wl.n_outlier, wl.seed + rank)
+    x_host = synth.activations(wl.T, wl.H, wl.n_outlier, rank_seed(wl.seed, rank))
     inp = synth.moe_inputs(wl)
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
     x = bf(x_host)
@@ -268,10 +288,7 @@ def run_native(args, wl, rank, world, dist):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks(dist, [ms, e2e_ms], dev)
     return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, stage_ms=stage_ms, counts=counts,
                 clocks=clk.summary(), h2d=wl.T * wl.H * 2, d2h=wl.T * wl.H * 2)
 
@@ -287,7 +304,7 @@ def run_linear(args, wl, rank, dist):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     B.lib()
-    x_host = synth.activations(wl.M, wl.K, wl.n_outlier, wl.seed + rank)
+    x_host = synth.activations(wl.M, wl.K, wl.n_outlier, rank_seed(wl.seed, rank))
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
     x = bf(x_host)
     packed, sw = B.w8a8_quantize_weight_int4_per_group(bf(synth.dense_weight(wl.N, wl.K, wl.seed)), wl.group)
@@ -349,10 +366,8 @@ def run_linear(args, wl, rank, dist):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return dict(ms=float(t[0]), e2e_ms=float(t[1]), e2e_steps=n_e2e, direct_ms=direct_ms, clocks=clk.summary(),
+    ms, e2e_ms = max_over_ranks(dist, [ms, e2e_ms], dev)
+    return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=n_e2e, direct_ms=direct_ms, clocks=clk.summary(),
                 h2d=wl.M * wl.K * 2, d2h=wl.M * wl.N * 2)
 
 
@@ -402,7 +417,7 @@ def main_linear(args, wl, world, rank, peaks, peak_kind):
     int8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = ops / (ms_step / 1e3) / 1e12
     out = {
-        "metric": METRIC, "value": world * wl.M * K / (res["ms"] / 1e3), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": whole_job_rate(world, wl.M, K, res["ms"]), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8 (int4 weights unpacked to int8)", "data": "synthetic",
         "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "group": wl.group,
@@ -414,7 +429,7 @@ def main_linear(args, wl, world, rank, peaks, peak_kind):
                      "kernel": "w4a8_gemm_kernel (tcgen05 kind::i8, int4 unpacked in shared memory) + x quantisation",
                      "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8:bf16 ratio)"},
         "direct_call_ms_per_step": res["direct_ms"] / K,
-        "e2e": {"value": world * wl.M * res["e2e_steps"] / (res["e2e_ms"] / 1e3), "unit": UNIT,
+        "e2e": {"value": whole_job_rate(world, wl.M, res["e2e_steps"], res["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": 2 * K, "clocks": res["clocks"],
     }
@@ -473,8 +488,8 @@ def main():
 
     K = args.steps
     ms_step = res["ms"] / K
-    value = world * wl.T * K / (res["ms"] / 1e3)
-    e2e_value = world * wl.T * res["e2e_steps"] / (res["e2e_ms"] / 1e3)
+    value = whole_job_rate(world, wl.T, K, res["ms"])
+    e2e_value = whole_job_rate(world, wl.T, res["e2e_steps"], res["e2e_ms"])
     alg = algorithmic(wl, res["counts"])
     st = dict(zip(("router", "group_quant", "gate_up", "requant", "down", "combine"), res["stage_ms"].tolist()))
     # dominant kernel: the gate_up GEMM (largest share of every step)
