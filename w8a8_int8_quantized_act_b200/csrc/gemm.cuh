@@ -167,6 +167,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+// Two 16-column loads (e.g. the gate and up accumulators of the same tokens) behind one wait.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, uint32_t (&a)[16], uint32_t (&b)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+        "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+        "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+        "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+      : "r"(ta), "r"(tb));
+}
+
 // ---------------------------------------------------------------------------- epilogues
 // Expert GEMM epilogues: thread = one channel (TMEM lane), columns = the tile's token rows.
 // The two epilogue warps of a lane quarter take alternate 16-column chunks.
@@ -184,18 +199,37 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
     uint32_t ru[16];
 #pragma unroll 1
     for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
-      tmem_ld16(t_lane + j0, r);        // gate accumulators
-      tmem_ld16(t_lane + NB + j0, ru);  // up accumulators
+      const int nj = min(16, c.rows - j0);
+      const int row0 = c.tok0 + j0;
+      // every load of the chunk before any store, so the 16 values are independent chains
+      float sx[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sx[j] = (j < nj) ? __ldg(row_scale + row0 + j) : 0.0f;
+      tmem_ld16x2(t_lane + j0, t_lane + NB + j0, r, ru);  // gate | up accumulators
+      uint32_t hb[16];
+      uint32_t uncertified = 0;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        if (j0 + j < c.rows) {
-          const int row = c.tok0 + j0 + j;
-          const float sx = __ldg(row_scale + row);
-          const float g = dequant(int32_t(r[j]), sx, sg);
-          const float u = dequant(int32_t(ru[j]), sx, su);
-          out[size_t(row) * ldo] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu_exact(g), u)));
+        const float g = dequant(int32_t(r[j]), sx[j], sg);
+        const float u = dequant(int32_t(ru[j]), sx[j], su);
+        bool ok;
+        const float s = div_certified(g, __fadd_rn(1.0f, exp_cw(-g)), ok);
+        uncertified |= ok ? 0u : (1u << j);
+        hb[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(s, u)));
+      }
+      if (uncertified != 0u) {  // rare: quotients the fast divide could not prove
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if ((uncertified >> j) & 1u) {
+            const float g = dequant(int32_t(r[j]), sx[j], sg);
+            const float u = dequant(int32_t(ru[j]), sx[j], su);
+            hb[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(silu_exact(g), u)));
+          }
         }
       }
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < nj) out[size_t(row0 + j) * ldo] = uint16_t(hb[j]);
     }
   } else if constexpr (EPI == kEpiDown || EPI == kEpiDense) {
     // two 128-channel blocks: accumulator columns [0, NB) and [NB, 2NB)
@@ -207,17 +241,28 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
     uint32_t r1[16];
 #pragma unroll 1
     for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
-      tmem_ld16(t_lane + j0, r);
-      tmem_ld16(t_lane + NB + j0, r1);
+      const int nj = min(16, c.rows - j0);
+      const int row0 = c.tok0 + j0;
+      float srow[16];
+      int orow[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        if (j0 + j < c.rows) {
-          const int row = c.tok0 + j0 + j;
-          const int orow = (EPI == kEpiDown) ? __ldg(row_map + row) : row;
-          const float srow = __ldg(row_scale + row);
-          uint16_t* o = out + size_t(orow) * ldo;
-          o[0] = __bfloat16_as_ushort(__float2bfloat16_rn(dequant(int32_t(r[j]), srow, sc0)));
-          if (second) o[kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(dequant(int32_t(r1[j]), srow, sc1)));
+        srow[j] = (j < nj) ? __ldg(row_scale + row0 + j) : 0.0f;
+        orow[j] = (EPI == kEpiDown) ? ((j < nj) ? __ldg(row_map + row0 + j) : 0) : row0 + j;
+      }
+      tmem_ld16x2(t_lane + j0, t_lane + NB + j0, r, r1);
+      uint32_t v0[16], v1[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        v0[j] = __bfloat16_as_ushort(__float2bfloat16_rn(dequant(int32_t(r[j]), srow[j], sc0)));
+        v1[j] = __bfloat16_as_ushort(__float2bfloat16_rn(dequant(int32_t(r1[j]), srow[j], sc1)));
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j < nj) {
+          uint16_t* o = out + size_t(orow[j]) * ldo;
+          o[0] = uint16_t(v0[j]);
+          if (second) o[kBM] = uint16_t(v1[j]);
         }
       }
     }

@@ -44,14 +44,18 @@ __device__ __forceinline__ int sym_code_fast(float v, float scale, float inv, in
 // low part) and a degree-7 Taylor polynomial evaluated by Horner's rule with fused
 // multiply-adds, then an exact scaling by 2^n. x > 88 -> +inf, x < -87 -> 0.
 //   n = rint(x * log2 e); r = fma(-n, ln2_lo, fma(-n, ln2_hi, x)); p = fma(p, r, 1/i!)
+// Branch-free: x is clamped to [-87, 88] and the out-of-range results are selected at the end.
+// rint(y) for |y| < 2^22 is y + 1.5*2^23 rounded to nearest-even, minus 1.5*2^23 (both steps
+// exact apart from that one rounding), and the low bits of the biased sum are n itself.
 __device__ __forceinline__ float exp_cw(float x) {
-  if (x > 88.0f) return __int_as_float(0x7f800000);
-  if (x < -87.0f) return 0.0f;
   const float log2e = (float)1.4426950408889634;
   const float ln2_hi = (float)0.693145751953125;
   const float ln2_lo = (float)(0.6931471805599453 - 0.693145751953125);
-  const float n = rintf(__fmul_rn(x, log2e));
-  const float r = __fmaf_rn(-n, ln2_lo, __fmaf_rn(-n, ln2_hi, x));
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float xc = fminf(fmaxf(x, -87.0f), 88.0f);
+  const float t = __fadd_rn(__fmul_rn(xc, log2e), kRound);
+  const float n = __fsub_rn(t, kRound);
+  const float r = __fmaf_rn(-n, ln2_lo, __fmaf_rn(-n, ln2_hi, xc));
   float p = (float)(1.0 / 5040.0);
   p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
   p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
@@ -60,12 +64,42 @@ __device__ __forceinline__ float exp_cw(float x) {
   p = __fmaf_rn(p, r, 0.5f);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  const float two_n = __int_as_float((static_cast<int>(n) + 127) << 23);
-  return __fmul_rn(p, two_n);
+  // n + 127 in the exponent field; n = bits(t) - bits(1.5 * 2^23) lies in [-126, 127]
+  const float two_n = __int_as_float((__float_as_int(t) - 0x4B400000 + 127) << 23);
+  float v = __fmul_rn(p, two_n);
+  v = (x > 88.0f) ? __int_as_float(0x7f800000) : v;
+  v = (x < -87.0f) ? 0.0f : v;
+  return (x != x) ? x : v;
 }
 
 // SiLU(g) = g / (1 + exp(-g)) with a true divide.
 __device__ __forceinline__ float silu_exact(float g) { return __fdiv_rn(g, __fadd_rn(1.0f, exp_cw(-g))); }
+
+// q = g / d rounded to nearest-even (the IEEE quotient) for d >= 1, without a branch; `ok`
+// is false where the fast path cannot prove its answer, and the caller then takes __fdiv_rn.
+//   y  ~ 1/d  (hardware approximation, relative error below 2^-22)
+//   q0 = fl(g*y); r0 = fma(-d, q0, g); q1 = fma(r0, y, q0)
+// The correction step is Markstein's (IBM J. Res. Dev. 34(1), 1990): its pre-rounding value is
+// within 2^-44 relative of g/d, so q1 is a faithful rounding, and then r1 = g - d*q1 is exact
+// (the remainder of a faithful quotient is a float when nothing underflows; here |q1| >= 2^-100
+// and d >= 1). q1 is the nearest float to g/d iff |g/d - q1| < ulp(q1)/2, i.e. iff
+// |r1| < (ulp(q1)/2)*d, a product that is exact (a power of two times d). A q1 whose
+// significand is 1.0 (the gap below it is half as wide), an exact tie, a non-finite or a tiny
+// q1 is not certified; g = 0 returns g (signed zero). r1 = 0 means q1 is the exact quotient.
+__device__ __forceinline__ float div_certified(float g, float d, bool& ok) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
+  const float q0 = __fmul_rn(g, y);
+  const float r0 = __fmaf_rn(-d, q0, g);
+  const float q1 = __fmaf_rn(r0, y, q0);
+  const float r1 = __fmaf_rn(-d, q1, g);
+  const uint32_t qa = __float_as_uint(q1) & 0x7FFFFFFFu;
+  const float half_ulp_d = __fmul_rn(__uint_as_float((qa & 0x7F800000u) - (24u << 23)), d);
+  const bool in_range = qa >= 0x0D800000u && qa < 0x7F800000u;  // 2^-100 <= |q1| < inf
+  const bool nearest = (r1 == 0.0f) || (fabsf(r1) < half_ulp_d && (qa & 0x007FFFFFu) != 0u);
+  ok = (g == 0.0f) || (in_range && nearest);
+  return (g == 0.0f) ? g : q1;
+}
 
 // ((float)acc * s_row) * s_col, each product rounded to fp32.
 __device__ __forceinline__ float dequant(int32_t acc, float s_row, float s_col) {
