@@ -75,6 +75,8 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert lib.w8a8_quantize_weight_int4_per_group(None, 4, 256, 64, None, None, None) == B.W8A8_ERR_UNSUPPORTED
     assert lib.w8a8_gemm_s8s8s32(None, None, None, 4, 100, 128, None) == B.W8A8_ERR_UNSUPPORTED
     assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_debug_rcp_approx_ulp(0, 10, c(16), None) == B.W8A8_ERR_ARG  # not a normal input
+    assert lib.w8a8_debug_rcp_approx_ulp(0x7E7FFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # reciprocal subnormal
 
 
 def test_package_has_no_oracle_dependency():

@@ -31,7 +31,8 @@ def _clean_status():
 
 # ------------------------------------------------------------------ exact int8 GEMM
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (128, 128, 256), (300, 384, 2048), (1000, 256, 768),
-                                   (77, 6144, 128)])
+                                   (77, 6144, 128), (129, 128, 128), (136, 640, 384), (4133, 512, 1024),
+                                   (256, 6144, 2048)])
 def test_gemm_s8s8s32_exact(M, N, K):
     rng = np.random.default_rng(M + N + K)
     a = rng.integers(-127, 128, (M, K)).astype(np.int8)
@@ -145,6 +146,17 @@ def test_moe_edge_shapes(T, E, k, I):
     _full_check(G.run_moe(wl))
 
 
+# Long token lists (the CTA-pair GEMMs): several 256-row blocks per expert with ragged tails,
+# an odd number of 128-channel blocks in the down projection (H = 384), a single expert.
+@pytest.mark.parametrize("T,H,E,k,I", [(600, 384, 4, 2, 256), (1031, 256, 8, 3, 128), (700, 512, 1, 1, 384),
+                                       (2000, 640, 16, 4, 256)])
+def test_moe_long_token_lists(T, H, E, k, I):
+    wl = synth.MoEWorkload("long", T=T, H=H, E=E, k=k, I=I, n_outlier=3, seed=T)
+    run = G.run_moe(wl)
+    assert np.diff(run.mid["offsets"]).max() > 256
+    _full_check(run)
+
+
 def test_moe_zero_tokens_and_empty_experts():
     wl = synth.MoEWorkload("empty-experts", T=100, H=256, E=16, k=2, I=128, n_outlier=2)
     bias = np.zeros(16, np.float32)
@@ -209,6 +221,15 @@ def test_linear_w4a8_extreme_codes():
     y = B.w8a8_linear(G.bf16_dev(x), packed, s, B.W8A8_W_INT4_PER_GROUP, 128)
     op, os_ = O.quantize_weight_int4_per_group(w, 128)
     np.testing.assert_array_equal(G.host(y), O.linear_w4a8(x, op, os_, 128))
+
+
+# ------------------------------------------------------------------ hardware premise of the certified SiLU
+def test_rcp_approx_within_two_ulp():
+    # The gate_up epilogue of the CTA-pair GEMM accepts bf16(fl(fl(g * rcp.approx(d)) * u)) only
+    # when its fp32 bits are more than 16 ulps from a bf16 rounding midpoint; the proof needs
+    # rcp.approx within 2 ulps of the correctly rounded reciprocal. Every mantissa, three binades.
+    for first in (0x3F800000, 0x5F800000, 0x1F800000):
+        assert B.w8a8_debug_rcp_approx_ulp(first, 1 << 23) <= 2
 
 
 # ------------------------------------------------------------------ failure detection

@@ -63,6 +63,7 @@ SIGNATURES = {
     "w8a8_linear": (_int, [_c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _size, _c_p, _c_p]),
     "w8a8_gemm_s8s8s32": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
+    "w8a8_debug_rcp_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
 }
 
 _lib = None
@@ -295,6 +296,15 @@ def w8a8_gemm_s8s8s32(a, b, c=None, stream=None):
     c = torch.empty((M, N), dtype=torch.int32, device=a.device) if c is None else c
     _check(lib().w8a8_gemm_s8s8s32(_ptr(a), _ptr(b), _ptr(c), M, N, K, _stream(stream)), "w8a8_gemm_s8s8s32")
     return c
+
+
+def w8a8_debug_rcp_approx_ulp(first_bits: int, count: int, stream=None) -> int:
+    """Largest ulp distance of rcp.approx from the correctly rounded reciprocal over a range of
+    fp32 bit patterns."""
+    out = torch.empty(1, dtype=torch.int32, device="cuda")
+    _check(lib().w8a8_debug_rcp_approx_ulp(first_bits, count, _ptr(out), _stream(stream)),
+           "w8a8_debug_rcp_approx_ulp")
+    return int(out.cpu().item())
 
 
 def w8a8_debug_wait_timeout(timeout_ns: int, stream=None):

@@ -186,6 +186,22 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   }
 }
 
+// Largest distance, in units in the last place, between rcp.approx.ftz.f32(d) and the correctly
+// rounded reciprocal of d, over the fp32 bit patterns first .. first + count - 1 (positive normal
+// d with a normal reciprocal). The certified SiLU evaluation assumes this is at most 2.
+__global__ void rcp_approx_ulp_kernel(uint32_t first, uint32_t count, unsigned int* max_ulp) {
+  unsigned int worst = 0;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x) {
+    const float d = __uint_as_float(first + i);
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    const int diff = int(__float_as_uint(r)) - int(__float_as_uint(__frcp_rn(d)));
+    worst = max(worst, unsigned(diff < 0 ? -diff : diff));
+  }
+  worst = warp_max_u32(worst);
+  if ((threadIdx.x & 31) == 0) atomicMax(max_ulp, worst);
+}
+
 // Host-visible probe of the bounded-wait machinery: waits on an mbarrier phase that nothing
 // completes, so the wait must run out after `timeout_ns` and raise the error word.
 __global__ void wait_timeout_probe_kernel(uint64_t timeout_ns) {

@@ -44,18 +44,17 @@ __device__ __forceinline__ int sym_code_fast(float v, float scale, float inv, in
 // low part) and a degree-7 Taylor polynomial evaluated by Horner's rule with fused
 // multiply-adds, then an exact scaling by 2^n. x > 88 -> +inf, x < -87 -> 0.
 //   n = rint(x * log2 e); r = fma(-n, ln2_lo, fma(-n, ln2_hi, x)); p = fma(p, r, 1/i!)
-// Branch-free: x is clamped to [-87, 88] and the out-of-range results are selected at the end.
 // rint(y) for |y| < 2^22 is y + 1.5*2^23 rounded to nearest-even, minus 1.5*2^23 (both steps
 // exact apart from that one rounding), and the low bits of the biased sum are n itself.
-__device__ __forceinline__ float exp_cw(float x) {
+// exp_cw_core is that computation for -87 <= x <= 88 (where n lies in [-126, 127]).
+__device__ __forceinline__ float exp_cw_core(float x) {
   const float log2e = (float)1.4426950408889634;
   const float ln2_hi = (float)0.693145751953125;
   const float ln2_lo = (float)(0.6931471805599453 - 0.693145751953125);
   const float kRound = 12582912.0f;  // 1.5 * 2^23
-  const float xc = fminf(fmaxf(x, -87.0f), 88.0f);
-  const float t = __fadd_rn(__fmul_rn(xc, log2e), kRound);
+  const float t = __fadd_rn(__fmul_rn(x, log2e), kRound);
   const float n = __fsub_rn(t, kRound);
-  const float r = __fmaf_rn(-n, ln2_lo, __fmaf_rn(-n, ln2_hi, xc));
+  const float r = __fmaf_rn(-n, ln2_lo, __fmaf_rn(-n, ln2_hi, x));
   float p = (float)(1.0 / 5040.0);
   p = __fmaf_rn(p, r, (float)(1.0 / 720.0));
   p = __fmaf_rn(p, r, (float)(1.0 / 120.0));
@@ -64,9 +63,15 @@ __device__ __forceinline__ float exp_cw(float x) {
   p = __fmaf_rn(p, r, 0.5f);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  // n + 127 in the exponent field; n = bits(t) - bits(1.5 * 2^23) lies in [-126, 127]
-  const float two_n = __int_as_float((__float_as_int(t) - 0x4B400000 + 127) << 23);
-  float v = __fmul_rn(p, two_n);
+  // n + 127 in the exponent field; n = bits(t) - bits(1.5 * 2^23)
+  const float two_n = __uint_as_float((__float_as_uint(t) - 0x4B400000u + 127u) << 23);
+  return __fmul_rn(p, two_n);
+}
+
+// Branch-free: x is clamped to [-87, 88] and the out-of-range results are selected at the end.
+__device__ __forceinline__ float exp_cw(float x) {
+  const float xc = fminf(fmaxf(x, -87.0f), 88.0f);
+  float v = exp_cw_core(xc);
   v = (x > 88.0f) ? __int_as_float(0x7f800000) : v;
   v = (x < -87.0f) ? 0.0f : v;
   return (x != x) ? x : v;
@@ -99,6 +104,32 @@ __device__ __forceinline__ float div_certified(float g, float d, bool& ok) {
   const bool nearest = (r1 == 0.0f) || (fabsf(r1) < half_ulp_d && (qa & 0x007FFFFFu) != 0u);
   ok = (g == 0.0f) || (in_range && nearest);
   return (g == 0.0f) ? g : q1;
+}
+
+// bf16(fl(SiLU(g) * u)), the gated activation as the layer defines it (SiLU with the exact
+// quotient g / (1 + exp_cw(-g))), evaluated cheaply and certified at the bf16 level:
+//   Y = fl(fl(g * rcp.approx(d)) * u),  d = fl(1 + exp_cw(-g))   (the same d as the definition)
+// differs from S = fl(fl(g / d) * u) by the reciprocal's error and four fp32 roundings:
+// |Y/S - 1| <= eps_rcp + 4 * 2^-24 + O(2^-48). With rcp.approx within 2 ulp of the correctly
+// rounded reciprocal (eps_rcp <= 5 * 2^-24; a GPU test measures it over a whole binade), Y is
+// within 9 fp32 ulps of S whenever Y is a normal number. bf16 rounding looks only at the low 16
+// bits of the fp32 pattern (round up above 0x8000, ties to even at 0x8000), so if those bits of
+// Y are more than kBf16Margin = 16 ulps away from 0x8000, S lies in the same bf16 rounding
+// interval and bf16(Y) = bf16(S). (Near a binade boundary the low bits are near 0 or 0xFFFF and
+// both round to the same power of two.) Accepted only for |g| <= 64 (exp_cw needs no range
+// handling there and d < 2^93) and 2^-120 <= |Y| < 2^121; `ok` is false otherwise, and the
+// caller then evaluates silu_exact. Returns Y.
+constexpr uint32_t kBf16Margin = 16;
+__device__ __forceinline__ float silu_mul_bf16_certified(float g, float u, bool& ok) {
+  const float d = __fadd_rn(1.0f, exp_cw_core(-g));
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+  const float y = __fmul_rn(__fmul_rn(g, r), u);
+  const uint32_t b = __float_as_uint(y);
+  const bool normal = ((b >> 23) & 0xFFu) - 7u < 241u;
+  const bool clear_of_tie = (((b ^ 0x8000u) + kBf16Margin) & 0xFFFFu) > 2u * kBf16Margin;
+  ok = (fabsf(g) <= 64.0f) && normal && clear_of_tie;
+  return y;
 }
 
 // ((float)acc * s_row) * s_col, each product rounded to fp32.

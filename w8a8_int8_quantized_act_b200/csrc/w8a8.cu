@@ -9,6 +9,7 @@
 #include "../../include/w8a8.h"
 #include "elementwise.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_w4a8.cuh"
 
 namespace w8a8 {
@@ -87,6 +88,22 @@ bool make_plain_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// gate_up weights [E, 2I, H] int8 seen as the 5-D tensor (k, row within a 16-channel group,
+// gate or up half, 16-channel group, expert), so that one (128 B, 16, 2, 4, 1) box brings
+// 4 x (16 gate rows, the matching 16 up rows): the interleaved 128-row tile of the pair GEMM.
+// Every coordinate range stays inside the tensor.
+bool make_gate_up_pair_map(CUtensorMap* m, const void* base, uint64_t H, uint64_t I, uint64_t E) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || H == 0 || I % 64 || E == 0) return false;
+  const cuuint64_t dims[5] = {H, 16, 2, I / 16, E};
+  const cuuint64_t strides[4] = {H, I * H, 16 * H, 2 * I * H};
+  const cuuint32_t box[5] = {128, 16, 2, 4, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ launch helpers
 int launch_status() { return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_LAUNCH; }
 
@@ -100,6 +117,45 @@ int launch_gemm(const GemmParams& p, int max_tiles, cudaStream_t stream) {
   const int grid = max(1, min(num_sms(), max_tiles));
   kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(p);
   return launch_status();
+}
+
+// Clusters of gemm_pair_kernel<EPI> that fit on the device at once (one CTA per SM), cached.
+template <int EPI>
+int pair_clusters() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(unsigned(num_sms() & ~1), 1, 1);
+    cfg.blockDim = dim3(PairCfg<EPI>::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = PairCfg<EPI>::kSmemBytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<EPI>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int EPI>
+int launch_pair(const PairParams& p, int max_tiles, cudaStream_t stream) {
+  auto kern = gemm_pair_kernel<EPI>;
+  using Cfg = PairCfg<EPI>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) != cudaSuccess)
+    return W8A8_ERR_LAUNCH;
+  const int clusters = max(1, min(pair_clusters<EPI>(), max_tiles));
+  kern<<<2 * clusters, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
+  return launch_status();
+}
+
+// Token-row maps of a K-major int8 operand for the pair kernel: 128-, 16- and 8-row boxes.
+bool make_pair_b_maps(PairParams* p, const void* base, uint64_t inner, uint64_t rows) {
+  return make_kmajor_map(&p->tmB128, base, false, inner, rows, 128) &&
+         make_kmajor_map(&p->tmB16, base, false, inner, rows, 16) &&
+         make_kmajor_map(&p->tmB8, base, false, inner, rows, 8);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -256,7 +312,11 @@ int launch_group_quant(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* x
 // Upper bound of the number of token blocks of `nb` rows over all groups: ceil(A/nb) + min(E, A).
 int max_token_blocks(int64_t A, int64_t E, int nb) { return int((A + nb - 1) / nb + (E < A ? E : A)); }
 
-// Token block of the expert GEMMs: 32 rows when experts see few tokens (decode), else 128.
+// Dense GEMMs with more token rows than this run on CTA pairs.
+constexpr int64_t kPairMinRows = 128;
+
+// Token block of the expert GEMMs: 32 rows when experts see few tokens (decode), else 256 on
+// CTA pairs.
 bool small_token_blocks(int64_t A, int64_t E) { return A <= 32 * E; }
 
 // CTAs per 128-token chunk of the grouping kernel: enough warps for every token of a small
@@ -418,13 +478,13 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   if (rc != W8A8_OK) return rc;
 
   // 3. grouped gate_up GEMM (weights on M, tokens on N) with the dequant + SiLU(gate)*up
-  //    epilogue -> h
+  //    epilogue -> h. Few rows per expert (decode): one CTA per tile of <= 32 rows; otherwise
+  //    CTA pairs on tiles of <= 256 rows.
   const bool small = small_token_blocks(A, E);
-  const int nbt = small ? 32 : 128;
-  {
+  if (small) {
     GemmParams p{};
     if (!make_kmajor_map(&p.tmA, wgu, false, H, uint64_t(E) * 2 * I, 128) ||
-        !make_kmajor_map(&p.tmB, xq, false, H, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, xq, false, H, Ap, nbt))
+        !make_kmajor_map(&p.tmB, xq, false, H, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, xq, false, H, Ap, 32))
       return W8A8_ERR_UNSUPPORTED;
     p.num_kb = int(H / 128);
     p.n_cb = int(I / 128);
@@ -440,11 +500,29 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     p.col_scale = s_gu;
     p.col_scale_stride = int(2 * I);
     p.up_offset = int(I);
-    const int tiles = max_token_blocks(A, E, nbt) * p.n_cb;
+    const int tiles = max_token_blocks(A, E, 32) * p.n_cb;
     mark(ev, 2, s);
-    rc = small ? launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, tiles, s)
-               : launch_gemm<2, 128, kEpiGateUp, kKindI8>(p, tiles, s);
-    if (rc != W8A8_OK) return rc;
+    if ((rc = launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, tiles, s)) != W8A8_OK) return rc;
+  } else {
+    PairParams p{};
+    if (!make_gate_up_pair_map(&p.tmA, wgu, H, I, E) || !make_pair_b_maps(&p, xq, H, Ap))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(H / 128);
+    p.n_cb = int(I / 128);
+    p.num_groups = int(E);
+    p.group_offsets = offsets;
+    p.a_rows_per_group = int(2 * I);
+    p.n_channels = int(I);
+    p.timeout_ns = wait_timeout_ns();
+    p.out = h;
+    p.ldo = int(I);
+    p.row_scale = sx_sorted;
+    p.col_scale = s_gu;
+    p.col_scale_stride = int(2 * I);
+    p.up_offset = int(I);
+    const int tiles = max_token_blocks(A, E, kPairNB) * p.n_cb;
+    mark(ev, 2, s);
+    if ((rc = launch_pair<kEpiGateUp>(p, tiles, s)) != W8A8_OK) return rc;
   }
 
   // 4. per-row requantisation of h
@@ -454,10 +532,10 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   }
 
   // 5. grouped down GEMM with the dequant epilogue -> o in slot order
-  {
+  if (small) {
     GemmParams p{};
     if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(E) * H, 128) ||
-        !make_kmajor_map(&p.tmB, hq, false, I, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, hq, false, I, Ap, nbt))
+        !make_kmajor_map(&p.tmB, hq, false, I, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, hq, false, I, Ap, 32))
       return W8A8_ERR_UNSUPPORTED;
     p.num_kb = int(I / 128);
     p.n_cb = int((H + 255) / 256);
@@ -474,11 +552,29 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     p.col_scale = s_d;
     p.col_scale_stride = int(H);
     p.row_map = perm;
-    const int tiles = max_token_blocks(A, E, nbt) * p.n_cb;
+    const int tiles = max_token_blocks(A, E, 32) * p.n_cb;
     mark(ev, 4, s);
-    rc = small ? launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s)
-               : launch_gemm<2, 128, kEpiDown, kKindI8>(p, tiles, s);
-    if (rc != W8A8_OK) return rc;
+    if ((rc = launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s)) != W8A8_OK) return rc;
+  } else {
+    PairParams p{};
+    if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(E) * H, 128) || !make_pair_b_maps(&p, hq, I, Ap))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(I / 128);
+    p.n_cb = int((H + 255) / 256);
+    p.n_channels = int(H);
+    p.num_groups = int(E);
+    p.group_offsets = offsets;
+    p.a_rows_per_group = int(H);
+    p.timeout_ns = wait_timeout_ns();
+    p.out = o;
+    p.ldo = int(H);
+    p.row_scale = s_h;
+    p.col_scale = s_d;
+    p.col_scale_stride = int(H);
+    p.row_map = perm;
+    const int tiles = max_token_blocks(A, E, kPairNB) * p.n_cb;
+    mark(ev, 4, s);
+    if ((rc = launch_pair<kEpiDown>(p, tiles, s)) != W8A8_OK) return rc;
   }
 
   // 6. scatter-free weighted combine
@@ -609,6 +705,22 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
     kern<<<max(1, min(num_sms(), tiles)), kW4Threads, Cfg::kSmemBytes, s>>>(q);
     return launch_status();
   }
+  if (M > kPairMinRows) {
+    PairParams q{};
+    if (!make_kmajor_map(&q.tmA, wq, false, K, N, 128) || !make_pair_b_maps(&q, xq, K, Mp))
+      return W8A8_ERR_UNSUPPORTED;
+    q.num_kb = int(K / 128);
+    q.n_cb = int((N + 255) / 256);
+    q.n_channels = int(N);
+    q.num_groups = 1;
+    q.M = int(M);
+    q.timeout_ns = wait_timeout_ns();
+    q.out = y;
+    q.ldo = int(N);
+    q.row_scale = sx;
+    q.col_scale = sw;
+    return launch_pair<kEpiDense>(q, int((M + kPairNB - 1) / kPairNB) * q.n_cb, s);
+  }
   GemmParams p{};
   if (!make_kmajor_map(&p.tmA, wq, false, K, N, 128) || !make_kmajor_map(&p.tmB, xq, false, K, Mp, kBBoxRows) ||
       !make_kmajor_map(&p.tmB2, xq, false, K, Mp, 128))
@@ -637,6 +749,20 @@ int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, i
   if (!a || !b || !c) return W8A8_ERR_ARG;
   if (!aligned16(a) || !aligned16(b) || !aligned16(c) || M >= (int64_t(1) << 30)) return W8A8_ERR_UNSUPPORTED;
   // channels (rows of b) on the MMA M side, rows of a on N
+  if (M > kPairMinRows) {
+    PairParams q{};
+    if (!make_kmajor_map(&q.tmA, b, false, K, N, 128) || !make_pair_b_maps(&q, a, K, M))
+      return W8A8_ERR_UNSUPPORTED;
+    q.num_kb = int(K / 128);
+    q.n_cb = int((N + 255) / 256);
+    q.n_channels = int(N);
+    q.num_groups = 1;
+    q.M = int(M);
+    q.timeout_ns = wait_timeout_ns();
+    q.out = c;
+    q.ldo = int(N);
+    return launch_pair<kEpiRawS32>(q, int((M + kPairNB - 1) / kPairNB) * q.n_cb, as_stream(stream));
+  }
   GemmParams p{};
   if (!make_kmajor_map(&p.tmA, b, false, K, N, 128) || !make_kmajor_map(&p.tmB, a, false, K, M, kBBoxRows) ||
       !make_kmajor_map(&p.tmB2, a, false, K, M, 128))
@@ -653,6 +779,18 @@ int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, i
   p.ldo = int(N);
   const int tiles = int((M + 127) / 128) * p.n_cb;
   return launch_gemm<2, 128, kEpiRawS32, kKindI8>(p, tiles, as_stream(stream));
+}
+
+int w8a8_debug_rcp_approx_ulp(uint32_t first_bits, uint32_t count, unsigned int* max_ulp, w8a8_stream stream) {
+  if (!max_ulp || count == 0) return W8A8_ERR_ARG;
+  const uint64_t last = uint64_t(first_bits) + count - 1;
+  // positive normal inputs whose reciprocal is normal: [2^-126, 2^126)
+  if (first_bits < 0x00800000u || last >= 0x7E800000u) return W8A8_ERR_ARG;
+  if (cudaMemsetAsync(max_ulp, 0, sizeof(unsigned int), as_stream(stream)) != cudaSuccess) return W8A8_ERR_LAUNCH;
+  const uint64_t want = (uint64_t(count) + 255) / 256;
+  const unsigned blocks = unsigned(want < 4096 ? want : 4096);
+  rcp_approx_ulp_kernel<<<blocks, 256, 0, as_stream(stream)>>>(first_bits, count, max_ulp);
+  return launch_status();
 }
 
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {
