@@ -421,16 +421,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_parity = 0;
-      for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
-        const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
-        const uint32_t bytes = uint32_t(NA * Cfg::kABytes + c.nb * kKBlockBytes);
-        bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+    // The whole warp runs the loop (converged, warp-uniform values); one elected lane issues.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_parity = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
+      const uint32_t bytes = uint32_t(NA * Cfg::kABytes + c.nb * kKBlockBytes);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+        if (elect_one()) {
           uint8_t* st = smem + stage * Cfg::kStageBytes;
           mbar_arrive_expect_tx(full + stage, bytes);
           const int x = kb * KB_ELEMS;
@@ -443,64 +444,71 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
             for (int b = 0; b < c.nb; b += kBBoxRows)
               tma_load_2d(sb + b * kKBlockBytes, &p.tmB, full + stage, x, c.b_row + b);
           }
-          issued_mask |= 1u << stage;
-          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      if (*abort_flag) {
-        // let every load already issued land before the CTA's shared memory goes away
-        volatile int no_abort = 0;
-        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
-        for (int s = 0; s < STAGES; ++s)
-          if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
-      }
+    }
+    if (lane == 0 && *abort_flag) {
+      // let every load already issued land before the CTA's shared memory goes away
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool issued_any = false;
-      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-        const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
-        const uint32_t idesc = IDESC0 | (uint32_t(c.nb >> 3) << 17);
-        if (!mbar_wait(tempty + acc, acc_phase ^ 1u, wc)) break;
-        tc_fence_after();
-        const uint32_t d0 = tmem_base + uint32_t(acc * Cfg::kAccCols);
-        bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(full + stage, phase, wc)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t s0 = smem_addr(smem + stage * Cfg::kStageBytes);
-          const uint32_t sb = s0 + NA * Cfg::kABytes;
+    // Converged warp; descriptors are warp-uniform (stage and K offsets added to the 14-bit
+    // start-address field, which cannot carry: shared memory ends below 256 KB); one elected
+    // lane issues every MMA and commit.
+    const uint64_t adesc0 = sw128_kmajor_desc(smem_addr(smem));
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool issued_any = false;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
+      const uint32_t idesc = IDESC0 | (uint32_t(c.nb >> 3) << 17);
+      if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) break;
+      tc_fence_after();
+      const uint32_t d0 = tmem_base + uint32_t(acc * Cfg::kAccCols);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        // TMA completions on this barrier; the MMAs read the stage through the same async proxy
+        if (!mbar_wait_warp(full + stage, phase, wc)) { ok = false; break; }
+        if (elect_one()) {
+          const uint64_t ad = adesc0 + uint64_t(stage * (Cfg::kStageBytes >> 4));
+          const uint64_t bd = ad + uint64_t(NA * (Cfg::kABytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < kKBlockBytes / 32; ++kk) {
-            const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            tc_mma<KIND>(d0, sw128_kmajor_desc(s0 + kk * 32), bdesc, idesc, accum);
+            tc_mma<KIND>(d0, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc, accum);
             if (NA == 2)
-              tc_mma<KIND>(d0 + NB, sw128_kmajor_desc(s0 + Cfg::kABytes + kk * 32), bdesc, idesc, accum);
+              tc_mma<KIND>(d0 + NB, ad + uint64_t((Cfg::kABytes >> 4) + 2 * kk), bd + uint64_t(2 * kk), idesc,
+                           accum);
           }
-          issued_any = true;
           tc_commit(empty + stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
-        tc_commit(tfull + acc);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        __syncwarp();
+        issued_any = true;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      if (*abort_flag && issued_any) {
-        // wait for the MMAs already issued before TMEM is released
-        tc_commit(drain);
-        volatile int no_abort = 0;
-        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
-        mbar_wait(drain, 0, dw);
-      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(tfull + acc);
+      __syncwarp();
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0 && *abort_flag && issued_any) {
+      // wait for the MMAs already issued (by lane 0, the elected lane of the converged warp)
+      // before TMEM is released
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      mbar_wait(drain, 0, dw);
     }
     __syncwarp();
   } else {

@@ -137,17 +137,18 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0, issued_parity = 0;
-      for (int tile = blockIdx.x; tile < total_tiles && !*abort_flag; tile += gridDim.x) {
-        const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
-        const int tok0 = mt * NB, rows = min(NB, p.M - tok0), nb = (rows + 15) & ~15;
-        const uint32_t bytes = uint32_t(Cfg::kPackedBytes + nb * kKBlockBytes);
-        bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+    // Converged warp, one elected lane issues.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_parity = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      const int tok0 = mt * NB, rows = min(NB, p.M - tok0), nb = (rows + 15) & ~15;
+      const uint32_t bytes = uint32_t(Cfg::kPackedBytes + nb * kKBlockBytes);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+        if (elect_one()) {
           mbar_arrive_expect_tx(full + stage, bytes);
           tma_load_2d(packed_of(stage), &p.tmW, full + stage, kb * 64, cb * kBM);
           if (nb == NB) {
@@ -156,59 +157,61 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
             for (int b = 0; b < nb; b += kBBoxRows)
               tma_load_2d(b_of(stage) + b * kKBlockBytes, &p.tmX, full + stage, kb * 128, tok0 + b);
           }
-          issued_mask |= 1u << stage;
-          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        issued_mask |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      if (*abort_flag) {
-        volatile int no_abort = 0;
-        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
-        for (int s = 0; s < STAGES; ++s)
-          if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
-      }
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool issued_any = false;
-      for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-        const int mt = tile / p.n_cb;
-        const int rows = min(NB, p.M - mt * NB), nb = (rows + 15) & ~15;
-        const uint32_t idesc = IDESC0 | (uint32_t(nb >> 3) << 17);
-        bool ok = true;
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-          // one scale group per K-block: a fresh accumulator in the free TMEM buffer
-          if (!mbar_wait(tempty + acc, acc_phase ^ 1u, wc)) { ok = false; break; }
-          if (!mbar_wait(conv + stage, phase, wc)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem_base + uint32_t(acc * NB);
-          const uint32_t a0 = smem_addr(a_of(stage));
-          const uint32_t b0 = smem_addr(b_of(stage));
+    // Converged warp, warp-uniform descriptors, one elected lane issues.
+    const uint64_t adesc0 = sw128_kmajor_desc(smem_addr(a_of(0)));
+    const uint64_t bdesc0 = sw128_kmajor_desc(smem_addr(b_of(0)));
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool issued_any = false;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int mt = tile / p.n_cb;
+      const int rows = min(NB, p.M - mt * NB), nb = (rows + 15) & ~15;
+      const uint32_t idesc = IDESC0 | (uint32_t(nb >> 3) << 17);
+      for (int kb = 0; kb < nkb; ++kb) {
+        // one scale group per K-block: a fresh accumulator in the free TMEM buffer
+        if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) { ok = false; break; }
+        if (!mbar_wait_warp(conv + stage, phase, wc)) { ok = false; break; }
+        tc_fence_after();  // the converters' shared-memory writes (generic proxy, fenced) precede
+        const uint32_t d = tmem_base + uint32_t(acc * NB);
+        if (elect_one()) {
+          const uint64_t ad = adesc0 + uint64_t(stage * (Cfg::kStageBytes >> 4));
+          const uint64_t bd = bdesc0 + uint64_t(stage * (Cfg::kStageBytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < kKBlockBytes / 32; ++kk)
-            tc_mma<kKindI8>(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc,
-                            kk != 0 ? 1u : 0u);
-          issued_any = true;
+            tc_mma<kKindI8>(d, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc, kk != 0 ? 1u : 0u);
           tc_commit(empty + stage);
           tc_commit(tfull + acc);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++acc == Cfg::kAccBufs) { acc = 0; acc_phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        issued_any = true;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++acc == Cfg::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
-      if (*abort_flag && issued_any) {
-        tc_commit(drain);
-        volatile int no_abort = 0;
-        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
-        mbar_wait(drain, 0, dw);
-      }
+    }
+    if (lane == 0 && *abort_flag && issued_any) {
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      mbar_wait(drain, 0, dw);
     }
     __syncwarp();
   } else if (warp < 6) {

@@ -321,7 +321,7 @@ bool small_token_blocks(int64_t A, int64_t E) { return A <= 32 * E; }
 
 // CTAs per 128-token chunk of the grouping kernel: enough warps for every token of a small
 // batch, fewer for long ones (each CTA re-derives its chunk's positions).
-int group_quant_splits(int64_t T) { return T <= 1024 ? 8 : (T <= 4096 ? 4 : 2); }
+int group_quant_splits(int64_t T) { return T <= 1024 ? 8 : 8; }
 
 }  // namespace
 }  // namespace w8a8
