@@ -524,7 +524,7 @@ def main():
         "stage_ms": st,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": (7 if wl.T <= 512 else 6) * K,
+        "gpu_launches": (5 if (wl.T <= 128 and wl.H <= 2048) else (7 if wl.T <= 512 else 6)) * K,
         "clocks": res["clocks"],
     }
     if not args.no_cpu_baseline:

@@ -112,9 +112,10 @@ int w8a8_moe_route(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, i
  *   sx_sorted fp32 [A_pad]; xq int8 [A_pad, H] (token codes in sorted-row order);
  *   h bf16 [A_pad, I] (SiLU(gate)*up); s_h fp32 [A_pad]; hq int8 [A_pad, I];
  *   o bf16 [T*k, H] (expert outputs in slot order t*k + j);
- *   logits fp32 [T, E] (router logits; written only for short batches, T <= 512). */
+ *   logits fp32 [T, E] (router logits; written only for short batches, T <= 512);
+ *   sync uint32 (grid-barrier counter of the fused short-batch front end, T <= 128). */
 typedef struct {
-  size_t topk_ids, topk_w, tile_counts, offsets, perm, sx, sx_sorted, xq, h, s_h, hq, o, logits;
+  size_t topk_ids, topk_w, tile_counts, offsets, perm, sx, sx_sorted, xq, h, s_h, hq, o, logits, sync;
   size_t total;
 } w8a8_moe_ws_layout;
 

@@ -46,7 +46,7 @@ def test_workspace_queries_are_host_only(lib):
     assert B.w8a8_moe_workspace_size(64, 2048, 128, 8, 768) > 64 * 8 * 2048
     L = B.w8a8_moe_workspace_layout(64, 2048, 128, 8, 768)
     offs = [L[k] for k in ("topk_ids", "topk_w", "tile_counts", "offsets", "perm", "sx", "sx_sorted", "xq",
-                           "h", "s_h", "hq", "o", "logits")]
+                           "h", "s_h", "hq", "o", "logits", "sync")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and L["total"] > offs[-1]
     assert L["o"] + 64 * 8 * 2048 * 2 <= L["logits"] and L["logits"] + 64 * 128 * 4 <= L["total"]
     # rejected shapes report size 0

@@ -39,7 +39,7 @@ class W8A8Error(RuntimeError):
 class _Layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_ids", "topk_w", "tile_counts", "offsets", "perm", "sx", "sx_sorted", "xq", "h",
-                 "s_h", "hq", "o", "logits", "total")]
+                 "s_h", "hq", "o", "logits", "sync", "total")]
 
 
 # (name, restype, argtypes) of every exported entry point

@@ -14,6 +14,8 @@ template <int U>
 __global__ void __launch_bounds__(kRowWarps * 32) quant_rows_kernel(const uint16_t* __restrict__ src,
                                                                     int64_t R, int K, int8_t* __restrict__ q,
                                                                     float* __restrict__ scale) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t r = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
   if (r >= R) return;
   int8_t* dst = q + r * K;
@@ -62,6 +64,8 @@ __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
     const uint16_t* __restrict__ x, const int* __restrict__ ids, const int* __restrict__ tile_counts, int T,
     int H, int E, int k, int* __restrict__ offsets, int* __restrict__ perm, float* __restrict__ sx,
     float* __restrict__ sx_sorted, int8_t* __restrict__ xq_sorted) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ int sm[];
   int* base = sm;                                   // [E]  first sorted row of the chunk's rows of e
   int* before = sm + E;                             // [E]  rows of e in earlier chunks
@@ -161,6 +165,8 @@ __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
 // One CTA per token, 8 columns per thread, no atomics: every y element has one writer.
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ o, const float* __restrict__ w,
                                                       int T, int H, int k, uint16_t* __restrict__ y) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   if (t >= T) return;
   for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {

@@ -392,6 +392,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  // everything above touches only this CTA's own resources; inputs written by the previous
+  // kernel in the stream are read only below
+  pdl_wait();
+  pdl_launch_dependents();
   if (EPI != kEpiRouter && p.group_offsets != nullptr && warp >= 2) {
     // cache the group offsets and build the token-block prefix: one warp-wide scan per 32 groups
     for (int g = threadIdx.x - 64; g <= p.num_groups; g += 32 * kEpiWarps) goff[g] = __ldg(p.group_offsets + g);

@@ -294,6 +294,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
     tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish_pair();
   }
+  // everything above touches only this CTA's own resources; inputs written by the previous
+  // kernel in the stream are read only below
+  pdl_wait();
+  pdl_launch_dependents();
   if (p.group_offsets != nullptr && warp >= 2) {
     for (int g = threadIdx.x - 64; g <= p.num_groups; g += 32 * EW) goff[g] = __ldg(p.group_offsets + g);
     asm volatile("bar.sync 1, %0;" ::"r"(32 * EW) : "memory");

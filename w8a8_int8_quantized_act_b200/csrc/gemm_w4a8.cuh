@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4a8_gemm_kernel(const __grid_c
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();  // xq and sx come from the quantisation kernel launched just before
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -27,6 +27,14 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+// Programmatic dependent launch. Every kernel of the path is launched so that it may start
+// while its predecessor in the stream is finishing; pdl_wait() returns once the predecessor
+// grid has completed and its memory is visible (immediately when launched without the
+// attribute), so each kernel calls it before touching anything a predecessor writes or reads.
+// pdl_launch_dependents() then lets the successor grid be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");

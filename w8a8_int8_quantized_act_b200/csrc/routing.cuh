@@ -86,15 +86,19 @@ __device__ __forceinline__ void warp_topk_token(Logit logit, int E, int k, bool 
 // accumulator per token and vector slot); each lane holds its 1/32 of the expert's row
 // (H <= 256 * RU) in registers.
 constexpr int kSmallRouterTokens = 4;
+
+// One work item of the short-batch router: the calling warp (w8 = its index among the item's 8
+// warps) computes the logits of expert eg * 8 + w8 for tokens tg * kSmallRouterTokens ..
+// + kSmallRouterTokens - 1.
 template <int RU>
-__global__ void __launch_bounds__(256) router_logits_small_kernel(const uint16_t* __restrict__ x,
-                                                                  const uint16_t* __restrict__ wg, int T, int H,
-                                                                  int E, float* __restrict__ logits) {
+__device__ __forceinline__ void router_logits_item(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
+                                                   int T, int H, int E, float* __restrict__ logits, int eg, int tg,
+                                                   int w8) {
   constexpr int TT = kSmallRouterTokens;
   const int lane = threadIdx.x & 31;
-  const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int e = eg * 8 + w8;
   if (e >= E) return;
-  const int t0 = blockIdx.y * TT;
+  const int t0 = tg * TT;
   uint4 wv[RU];
   uint4 xv[TT][RU];
 #pragma unroll
@@ -139,12 +143,23 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(const uint16_t
   }
 }
 
+template <int RU>
+__global__ void __launch_bounds__(256) router_logits_small_kernel(const uint16_t* __restrict__ x,
+                                                                  const uint16_t* __restrict__ wg, int T, int H,
+                                                                  int E, float* __restrict__ logits) {
+  pdl_wait();
+  pdl_launch_dependents();
+  router_logits_item<RU>(x, wg, T, H, E, logits, blockIdx.x, blockIdx.y, threadIdx.x >> 5);
+}
+
 // Top-k over precomputed logits [T, E]: one warp per token. counts has one row of E per
 // 128-token chunk (count_stride = E) or a single row (count_stride = 0).
 template <int PER>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits, const float* bias, int T,
                                                           int E, int k, int renorm, int* ids, float* w, int* counts,
                                                           int count_stride) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
   const float* row = logits + size_t(t) * E;

@@ -8,6 +8,7 @@
 
 #include "../../include/w8a8.h"
 #include "elementwise.cuh"
+#include "front.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_w4a8.cuh"
@@ -107,6 +108,23 @@ bool make_gate_up_pair_map(CUtensorMap* m, const void* base, uint64_t H, uint64_
 // ------------------------------------------------------------------ launch helpers
 int launch_status() { return cudaGetLastError() == cudaSuccess ? W8A8_OK : W8A8_ERR_LAUNCH; }
 
+// Launches `kern` with programmatic stream serialization: it may begin while the previous
+// kernel in the stream finishes (each kernel waits in pdl_wait() before using its inputs).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? W8A8_OK : W8A8_ERR_LAUNCH;
+}
+
 template <int NA, int NB, int EPI, int KIND>
 int launch_gemm(const GemmParams& p, int max_tiles, cudaStream_t stream) {
   using Cfg = GemmCfg<NA, NB, EPI>;
@@ -115,8 +133,7 @@ int launch_gemm(const GemmParams& p, int max_tiles, cudaStream_t stream) {
       cudaSuccess)
     return W8A8_ERR_LAUNCH;
   const int grid = max(1, min(num_sms(), max_tiles));
-  kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(p);
-  return launch_status();
+  return launch_pdl(kern, dim3(grid), dim3(kGemmThreads), Cfg::kSmemBytes, stream, p);
 }
 
 // Clusters of gemm_pair_kernel<EPI> that fit on the device at once (one CTA per SM), cached.
@@ -147,8 +164,7 @@ int launch_pair(const PairParams& p, int max_tiles, cudaStream_t stream) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) != cudaSuccess)
     return W8A8_ERR_LAUNCH;
   const int clusters = max(1, min(pair_clusters<EPI>(), max_tiles));
-  kern<<<2 * clusters, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(p);
-  return launch_status();
+  return launch_pdl(kern, dim3(2 * clusters), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, p);
 }
 
 // Token-row maps of a K-major int8 operand for the pair kernel: 128-, 16- and 8-row boxes.
@@ -203,6 +219,7 @@ void fill_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_
   L->hq = take(size_t(Ap) * I);
   L->o = take(size_t(A) * H * 2);
   L->logits = take(sizeof(float) * T * E);
+  L->sync = take(sizeof(uint32_t));
   L->total = off;
 }
 
@@ -218,26 +235,27 @@ int run_router_small(const uint16_t* x, const uint16_t* wg, const float* bias, i
                      int k, int renorm, int* ids, float* w, int* counts, int64_t count_stride, float* logits,
                      cudaStream_t stream) {
   const dim3 grid1(unsigned((E + 7) / 8), unsigned((T + kSmallRouterTokens - 1) / kSmallRouterTokens));
-  switch (row_units(int(H))) {
-    case 1: router_logits_small_kernel<1><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
-    case 2: router_logits_small_kernel<2><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
-    case 4: router_logits_small_kernel<4><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
-    case 8: router_logits_small_kernel<8><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
-    case 16: router_logits_small_kernel<16><<<grid1, 256, 0, stream>>>(x, wg, int(T), int(H), int(E), logits); break;
+  const dim3 blk(256);
+  const int Ti = int(T), Hi = int(H), Ei = int(E);
+  int rc;
+  switch (row_units(Hi)) {
+    case 1: rc = launch_pdl(router_logits_small_kernel<1>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 2: rc = launch_pdl(router_logits_small_kernel<2>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 4: rc = launch_pdl(router_logits_small_kernel<4>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 8: rc = launch_pdl(router_logits_small_kernel<8>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 16: rc = launch_pdl(router_logits_small_kernel<16>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
     default: return W8A8_ERR_UNSUPPORTED;
   }
-  int rc = launch_status();
   if (rc != W8A8_OK) return rc;
-  const unsigned grid2 = unsigned((T + 7) / 8);
+  const dim3 grid2(unsigned((T + 7) / 8));
   const int cs = int(count_stride);
   switch ((E + 31) / 32) {
-    case 1: router_topk_kernel<1><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
-    case 2: router_topk_kernel<2><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
+    case 1: return launch_pdl(router_topk_kernel<1>, grid2, blk, 0, stream, logits, bias, Ti, Ei, k, renorm, ids, w, counts, cs);
+    case 2: return launch_pdl(router_topk_kernel<2>, grid2, blk, 0, stream, logits, bias, Ti, Ei, k, renorm, ids, w, counts, cs);
     case 3:
-    case 4: router_topk_kernel<4><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
-    default: router_topk_kernel<8><<<grid2, 256, 0, stream>>>(logits, bias, int(T), int(E), k, renorm, ids, w, counts, cs); break;
+    case 4: return launch_pdl(router_topk_kernel<4>, grid2, blk, 0, stream, logits, bias, Ti, Ei, k, renorm, ids, w, counts, cs);
+    default: return launch_pdl(router_topk_kernel<8>, grid2, blk, 0, stream, logits, bias, Ti, Ei, k, renorm, ids, w, counts, cs);
   }
-  return launch_status();
 }
 
 int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t T, int64_t H, int64_t E, int k,
@@ -282,16 +300,15 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
 
 // Launches quant_rows_kernel with the register depth that fits rows of K values.
 int launch_quant_rows(const uint16_t* src, int64_t R, int K, int8_t* q, float* scale, cudaStream_t s) {
-  const unsigned blocks = unsigned((R + kRowWarps - 1) / kRowWarps);
+  const dim3 grid(unsigned((R + kRowWarps - 1) / kRowWarps)), blk(kRowWarps * 32);
   switch (row_units(K)) {
-    case 1: quant_rows_kernel<1><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
-    case 2: quant_rows_kernel<2><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
-    case 4: quant_rows_kernel<4><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
-    case 8: quant_rows_kernel<8><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
-    case 16: quant_rows_kernel<16><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
-    default: quant_rows_kernel<0><<<blocks, kRowWarps * 32, 0, s>>>(src, R, K, q, scale); break;
+    case 1: return launch_pdl(quant_rows_kernel<1>, grid, blk, 0, s, src, R, K, q, scale);
+    case 2: return launch_pdl(quant_rows_kernel<2>, grid, blk, 0, s, src, R, K, q, scale);
+    case 4: return launch_pdl(quant_rows_kernel<4>, grid, blk, 0, s, src, R, K, q, scale);
+    case 8: return launch_pdl(quant_rows_kernel<8>, grid, blk, 0, s, src, R, K, q, scale);
+    case 16: return launch_pdl(quant_rows_kernel<16>, grid, blk, 0, s, src, R, K, q, scale);
+    default: return launch_pdl(quant_rows_kernel<0>, grid, blk, 0, s, src, R, K, q, scale);
   }
-  return launch_status();
 }
 
 int launch_group_quant(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* x, const int* ids,
@@ -300,13 +317,64 @@ int launch_group_quant(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* x
   switch (row_units(H)) {
 #define W8A8_GQ(U_)                                                                                        \
   case U_:                                                                                                 \
-    group_quant_kernel<U_><<<grid, kPermThreads, smem, s>>>(x, ids, tile_counts, T, H, E, k, offsets, perm, \
-                                                            sx, sx_sorted, xq);                            \
-    break;
+    return launch_pdl(group_quant_kernel<U_>, grid, dim3(kPermThreads), smem, s, x, ids, tile_counts, T, H, E, k, \
+                      offsets, perm, sx, sx_sorted, xq);
     W8A8_GQ(1) W8A8_GQ(2) W8A8_GQ(4) W8A8_GQ(8) W8A8_GQ(16) W8A8_GQ(0)
 #undef W8A8_GQ
   }
-  return launch_status();
+  return W8A8_ERR_UNSUPPORTED;
+}
+
+// The fused short-batch front end (front.cuh): one cooperative launch of up to one CTA per SM
+// (all resident at once, which its grid barriers need). Rows of up to 2048 values keep the
+// router's per-lane slices in registers at 512 threads per CTA.
+constexpr int64_t kFrontMaxH = 2048;
+template <int RU, int PER>
+int launch_front_t(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int H, int E, int k, int renorm,
+                   float* logits, unsigned* sync, int* ids, float* w, int* tile_counts, int* offsets, int* perm,
+                   float* sx, float* sx_sorted, int8_t* xq, cudaStream_t s) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(min(num_sms(), kFrontMaxT)));
+  cfg.blockDim = dim3(kFrontThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint64_t timeout = wait_timeout_ns();
+  return cudaLaunchKernelEx(&cfg, front_small_kernel<RU, PER>, x, wg, bias, T, H, E, k, renorm, logits, sync,
+                            timeout, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq) == cudaSuccess
+             ? W8A8_OK
+             : W8A8_ERR_LAUNCH;
+}
+
+template <int RU>
+int launch_front_per(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int H, int E, int k,
+                     int renorm, float* logits, unsigned* sync, int* ids, float* w, int* tile_counts, int* offsets,
+                     int* perm, float* sx, float* sx_sorted, int8_t* xq,
+                     cudaStream_t s) {
+  switch ((E + 31) / 32) {
+    case 1: return launch_front_t<RU, 1>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    case 2: return launch_front_t<RU, 2>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    case 3:
+    case 4: return launch_front_t<RU, 4>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    default: return launch_front_t<RU, 8>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+  }
+}
+
+int launch_front_small(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int H, int E, int k,
+                       int renorm, float* logits, unsigned* sync, int* ids, float* w, int* tile_counts, int* offsets,
+                       int* perm, float* sx, float* sx_sorted, int8_t* xq,
+                     cudaStream_t s) {
+  switch (row_units(H)) {
+    case 1: return launch_front_per<1>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    case 2: return launch_front_per<2>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    case 4: return launch_front_per<4>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    case 8: return launch_front_per<8>(x, wg, bias, T, H, E, k, renorm, logits, sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    default: return W8A8_ERR_UNSUPPORTED;
+  }
 }
 
 // Upper bound of the number of token blocks of `nb` rows over all groups: ceil(A/nb) + min(E, A).
@@ -464,18 +532,29 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   const int C = int((T + kChunk - 1) / kChunk);
   int rc;
 
-  // 1. router (bf16 tcgen05 GEMM + softmax / top-k epilogue, per-chunk expert histogram)
-  mark(ev, 0, s);
-  rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E,
-                  reinterpret_cast<float*>(ws + L.logits), s);
-  if (rc != W8A8_OK) return rc;
+  if (T <= kFrontMaxT && H <= kFrontMaxH) {
+    // 1+2. short batch: routing, grouping and quantisation in one cooperative launch
+    mark(ev, 0, s);
+    unsigned* sync = reinterpret_cast<unsigned*>(ws + L.sync);
+    if (cudaMemsetAsync(sync, 0, sizeof(unsigned), s) != cudaSuccess) return W8A8_ERR_LAUNCH;
+    rc = launch_front_small(x, wg, bias, int(T), int(H), int(E), k, renorm, reinterpret_cast<float*>(ws + L.logits),
+                            sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    if (rc != W8A8_OK) return rc;
+    mark(ev, 1, s);
+  } else {
+    // 1. router (bf16 tcgen05 GEMM + softmax / top-k epilogue, per-chunk expert histogram)
+    mark(ev, 0, s);
+    rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E,
+                    reinterpret_cast<float*>(ws + L.logits), s);
+    if (rc != W8A8_OK) return rc;
 
-  // 2. group assignments by expert and quantise every token once into its sorted rows
-  const size_t gq_smem = sizeof(int) * (2 * E + 2 * kChunk * k + 4 * E);
-  mark(ev, 1, s);
-  rc = launch_group_quant(dim3(C, group_quant_splits(T)), gq_smem, s, x, ids, tile_counts, int(T), int(H), int(E),
-                          k, offsets, perm, sx, sx_sorted, xq);
-  if (rc != W8A8_OK) return rc;
+    // 2. group assignments by expert and quantise every token once into its sorted rows
+    const size_t gq_smem = sizeof(int) * (2 * E + 2 * kChunk * k + 4 * E);
+    mark(ev, 1, s);
+    rc = launch_group_quant(dim3(C, group_quant_splits(T)), gq_smem, s, x, ids, tile_counts, int(T), int(H),
+                            int(E), k, offsets, perm, sx, sx_sorted, xq);
+    if (rc != W8A8_OK) return rc;
+  }
 
   // 3. grouped gate_up GEMM (weights on M, tokens on N) with the dequant + SiLU(gate)*up
   //    epilogue -> h. Few rows per expert (decode): one CTA per tile of <= 32 rows; otherwise
@@ -579,8 +658,7 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
 
   // 6. scatter-free weighted combine
   mark(ev, 5, s);
-  combine_kernel<<<unsigned(T), 256, 0, s>>>(o, w, int(T), int(H), k, y);
-  rc = launch_status();
+  rc = launch_pdl(combine_kernel, dim3(unsigned(T)), dim3(256), 0, s, o, w, int(T), int(H), k, y);
   mark(ev, 6, s);
   return rc;
 }
@@ -702,8 +780,7 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) != cudaSuccess)
       return W8A8_ERR_LAUNCH;
     const int tiles = int((M + 127) / 128) * q.n_cb;
-    kern<<<max(1, min(num_sms(), tiles)), kW4Threads, Cfg::kSmemBytes, s>>>(q);
-    return launch_status();
+    return launch_pdl(kern, dim3(max(1, min(num_sms(), tiles))), dim3(kW4Threads), Cfg::kSmemBytes, s, q);
   }
   if (M > kPairMinRows) {
     PairParams q{};
