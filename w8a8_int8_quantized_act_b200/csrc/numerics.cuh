@@ -138,25 +138,47 @@ __device__ __forceinline__ float dequant(int32_t acc, float s_row, float s_col) 
 }
 
 // Codes of 8 bf16 values (one 16-byte vector) packed into 8 bytes; inv = __frcp_rn(s).
+// Each value: y = v * inv; r = y + 1.5 * 2^23 rounds y to the nearest integer, ties to even,
+// exactly as __float2int_rn for |y| < 2^22, and the low byte of r's bit pattern is that integer
+// as an int8 code (|y| <= 127 * (1 + 2^-22) here, so no clamp is needed). d = y - rint(y) is
+// exact; |d| >= 0.5 - 3e-5 is the same near-tie test as sym_code_fast, and a vector holding such a
+// value takes the true divide for all eight.
 __device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t lo = 0, hi = 0;
+  uint32_t c[8];
+  bool unsure = false;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint32_t a = uint32_t(sym_code_fast(bf16_lo(w[j]), s, inv, 127)) & 0xFFu;
-    const uint32_t b = uint32_t(sym_code_fast(bf16_hi(w[j]), s, inv, 127)) & 0xFFu;
-    const uint32_t pair = a | (b << 8);
-    if (j < 2) lo |= pair << (16 * j); else hi |= pair << (16 * (j - 2));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float x = h ? bf16_hi(w[j]) : bf16_lo(w[j]);
+      const float y = __fmul_rn(x, inv);
+      const float r = __fadd_rn(y, kMagic);
+      const float d = __fsub_rn(y, __fsub_rn(r, kMagic));
+      unsure |= fabsf(d) >= 0.49997f;
+      c[2 * j + h] = __float_as_uint(r);
+    }
   }
+  if (unsure) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      c[2 * j] = uint32_t(sym_code(bf16_lo(w[j]), s, 127));
+      c[2 * j + 1] = uint32_t(sym_code(bf16_hi(w[j]), s, 127));
+    }
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
   return make_uint2(lo, hi);
 }
 
+// max |v| over 8 bf16 values: with the sign bits cleared, the 16-bit patterns of finite bf16
+// values (subnormals included) order like the values, so a per-halfword unsigned maximum is exact.
 __device__ __forceinline__ float amax8(const uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float m = 0.0f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
-  return m;
+  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                              __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return __uint_as_float((m > 0xFFFFu ? (m >> 16) > (m & 0xFFFFu) ? m >> 16 : m & 0xFFFFu : m) << 16);
 }
 
 // Quantises one row of K bf16 values with one warp (K a multiple of 8, row 16-byte aligned):
