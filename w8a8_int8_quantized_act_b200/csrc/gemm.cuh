@@ -335,13 +335,16 @@ __device__ __forceinline__ void epilogue_router(const GemmParams& p, const Tile&
   mbar_arrive(xbar);
   if (!mbar_wait(xbar, xphase, wc)) return;
   xphase ^= 1u;
-  // 2. one warp per token
+  // 2. each warp takes tokens ew, ew + 8, ... four at a time (their selections interleaved)
   int* counts = p.tile_counts != nullptr ? p.tile_counts + size_t(c.tt) * p.tile_count_stride : nullptr;
+  constexpr int NT = 4;
 #pragma unroll 1
-  for (int tl = ew; tl < c.rows; tl += kEpiWarps) {
-    const int row = c.tok0 + tl;
-    warp_topk_token<PER>([&](int e) { return xs[e * 129 + tl]; }, E, k, p.renorm != 0, bias,
-                         static_cast<int*>(p.out) + size_t(row) * k, p.topk_w + size_t(row) * k, counts);
+  for (int tb = ew; tb < c.rows; tb += kEpiWarps * NT) {
+    const int nt = min(NT, (c.rows - tb + kEpiWarps - 1) / kEpiWarps);
+    const int row = c.tok0 + tb;
+    warp_topk_tokens<PER, NT>([&](int u, int e) { return xs[e * 129 + tb + u * kEpiWarps]; }, nt, E, k,
+                              p.renorm != 0, bias, static_cast<int*>(p.out) + size_t(row) * k,
+                              p.topk_w + size_t(row) * k, kEpiWarps * k, counts);
   }
   // 3. buffer free for the next tile once every epilogue thread is past step 2
   mbar_arrive(xbar);

@@ -80,6 +80,102 @@ __device__ __forceinline__ void warp_topk_token(Logit logit, int E, int k, bool 
   }
 }
 
+// The same selection for NT tokens at once by one warp: token u's steps are exactly those of
+// warp_topk_token, and the NT tokens' warp reductions are independent, so they overlap instead
+// of running one dependent chain after another. logit(u, e) for u < nt; token u's outputs at
+// ids + u * ld_out, w + u * ld_out.
+template <int PER, int NT, typename Logit>
+__device__ __forceinline__ void warp_topk_tokens(Logit logit, int nt, int E, int k, bool renorm,
+                                                 const float* __restrict__ bias, int* ids, float* w, int ld_out,
+                                                 int* counts) {
+  const int lane = threadIdx.x & 31;
+  float lv[NT][PER];
+  uint32_t key[NT][PER];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane + 32 * i;
+      const bool valid = e < E && u < nt;
+      float l = 0.0f;
+      if (valid) {
+        l = logit(u, e);
+        if (bias != nullptr) l += __ldg(bias + e);
+      }
+      lv[u][i] = l;
+      key[u][i] = valid ? ordered_key(l) : 0u;
+    }
+  }
+  float pick_v[NT], m[NT];
+  int pick_e[NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    pick_v[u] = 0.0f;
+    m[u] = 0.0f;
+    pick_e[u] = -1;
+  }
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) {
+    uint32_t lbest[NT], wbest[NT], ebest[NT];
+    int li[NT];
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      lbest[u] = 0;
+      li[u] = 0;
+#pragma unroll
+      for (int i = PER - 1; i >= 0; --i)
+        if (key[u][i] >= lbest[u]) { lbest[u] = key[u][i]; li[u] = i; }
+    }
+#pragma unroll
+    for (int u = 0; u < NT; ++u) wbest[u] = warp_max_u32(lbest[u]);
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      const uint32_t cand = (wbest[u] != 0u && lbest[u] == wbest[u]) ? uint32_t(lane + 32 * li[u]) : 0xFFFFFFFFu;
+      ebest[u] = warp_min_u32(cand);
+    }
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      if (ebest[u] != 0xFFFFFFFFu && int(ebest[u] & 31u) == lane) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+          if (i == int(ebest[u] >> 5)) key[u][i] = 0u;
+      }
+      const float v = from_ordered_key(wbest[u]);
+      if (j == 0) m[u] = v;
+      if (lane == j) {
+        pick_v[u] = v;
+        pick_e[u] = (ebest[u] == 0xFFFFFFFFu) ? -1 : int(ebest[u]);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    const float ev = (lane < k && pick_e[u] >= 0) ? expf(pick_v[u] - m[u]) : 0.0f;
+    float denom = ev;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+    if (!renorm) {
+      float sall = 0.0f;
+#pragma unroll
+      for (int i = 0; i < PER; ++i)
+        if (lane + 32 * i < E) sall += expf(lv[u][i] - m[u]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sall += __shfl_xor_sync(0xffffffffu, sall, o);
+      denom = sall;
+    }
+    if (u < nt && lane < k) {
+      int e = pick_e[u];
+      if (e < 0) {
+        atomicOr(&g_error_word, kErrBadIndex);
+        e = lane;
+      }
+      ids[u * ld_out + lane] = e;
+      w[u * ld_out + lane] = ev / denom;
+      if (counts != nullptr) atomicAdd(counts + e, 1);
+    }
+  }
+}
+
 // Router logits on the CUDA cores for short batches: logits[t, e] = sum_h x[t, h] * wg[e, h] in
 // fp32 (bf16 inputs). Block = 8 warps; warp w takes expert blockIdx.x * 8 + w and the
 // kSmallRouterTokens tokens of blockIdx.y together (all their loads in flight at once, one
