@@ -64,8 +64,11 @@ struct PairCfg {
   static constexpr int kBarBytes = 512;
   // per accumulator set: the tile's row scales and row map, staged once for all epilogue warps
   static constexpr int kRowBytes = 2 * 2 * kPairNB * 4;
-  static constexpr size_t kSmemBytes =
-      1024 + size_t(kStages) * kStageBytes + kBarBytes + kRowBytes + 2 * sizeof(int) * (kMaxGroups + 1);
+  // down / dense: per epilogue warp a 16-token x 32-channel bf16 block, transposed through
+  // shared memory so that the output leaves in 16-byte row pieces
+  static constexpr int kXposeBytes = (EPI == kEpiDown || EPI == kEpiDense) ? kEpiWarps * 16 * 32 * 2 : 0;
+  static constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + kBarBytes + kRowBytes + kXposeBytes +
+                                       2 * sizeof(int) * (kMaxGroups + 1);
   static_assert(kTmemCols <= 512, "two accumulator sets must fit in TMEM");
   static_assert(kEpiWarps % 4 == 0, "whole lane quarters");
 };
@@ -199,10 +202,12 @@ __device__ __forceinline__ void pair_epilogue_gate_up(const PairParams& p, const
 }
 
 // down / dense / raw epilogue: lane = one output channel of the CTA's 128, columns = tokens.
-// srow / smap: the tile's row scales and (down) output rows in shared memory.
+// srow / smap: the tile's row scales and (down) output rows in shared memory; xp: this warp's
+// 16 x 32 bf16 transpose block (down / dense).
 template <int EPI, int W>
 __device__ __forceinline__ void pair_epilogue_channels(const PairParams& p, const PairTile& c, uint32_t t_lane,
-                                                       int ch, int wq, const float* srow, const int* smap) {
+                                                       int ch, int wq, const float* srow, const int* smap,
+                                                       uint16_t* xp) {
   const bool valid = ch < p.n_channels;
   const size_t ldo = size_t(p.ldo);
   const int rows = c.rows;
@@ -215,34 +220,40 @@ __device__ __forceinline__ void pair_epilogue_channels(const PairParams& p, cons
         if (valid && j < nj) out[size_t(c.tok0 + j0 + j) * ldo] = int32_t(r[j]);
     });
   } else {
+    // bf16 values go through this warp's 16 x 32 shared-memory block: lane = channel on the way
+    // in, then four lanes per token row (8 channels = 16 bytes each) on the way out
     const float s_col = valid ? __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch) : 0.0f;
-    uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
+    const int lane = threadIdx.x & 31;
+    const int ch0 = ch - lane;                      // first channel of the warp's 32
+    const int jr = lane >> 2, cc = (lane & 3) * 8;  // token row (and row + 8), channel piece
+    uint16_t* outb = static_cast<uint16_t*>(p.out) + ch0 + cc;
     pair_chunks<W>(t_lane, rows, wq, [&](uint32_t(&r)[16], int j0) {
       const int nj = min(16, rows - j0);
       float sr[16];
-      int orow[16];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float4 f = *reinterpret_cast<const float4*>(srow + j0 + 4 * i);
         sr[4 * i] = f.x; sr[4 * i + 1] = f.y; sr[4 * i + 2] = f.z; sr[4 * i + 3] = f.w;
-        if constexpr (EPI == kEpiDown) {
-          const int4 m = *reinterpret_cast<const int4*>(smap + j0 + 4 * i);
-          orow[4 * i] = m.x; orow[4 * i + 1] = m.y; orow[4 * i + 2] = m.z; orow[4 * i + 3] = m.w;
-        } else {
+      }
 #pragma unroll
-          for (int t = 0; t < 4; ++t) orow[4 * i + t] = c.tok0 + j0 + 4 * i + t;
+      for (int j = 0; j < 16; j += 2) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(dequant(int32_t(r[j]), sr[j], s_col),
+                                                        dequant(int32_t(r[j + 1]), sr[j + 1], s_col));
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(&h2);
+        xp[j * 32 + lane] = uint16_t(v);
+        xp[(j + 1) * 32 + lane] = uint16_t(v >> 16);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int j = jr + 8 * hr;
+        const uint4 piece = *reinterpret_cast<const uint4*>(xp + j * 32 + cc);
+        if (j < nj && ch0 < p.n_channels) {
+          const int orow = (EPI == kEpiDown) ? smap[j0 + j] : c.tok0 + j0 + j;
+          *reinterpret_cast<uint4*>(outb + size_t(orow) * ldo) = piece;
         }
       }
-      uint32_t v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(dequant(int32_t(r[2 * j]), sr[2 * j], s_col),
-                                                        dequant(int32_t(r[2 * j + 1]), sr[2 * j + 1], s_col));
-        v[j] = *reinterpret_cast<const uint32_t*>(&h2);
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (valid && j < nj) out[size_t(orow[j]) * ldo] = uint16_t(v[j >> 1] >> (16 * (j & 1)));
+      __syncwarp();  // the block is rewritten by the next chunk
     });
   }
 }
@@ -265,7 +276,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rready + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* rows_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + Cfg::kBarBytes);  // [2][2][256]
-  int* mt_prefix = reinterpret_cast<int*>(rows_smem + 4 * kPairNB);
+  uint16_t* xpose = reinterpret_cast<uint16_t*>(rows_smem + 4 * kPairNB);  // [EW][16][32] (down / dense)
+  int* mt_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(xpose) + Cfg::kXposeBytes);
   int* goff = mt_prefix + (kMaxGroups + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -462,21 +474,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
     const uint32_t tempty0 = map_to_rank(smem_addr(tempty), 0);
     int acc = 0, g_hint = 0;
     uint32_t acc_phase = 0;
-    for (PairTileIter it(cluster, nclusters, p.n_cb); it.mt < total_mt; it.next()) {
-      const PairTile c = pair_tile(p, mt_prefix, goff, it.mt, it.cb, g_hint);
-      // stage the tile's row scales (and output rows) while the MMAs run. The buffer of this
-      // accumulator set was last read two tiles ago, and every epilogue thread has arrived on
-      // the previous tile's rready barrier, so all of them are done with it. (An mbarrier, not
-      // a named barrier: its wait is bounded, so a CTA that aborts cannot strand the others.)
+    // Row scales (and output rows) of a tile are loaded into registers one tile ahead, so their
+    // memory latency overlaps the previous tile's epilogue; thread et holds row et (< 256).
+    static_assert(32 * EW >= kPairNB, "one row per epilogue thread");
+    float pre_s = 0.0f;
+    int pre_m = 0;
+    auto load_rows = [&](const PairTile& t) {
+      const bool in = et < t.rows;
+      if constexpr (EPI != kEpiRawS32) pre_s = in ? __ldg(p.row_scale + t.tok0 + et) : 0.0f;
+      if constexpr (EPI == kEpiDown) pre_m = in ? __ldg(p.row_map + t.tok0 + et) : 0;
+    };
+    PairTileIter it(cluster, nclusters, p.n_cb);
+    PairTile c{};
+    if (it.mt < total_mt) {
+      c = pair_tile(p, mt_prefix, goff, it.mt, it.cb, g_hint);
+      load_rows(c);
+    }
+    while (it.mt < total_mt) {
+      // stage the tile's rows for all epilogue warps. The buffer of this accumulator set was last
+      // read two tiles ago, and every epilogue thread has arrived on the previous tile's rready
+      // barrier, so all of them are done with it. (An mbarrier, not a named barrier: its wait
+      // is bounded, so a CTA that aborts cannot strand the others.)
       float* srow = rows_smem + acc * 2 * kPairNB;
       int* smap = reinterpret_cast<int*>(srow + kPairNB);
-      for (int i = et; i < kPairNB; i += 32 * EW) {
-        const bool in = i < c.rows;
-        if constexpr (EPI != kEpiRawS32) srow[i] = in ? __ldg(p.row_scale + c.tok0 + i) : 0.0f;
-        if constexpr (EPI == kEpiDown) smap[i] = in ? __ldg(p.row_map + c.tok0 + i) : 0;
+      if (et < kPairNB) {
+        srow[et] = pre_s;
+        smap[et] = pre_m;
       }
       mbar_arrive(rready + acc);
       if (!mbar_wait(rready + acc, acc_phase, wc)) break;
+      PairTileIter nx = it;
+      nx.next();
+      PairTile cn{};
+      if (nx.mt < total_mt) {
+        cn = pair_tile(p, mt_prefix, goff, nx.mt, nx.cb, g_hint);
+        load_rows(cn);
+      }
       if (!mbar_wait(tfull + acc, acc_phase, wc)) break;
       tc_fence_after();
       const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * Cfg::kAccCols);
@@ -485,12 +518,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
         pair_epilogue_gate_up<EW / 4>(p, c, t_lane, ch, lane >= 16, wq, srow);
       } else {
         pair_epilogue_channels<EPI, EW / 4>(p, c, t_lane, c.cb * 256 + int(rank) * 128 + q * 32 + lane, wq, srow,
-                                            smap);
+                                            smap, xpose + (warp - 2) * 16 * 32);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      it = nx;
+      c = cn;
     }
   }
 
