@@ -146,6 +146,16 @@ def test_moe_edge_shapes(T, E, k, I):
     _full_check(G.run_moe(wl))
 
 
+# The fused short-batch front end (one cooperative kernel, T <= 128, H <= 2048) at its extremes:
+# a full 128-token chunk, 256 experts with k = 16, one token, hidden 2048 (the largest row held in
+# registers). Routing against the oracle's router, every integer stage and y bit for bit.
+@pytest.mark.parametrize("T,H,E,k,I", [(128, 2048, 128, 8, 128), (1, 2048, 256, 16, 128), (97, 1024, 64, 6, 256),
+                                       (128, 128, 256, 1, 128)])
+def test_moe_fused_front_end_shapes(T, H, E, k, I):
+    wl = synth.MoEWorkload("front", T=T, H=H, E=E, k=k, I=I, n_outlier=2, seed=T + E)
+    _full_check(G.run_moe(wl))
+
+
 # Long token lists (the CTA-pair GEMMs): several 256-row blocks per expert with ragged tails,
 # an odd number of 128-channel blocks in the down projection (H = 384), a single expert.
 @pytest.mark.parametrize("T,H,E,k,I", [(600, 384, 4, 2, 256), (1031, 256, 8, 3, 128), (700, 512, 1, 1, 384),
