@@ -206,6 +206,14 @@ int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, i
  * CTA-pair gate_up GEMM relies on this distance being at most 2. */
 int w8a8_debug_rcp_approx_ulp(uint32_t first_bits, uint32_t count, unsigned int* max_ulp, w8a8_stream stream);
 
+/* Test hook for the certified SiLU evaluation: writes to *max_ulp (device memory, one uint32)
+ * the largest distance, in units in the last place, between the hardware's approximate base-2
+ * exponential (ex2.approx.ftz.f32) and 2^x computed in double precision and rounded to fp32, over
+ * the `count` fp32 bit patterns starting at `first_bits`. They must share one sign and satisfy
+ * |x| < 126 (2^x normal), else W8A8_ERR_ARG. The gated-activation epilogue of the CTA-pair
+ * gate_up GEMM relies on this distance being at most 3. */
+int w8a8_debug_ex2_approx_ulp(uint32_t first_bits, uint32_t count, unsigned int* max_ulp, w8a8_stream stream);
+
 /* Test hook for the bounded waits: launches one CTA that waits on an mbarrier phase nothing
  * completes; after `timeout_ns` the wait gives up and sets the device error word, which the
  * next w8a8_check_status() reports as W8A8_ERR_DEVICE. The context stays usable. */

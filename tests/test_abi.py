@@ -77,6 +77,8 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_debug_rcp_approx_ulp(0, 10, c(16), None) == B.W8A8_ERR_ARG  # not a normal input
     assert lib.w8a8_debug_rcp_approx_ulp(0x7E7FFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # reciprocal subnormal
+    assert lib.w8a8_debug_ex2_approx_ulp(0x7FFFFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # crosses the sign
+    assert lib.w8a8_debug_ex2_approx_ulp(0x43000000, 4, c(16), None) == B.W8A8_ERR_ARG  # 2^128 overflows
 
 
 def test_package_has_no_oracle_dependency():

@@ -242,6 +242,19 @@ def test_rcp_approx_within_two_ulp():
         assert B.w8a8_debug_rcp_approx_ulp(first, 1 << 23) <= 2
 
 
+def test_ex2_approx_within_three_ulp():
+    # The same epilogue computes e^-g as ex2.approx of a split argument; its bound needs ex2.approx
+    # within 3 ulps of 2^x. Every fp32 x with 2^-40 <= |x| < 126, both signs (the fast path only
+    # takes |g| <= 64, i.e. |x| < 93).
+    worst = 0
+    for sign in (0, 0x80000000):
+        for exp_field in range(127 - 40, 127 + 6):  # 2^-40 <= |x| < 64, whole binades
+            worst = max(worst, B.w8a8_debug_ex2_approx_ulp(sign | (exp_field << 23), 1 << 23))
+        first = sign | 0x42800000  # 64 <= |x| < 126
+        worst = max(worst, B.w8a8_debug_ex2_approx_ulp(first, 0x42FC0000 - 0x42800000))
+    assert worst <= 3, worst
+
+
 # ------------------------------------------------------------------ failure detection
 def test_bounded_wait_reports_timeout_and_context_survives():
     B.w8a8_debug_wait_timeout(2_000_000)  # 2 ms

@@ -64,6 +64,7 @@ SIGNATURES = {
     "w8a8_gemm_s8s8s32": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
     "w8a8_debug_rcp_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
+    "w8a8_debug_ex2_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
 }
 
 _lib = None
@@ -304,6 +305,15 @@ def w8a8_debug_rcp_approx_ulp(first_bits: int, count: int, stream=None) -> int:
     out = torch.empty(1, dtype=torch.int32, device="cuda")
     _check(lib().w8a8_debug_rcp_approx_ulp(first_bits, count, _ptr(out), _stream(stream)),
            "w8a8_debug_rcp_approx_ulp")
+    return int(out.cpu().item())
+
+
+def w8a8_debug_ex2_approx_ulp(first_bits: int, count: int, stream=None) -> int:
+    """Largest ulp distance of ex2.approx from 2^x (computed in double, rounded to fp32) over a
+    range of fp32 bit patterns."""
+    out = torch.empty(1, dtype=torch.int32, device="cuda")
+    _check(lib().w8a8_debug_ex2_approx_ulp(first_bits, count, _ptr(out), _stream(stream)),
+           "w8a8_debug_ex2_approx_ulp")
     return int(out.cpu().item())
 
 

@@ -208,6 +208,23 @@ __global__ void rcp_approx_ulp_kernel(uint32_t first, uint32_t count, unsigned i
   if ((threadIdx.x & 31) == 0) atomicMax(max_ulp, worst);
 }
 
+// Largest distance, in units in the last place, between ex2.approx.ftz.f32(x) and 2^x computed
+// in double and rounded to fp32, over the fp32 bit patterns first .. first + count - 1 (finite x
+// whose 2^x is a normal fp32). The certified SiLU evaluation assumes this is at most 3.
+__global__ void ex2_approx_ulp_kernel(uint32_t first, uint32_t count, unsigned int* max_ulp) {
+  unsigned int worst = 0;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x) {
+    const float x = __uint_as_float(first + i);
+    float a;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(a) : "f"(x));
+    const float ref = __double2float_rn(exp2(double(x)));
+    const int diff = int(__float_as_uint(a)) - int(__float_as_uint(ref));
+    worst = max(worst, unsigned(diff < 0 ? -diff : diff));
+  }
+  worst = warp_max_u32(worst);
+  if ((threadIdx.x & 31) == 0) atomicMax(max_ulp, worst);
+}
+
 // Host-visible probe of the bounded-wait machinery: waits on an mbarrier phase that nothing
 // completes, so the wait must run out after `timeout_ns` and raise the error word.
 __global__ void wait_timeout_probe_kernel(uint64_t timeout_ns) {

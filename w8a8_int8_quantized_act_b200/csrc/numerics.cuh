@@ -106,22 +106,33 @@ __device__ __forceinline__ float div_certified(float g, float d, bool& ok) {
   return (g == 0.0f) ? g : q1;
 }
 
-// bf16(fl(SiLU(g) * u)), the gated activation as the layer defines it (SiLU with the exact
-// quotient g / (1 + exp_cw(-g))), evaluated cheaply and certified at the bf16 level:
-//   Y = fl(fl(g * rcp.approx(d)) * u),  d = fl(1 + exp_cw(-g))   (the same d as the definition)
-// differs from S = fl(fl(g / d) * u) by the reciprocal's error and four fp32 roundings:
-// |Y/S - 1| <= eps_rcp + 4 * 2^-24 + O(2^-48). With rcp.approx within 2 ulp of the correctly
-// rounded reciprocal (eps_rcp <= 5 * 2^-24; a GPU test measures it over a whole binade), Y is
-// within 9 fp32 ulps of S whenever Y is a normal number. bf16 rounding looks only at the low 16
-// bits of the fp32 pattern (round up above 0x8000, ties to even at 0x8000), so if those bits of
-// Y are more than kBf16Margin = 16 ulps away from 0x8000, S lies in the same bf16 rounding
-// interval and bf16(Y) = bf16(S). (Near a binade boundary the low bits are near 0 or 0xFFFF and
-// both round to the same power of two.) Accepted only for |g| <= 64 (exp_cw needs no range
-// handling there and d < 2^93) and 2^-120 <= |Y| < 2^121; `ok` is false otherwise, and the
-// caller then evaluates silu_exact. Returns Y.
-constexpr uint32_t kBf16Margin = 16;
+// bf16(fl(SiLU(g) * u)), the gated activation as the layer defines it, S = fl(fl(g / d) * u)
+// with d = fl(1 + exp_cw(-g)), evaluated cheaply and certified at the bf16 level:
+//   x = -g * log2(e) as xh + xl (xh = fl(-g * L), xl its exact FMA residual plus -g * (log2 e - L));
+//   e' = 2^xh (ex2.approx) * (1 + xl ln 2);  d' = fl(1 + e');  Y = fl(fl(g * rcp.approx(d')) * u).
+// Error: e' is within eps_ex2 + 2^-23 of e^-g (the split leaves |xl| <= 2^-18, so the first-order
+// correction is exact to 2^-36); exp_cw is within 3 ulp (6 * 2^-24) of it; hence
+// |d'/d - 1| <= eps_ex2 + 10 * 2^-24, and with the reciprocal's eps_rcp and four fp32 roundings,
+// |Y/S - 1| <= eps_ex2 + eps_rcp + 14 * 2^-24. GPU tests measure ex2.approx within 3 ulp and
+// rcp.approx within 2 ulp of the correctly rounded results (eps <= 7 and 5 * 2^-24), so Y is
+// within 26 fp32 ulps of S whenever Y is a normal number. bf16 rounding looks only at the low 16
+// bits of the fp32 pattern (round up above 0x8000, ties to even at 0x8000), so if those bits of Y
+// are more than kBf16Margin = 40 ulps away from 0x8000, S lies in the same bf16 rounding interval
+// and bf16(Y) = bf16(S). (Near a binade boundary the low bits are near 0 or 0xFFFF and both round
+// to the same power of two.) Accepted only for |g| <= 64 (d < 2^93, every step in range) and
+// 2^-120 <= |Y| < 2^121; `ok` is false otherwise, and the caller then evaluates silu_exact.
+constexpr uint32_t kBf16Margin = 40;
 __device__ __forceinline__ float silu_mul_bf16_certified(float g, float u, bool& ok) {
-  const float d = __fadd_rn(1.0f, exp_cw_core(-g));
+  const float L = 1.44269502162933349609375f;                  // fl(log2 e)
+  const float Llo = (float)(1.4426950408889634 - 1.44269502162933349609375);
+  const float ng = -g;
+  const float xh = __fmul_rn(ng, L);
+  float xl = __fmaf_rn(ng, L, -xh);
+  xl = __fmaf_rn(ng, Llo, xl);
+  float e1;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(xh));
+  const float e = __fmaf_rn(e1, __fmul_rn(xl, 0.693147180559945309f), e1);
+  const float d = __fadd_rn(1.0f, e);
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
   const float y = __fmul_rn(__fmul_rn(g, r), u);

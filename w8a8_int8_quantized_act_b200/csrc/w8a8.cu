@@ -870,6 +870,19 @@ int w8a8_debug_rcp_approx_ulp(uint32_t first_bits, uint32_t count, unsigned int*
   return launch_status();
 }
 
+int w8a8_debug_ex2_approx_ulp(uint32_t first_bits, uint32_t count, unsigned int* max_ulp, w8a8_stream stream) {
+  if (!max_ulp || count == 0) return W8A8_ERR_ARG;
+  const uint64_t first = first_bits, last = first + count - 1;
+  // one sign only, and 2^x a normal number: |x| < 126
+  if ((first >> 31) != (last >> 31) || (first & 0x7FFFFFFFu) >= 0x42FC0000u || (last & 0x7FFFFFFFu) >= 0x42FC0000u)
+    return W8A8_ERR_ARG;
+  if (cudaMemsetAsync(max_ulp, 0, sizeof(unsigned int), as_stream(stream)) != cudaSuccess) return W8A8_ERR_LAUNCH;
+  const uint64_t want = (uint64_t(count) + 255) / 256;
+  const unsigned blocks = unsigned(want < 4096 ? want : 4096);
+  ex2_approx_ulp_kernel<<<blocks, 256, 0, as_stream(stream)>>>(first_bits, count, max_ulp);
+  return launch_status();
+}
+
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {
   if (timeout_ns == 0 || timeout_ns > 10ull * 1000 * 1000 * 1000) return W8A8_ERR_ARG;
   wait_timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns);
