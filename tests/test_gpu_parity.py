@@ -233,6 +233,20 @@ def test_linear_w4a8_extreme_codes():
     np.testing.assert_array_equal(G.host(y), O.linear_w4a8(x, op, os_, 128))
 
 
+def test_linear_w4a8_largest_group_sums():
+    # every group partial at the largest magnitude the codes allow, 127 * 7 * 128, with both signs
+    M, K, N = 96, 384, 256
+    sign = np.where(np.arange(M) % 2 == 1, -1.0, 1.0).astype(np.float32)
+    x = O.f32_to_bf16(np.repeat((sign * (1.0 + 0.01 * np.arange(M)))[:, None], K, axis=1).astype(np.float32))
+    w = O.f32_to_bf16(np.full((N, K), 0.07, np.float32) * np.where(np.arange(N) % 3 == 0, -1.0, 1.0)[:, None]
+                      .astype(np.float32))
+    packed, s = B.w8a8_quantize_weight_int4_per_group(G.bf16_dev(w), 128)
+    op, os_ = O.quantize_weight_int4_per_group(w, 128)
+    assert np.all((op == 0x77) | (op == 0x99))  # +7 and -7 in both nibbles
+    y = B.w8a8_linear(G.bf16_dev(x), packed, s, B.W8A8_W_INT4_PER_GROUP, 128)
+    np.testing.assert_array_equal(G.host(y), O.linear_w4a8(x, op, os_, 128))
+
+
 # ------------------------------------------------------------------ hardware premise of the certified SiLU
 def test_rcp_approx_within_two_ulp():
     # The gate_up epilogue of the CTA-pair GEMM accepts bf16(fl(fl(g * rcp.approx(d)) * u)) only

@@ -775,12 +775,12 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
     q.sx = sx;
     q.y = y;
     q.timeout_ns = wait_timeout_ns();
-    using Cfg = W4Cfg<128>;
-    auto kern = w4a8_gemm_kernel<128>;
+    using Cfg = W4Cfg<128, 4, 8>;
+    auto kern = w4a8_gemm_kernel<128, 4, 8>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) != cudaSuccess)
       return W8A8_ERR_LAUNCH;
     const int tiles = int((M + 127) / 128) * q.n_cb;
-    return launch_pdl(kern, dim3(max(1, min(num_sms(), tiles))), dim3(kW4Threads), Cfg::kSmemBytes, s, q);
+    return launch_pdl(kern, dim3(max(1, min(num_sms(), tiles))), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, q);
   }
   if (M > kPairMinRows) {
     PairParams q{};
