@@ -26,8 +26,8 @@
 //               kASlots K-blocks ahead of the MMA;
 //   EW warps    epilogue: each K-block out of TMEM, acc = fma((float)acc_g, s_w[n, g], acc) in
 //               fp32 registers, and the TMEM buffer reset to the start pattern. At a tile's end
-//               bf16(acc * s_x[t]) leaves through a per-warp shared-memory transpose in 16-byte
-//               row pieces.
+//               bf16(acc * s_x[t]) goes into a shared-memory copy of the output tile, which one
+//               thread hands to a TMA bulk store while the warps go on with the next tile.
 // The packed ring is released as soon as a block is in registers, so weight loads run far ahead;
 // the MMA waits only for the converted block, its token rows and a free TMEM buffer.
 #pragma once
@@ -39,13 +39,14 @@ struct W4A8Params {
   CUtensorMap tmW;   // packed weights [N, K/2] bytes, box 128 rows x 64 bytes, no swizzle
   CUtensorMap tmX;   // xq [Mp, K] int8, box 16 rows x 128 bytes, 128-byte swizzle
   CUtensorMap tmX2;  // xq, box NB rows (full token tiles)
+  CUtensorMap tmY;   // y [M, N] bf16 seen as bytes, box NB rows x 256 bytes (128 channels), no swizzle
   int num_kb;        // K / 128 (= number of scale groups)
   int n_cb;          // N / 128
   int M;             // tokens
   int N;
   const float* sw;   // [N, num_kb]
+  int sw_vec;        // rows of sw start on 16-byte boundaries (num_kb % 4 == 0, sw aligned)
   const float* sx;   // [M]
-  uint16_t* y;       // [M, N] bf16
   uint64_t timeout_ns;
 };
 
@@ -65,7 +66,7 @@ struct W4Cfg {
   static constexpr int kWBytes = kBM * 64;            // packed weights of one K-block
   static constexpr int kXStages = 6;
   static constexpr int kASlots = 3;
-  static constexpr int kWStages = 6;
+  static constexpr int kWStages = 5;
   static constexpr int kAccBufs = 4;
   static constexpr int kTmemCols = 512;
   static_assert(kAccBufs * NB <= kTmemCols, "accumulator buffers must fit in TMEM");
@@ -73,13 +74,13 @@ struct W4Cfg {
   static constexpr int kAOff = kXOff + kXStages * kXBytes;
   static constexpr int kWOff = kAOff + kASlots * kABytes;
   static constexpr int kBarOff = kWOff + kWStages * kWBytes;
-  static constexpr int kXposeOff = kBarOff + 512;
-  static constexpr int kXposeBytes = EW * 16 * 32 * 2;  // per warp: 16 tokens x 32 channels
-  static constexpr int kSxOff = kXposeOff + kXposeBytes;
+  static constexpr int kOutOff = kBarOff + 512;
+  static constexpr int kOutBytes = NB * kBM * 2;  // the bf16 output tile, [token][channel]
+  static constexpr int kSxOff = kOutOff + kOutBytes;
   static constexpr int kSxBytes = EW * kCols * 4;       // per warp: its tokens' s_x
   static constexpr size_t kSmemBytes = 1024 + size_t(kSxOff) + kSxBytes;
   static_assert(kXBytes % 1024 == 0 && kABytes % 1024 == 0, "128-byte swizzled tiles sit on 1 KB boundaries");
-  static_assert(2 * (kXStages + kWStages + kASlots + kAccBufs) * 8 + 8 + 8 + 8 <= 512, "barrier block");
+  static_assert(2 * (kXStages + kWStages + kASlots + kAccBufs + 1) * 8 + 8 + 8 + 8 <= 512, "barrier block");
 };
 
 // 8 packed bytes (16 int4 codes) -> 16 int8 bytes in k order holding 16 * code: the high nibble
@@ -163,10 +164,12 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
   uint64_t* aempty = aready + AS;
   uint64_t* tfull = aempty + AS;
   uint64_t* tempty = tfull + Cfg::kAccBufs;
-  uint64_t* drain = tempty + Cfg::kAccBufs;
+  uint64_t* ofree = tempty + Cfg::kAccBufs;  // the output tile may be rewritten
+  uint64_t* ostaged = ofree + 1;              // the output tile is written
+  uint64_t* drain = ostaged + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint16_t* xpose = reinterpret_cast<uint16_t*>(smem + Cfg::kXposeOff);
+  uint8_t* out_tile = smem + Cfg::kOutOff;
   float* sx_smem = reinterpret_cast<float*>(smem + Cfg::kSxOff);
   auto x_of = [&](int s) { return smem + Cfg::kXOff + s * Cfg::kXBytes; };
   auto a_of = [&](int s) { return smem + Cfg::kAOff + s * Cfg::kABytes; };
@@ -181,12 +184,15 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
     for (int s = 0; s < WS; ++s) { mbar_init(wfull + s, 1); mbar_init(wempty + s, Cfg::kConverters); }
     for (int s = 0; s < AS; ++s) { mbar_init(aready + s, Cfg::kConverters); mbar_init(aempty + s, 1); }
     for (int a = 0; a < Cfg::kAccBufs; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, Cfg::kEpilogue); }
+    mbar_init(ofree, 1);
+    mbar_init(ostaged, Cfg::kEpilogue);
     mbar_init(drain, 1);
     fence_mbar_init();
     *abort_flag = 0;
     tma_prefetch_map(&p.tmW);
     tma_prefetch_map(&p.tmX);
     tma_prefetch_map(&p.tmX2);
+    tma_prefetch_map(&p.tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
@@ -339,30 +345,45 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
     // ------------------------------------------------------------ epilogue (warps E0 ..)
     const int q = warp & 3;
     const int j0 = ((warp - E0) >> 2) * CW;  // this warp's token columns [j0, j0 + CW)
-    uint16_t* xp = xpose + (warp - E0) * 16 * 32;
+    const bool leader = threadIdx.x == E0 * 32;  // hands the output tile to the TMA store
     float* sxw = sx_smem + (warp - E0) * CW;
     const uint64_t neg_c2 = pack_f32x2(-kW4AccStart, -kW4AccStart);
-    const int jr = lane >> 2, cc = (lane & 3) * 8;  // store phase: token row (and row + 8), channel piece
+    // s_w of this lane's channel, four K-blocks per load, one group of four ahead
+    auto load_s4 = [&](const float* row, int k0) -> float4 {
+      if (p.sw_vec) return __ldg(reinterpret_cast<const float4*>(row + k0));
+      float4 v;
+      v.x = k0 < nkb ? __ldg(row + k0) : 0.0f;
+      v.y = k0 + 1 < nkb ? __ldg(row + k0 + 1) : 0.0f;
+      v.z = k0 + 2 < nkb ? __ldg(row + k0 + 2) : 0.0f;
+      v.w = k0 + 3 < nkb ? __ldg(row + k0 + 3) : 0.0f;
+      return v;
+    };
     bool ok = true;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int stored = 0;  // output tiles handed to the TMA store so far
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
       const int tok0 = mt * NB, rows = min(NB, p.M - tok0);
-      const int ch0 = cb * kBM + q * 32;  // first channel of the warp's 32
-      const float* __restrict__ swr = p.sw + size_t(ch0 + lane) * nkb;
+      const int ch = q * 32 + lane;  // channel within the tile
+      const float* __restrict__ swr = p.sw + size_t(cb * kBM + ch) * nkb;
       float accf[CW];
 #pragma unroll
       for (int j = 0; j < CW; ++j) accf[j] = 0.0f;
-      float s_next = __ldg(swr);
+      float4 s_cur = load_s4(swr, 0);
+      float4 s_nxt = load_s4(swr, 4);
       // the s_x of the warp's tokens, needed only at the tile's end: loaded now
       float sxr[CW / 32];
 #pragma unroll
       for (int i = 0; i < CW / 32; ++i)
         sxr[i] = (j0 + 32 * i + lane < rows) ? __ldg(p.sx + tok0 + j0 + 32 * i + lane) : 0.0f;
       for (int kb = 0; kb < nkb; ++kb) {
-        const float s = s_next;
-        if (kb + 1 < nkb) s_next = __ldg(swr + kb + 1);  // next group's scale, loaded early
+        const int k4 = kb & 3;
+        const float s = k4 == 0 ? s_cur.x : (k4 == 1 ? s_cur.y : (k4 == 2 ? s_cur.z : s_cur.w));
+        if (k4 == 3) {
+          s_cur = s_nxt;
+          if (kb + 5 < nkb) s_nxt = load_s4(swr, kb + 5);
+        }
         // warp-uniform outcome: the TMEM loads and stores below are warp-collective
         if (!mbar_wait_warp(tfull + acc, acc_phase, wc)) { ok = false; break; }
         tc_fence_after();
@@ -387,38 +408,39 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
         if (++acc == Cfg::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) break;
-      if (j0 >= rows) continue;
-#pragma unroll
-      for (int i = 0; i < CW / 32; ++i) sxw[32 * i + lane] = sxr[i];
-      __syncwarp();
-      uint16_t* outb = p.y + ch0 + cc;
-#pragma unroll
-      for (int c16 = 0; c16 < CW; c16 += 16) {
-        // lane = channel on the way in, four lanes per token row (16 bytes each) on the way out
-#pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const float4 sv = *reinterpret_cast<const float4*>(sxw + c16 + j);
-          const __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(accf[c16 + j], sv.x),
-                                                          __fmul_rn(accf[c16 + j + 1], sv.y));
-          const __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(accf[c16 + j + 2], sv.z),
-                                                          __fmul_rn(accf[c16 + j + 3], sv.w));
-          const uint32_t v0 = *reinterpret_cast<const uint32_t*>(&h0);
-          const uint32_t v1 = *reinterpret_cast<const uint32_t*>(&h1);
-          xp[j * 32 + lane] = uint16_t(v0);
-          xp[(j + 1) * 32 + lane] = uint16_t(v0 >> 16);
-          xp[(j + 2) * 32 + lane] = uint16_t(v1);
-          xp[(j + 3) * 32 + lane] = uint16_t(v1 >> 16);
+      // the previous tile's bulk store has read the output tile: it may be rewritten
+      if (stored > 0) {
+        if (leader) {
+          bulk_wait_read_all();
+          mbar_arrive(ofree);
         }
-        __syncwarp();
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int t = j0 + c16 + jr + 8 * hr;
-          const uint4 piece = *reinterpret_cast<const uint4*>(xp + (jr + 8 * hr) * 32 + cc);
-          if (t < rows) *reinterpret_cast<uint4*>(outb + size_t(tok0 + t) * p.N) = piece;
-        }
-        __syncwarp();  // the block is rewritten by the next 16 tokens
+        if (!mbar_wait(ofree, uint32_t(stored - 1) & 1u, wc)) { ok = false; break; }
       }
+      if (j0 < rows) {
+#pragma unroll
+        for (int i = 0; i < CW / 32; ++i) sxw[32 * i + lane] = sxr[i];
+        __syncwarp();
+        uint16_t* orow = reinterpret_cast<uint16_t*>(out_tile) + j0 * kBM + ch;
+#pragma unroll
+        for (int j = 0; j < CW; j += 4) {
+          const float4 sv = *reinterpret_cast<const float4*>(sxw + j);
+          orow[(j + 0) * kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(accf[j + 0], sv.x)));
+          orow[(j + 1) * kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(accf[j + 1], sv.y)));
+          orow[(j + 2) * kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(accf[j + 2], sv.z)));
+          orow[(j + 3) * kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(accf[j + 3], sv.w)));
+        }
+        __syncwarp();  // sxw is rewritten by the next tile
+      }
+      fence_proxy_async_smem();  // the tile's generic-proxy writes become visible to the TMA store
+      mbar_arrive(ostaged);
+      if (leader) {
+        if (!mbar_wait(ostaged, uint32_t(stored) & 1u, wc)) { ok = false; break; }
+        tma_store_2d(&p.tmY, out_tile, cb * kBM * 2, tok0);  // rows past M are not written
+        bulk_commit_group();
+      }
+      ++stored;
     }
+    if (leader) bulk_wait_all();  // the CTA's shared memory outlives every bulk store
   }
 
   tc_fence_before();

@@ -765,6 +765,7 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
   if (w_format == W8A8_W_INT4_PER_GROUP) {
     W4A8Params q{};
     if (!make_plain_map(&q.tmW, wq, uint64_t(K / 2), uint64_t(N), 64, 128) ||
+        !make_plain_map(&q.tmY, y, uint64_t(N) * 2, uint64_t(M), 256, 128) ||
         !make_kmajor_map(&q.tmX, xq, false, K, Mp, kBBoxRows) || !make_kmajor_map(&q.tmX2, xq, false, K, Mp, 128))
       return W8A8_ERR_UNSUPPORTED;
     q.num_kb = int(K / 128);
@@ -772,8 +773,8 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
     q.M = int(M);
     q.N = int(N);
     q.sw = sw;
+    q.sw_vec = (K / 128) % 4 == 0 && aligned16(sw);
     q.sx = sx;
-    q.y = y;
     q.timeout_ns = wait_timeout_ns();
     using Cfg = W4Cfg<128, 4, 8>;
     auto kern = w4a8_gemm_kernel<128, 4, 8>;
