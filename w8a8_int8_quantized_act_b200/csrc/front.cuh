@@ -2,16 +2,18 @@
 // case): router logits, softmax / top-k, the stable grouping of the T*k assignments by expert
 // and the per-token activation quantisation into the sorted rows, in one cooperative launch
 // instead of three latency-bound ones:
-//   phase 1  logits [T, E] in fp32: the short-batch router's work items, two per CTA at a time;
+//   phase 1  logits [T, E] in fp32: the short-batch router's work items, two per CTA at a time
+//            (each half of the CTA stages its item's token rows in shared memory once);
 //   barrier
-//   phase 2  top-k of token t by one warp (global warp index t); ids and weights to the workspace;
+//   phase 2  top-k of token t by one warp (warp t / G of CTA t % G); ids and weights to the
+//            workspace;
 //   barrier
 //   phase 3  every CTA reads the T*k expert ids and builds the counting sort by expert (stable
 //            by token) in shared memory; CTA 0 stores offsets, perm and the expert histogram;
 //   phase 4  token t is quantised by CTA t (all its warps; the row maximum through shared
 //            memory) and its codes written to its k sorted rows.
 // Both barriers are bounded: a CTA that waits too long raises the error word and returns. The
-// arithmetic is that of router_logits_item, warp_topk_token and the symmetric quantiser (a
+// arithmetic is that of the short-batch router, warp_topk_token and the symmetric quantiser (a
 // maximum does not depend on the order it is taken in), so the results are those of the
 // separate kernels bit for bit.
 #pragma once
@@ -21,6 +23,7 @@
 namespace w8a8 {
 
 constexpr int kFrontMaxT = 128;
+constexpr int kFrontMaxH = 2048;  // token row length the front end takes (its phase-1 staging)
 constexpr int kFrontThreads = 512;
 constexpr int kFrontWarps = kFrontThreads / 32;
 
@@ -63,6 +66,7 @@ __global__ void __launch_bounds__(kFrontThreads) front_small_kernel(
   __shared__ uint32_t mask[256 * 4];            // per expert: which tokens chose it
   __shared__ float red[kFrontWarps];
   __shared__ int ok_smem;
+  __shared__ __align__(16) uint16_t xrows[2][kSmallRouterTokens * kFrontMaxH];  // phase 1, per half
 
   pdl_wait();
   pdl_launch_dependents();
@@ -70,16 +74,25 @@ __global__ void __launch_bounds__(kFrontThreads) front_small_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x;
 
-  // phase 1: logits; the two halves of the CTA take one work item each
+  // phase 1: logits; the two halves of the CTA take one work item each (a half syncs on its
+  // own named barrier, 1 or 2: the halves may run different numbers of items)
   const int neg = (E + 7) / 8, ntg = (T + kSmallRouterTokens - 1) / kSmallRouterTokens;
-  for (int item = 2 * blockIdx.x + (warp >> 3); item < neg * ntg; item += 2 * G) {
+  const int hf = warp >> 3;
+  for (int item = 2 * blockIdx.x + hf; item < neg * ntg; item += 2 * G) {
     const int tg = item / neg;
-    router_logits_item<RU>(x, wg, T, H, E, logits, item - tg * neg, tg, warp & 7);
+    uint4 wv[RU];
+    router_item_weights<RU>(wg, H, E, item - tg * neg, warp & 7, wv);
+    stage_router_rows(x, T, H, tg, threadIdx.x & 255, xrows[hf]);
+    asm volatile("bar.sync %0, 256;" ::"r"(1 + hf) : "memory");
+    router_logits_item_xs<RU>(xrows[hf], wv, T, H, E, logits, item - tg * neg, tg, warp & 7);
+    asm volatile("bar.sync %0, 256;" ::"r"(1 + hf) : "memory");  // the rows are rewritten by the next item
   }
   if (!grid_barrier(sync_count, unsigned(G), 1u, deadline, &ok_smem)) return;
 
-  // phase 2: top-k, one warp per token (logits written by other CTAs: read through L2)
-  for (int t = blockIdx.x * kFrontWarps + warp; t < T; t += G * kFrontWarps) {
+  // phase 2: top-k, one warp per token, spread over the CTAs first (token t on warp t / G of
+  // CTA t % G), so that no SM sub-partition interleaves several tokens' selections (logits
+  // written by other CTAs: read through L2)
+  for (int t = warp * G + blockIdx.x; t < T; t += G * kFrontWarps) {
     const float* row = logits + size_t(t) * E;
     warp_topk_token<PER>([&](int e) { return __ldcg(row + e); }, E, k, renorm != 0, bias, ids + size_t(t) * k,
                          w + size_t(t) * k, nullptr);

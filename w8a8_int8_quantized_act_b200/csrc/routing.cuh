@@ -239,13 +239,91 @@ __device__ __forceinline__ void router_logits_item(const uint16_t* __restrict__ 
   }
 }
 
+// Same work item in two steps, with the item's kSmallRouterTokens token rows in shared memory
+// (xs: [kSmallRouterTokens][H] bf16, rows past T zero), so that each row is read from global
+// memory once per item instead of once per warp: router_item_weights loads the warp's expert
+// row (issue it before staging the token rows, so that both loads are in flight together),
+// router_logits_item_xs computes and stores the logits.
+template <int RU>
+__device__ __forceinline__ void router_item_weights(const uint16_t* __restrict__ wg, int H, int E, int eg, int w8,
+                                                    uint4 (&wv)[RU]) {
+  const int lane = threadIdx.x & 31;
+  const int e = eg * 8 + w8;
+#pragma unroll
+  for (int u = 0; u < RU; ++u) {
+    const int i = lane * 8 + u * 256;
+    wv[u] = (i < H && e < E) ? __ldg(reinterpret_cast<const uint4*>(wg + size_t(e) * H + i)) : make_uint4(0, 0, 0, 0);
+  }
+}
+template <int RU>
+__device__ __forceinline__ void router_logits_item_xs(const uint16_t* __restrict__ xs, const uint4 (&wv)[RU], int T,
+                                                      int H, int E, float* __restrict__ logits, int eg, int tg,
+                                                      int w8) {
+  constexpr int TT = kSmallRouterTokens;
+  const int lane = threadIdx.x & 31;
+  const int e = eg * 8 + w8;
+  if (e >= E) return;
+  const int t0 = tg * TT;
+  float acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    float part[RU];
+#pragma unroll
+    for (int u = 0; u < RU; ++u) {
+      const int i = lane * 8 + u * 256;
+      const uint4 xv = (i < H) ? *reinterpret_cast<const uint4*>(xs + t * H + i) : make_uint4(0, 0, 0, 0);
+      const uint32_t a[4] = {xv.x, xv.y, xv.z, xv.w};
+      const uint32_t b[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+      float s2 = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s2 = fmaf(bf16_lo(a[j]), bf16_lo(b[j]), s2);
+        s2 = fmaf(bf16_hi(a[j]), bf16_hi(b[j]), s2);
+      }
+      part[u] = s2;
+    }
+    float sum = 0.0f;
+#pragma unroll
+    for (int u = 0; u < RU; ++u) sum += part[u];
+    acc[t] = sum;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+  if (lane < TT && t0 + lane < T) {
+    float v = acc[0];
+#pragma unroll
+    for (int t = 1; t < TT; ++t) v = (lane == t) ? acc[t] : v;
+    logits[size_t(t0 + lane) * E + e] = v;
+  }
+}
+
+// The item's token rows into shared memory by the 256 threads of one item (thread index it),
+// zero rows past T.
+__device__ __forceinline__ void stage_router_rows(const uint16_t* __restrict__ x, int T, int H, int tg, int it,
+                                                  uint16_t* xs) {
+  const int t0 = tg * kSmallRouterTokens;
+  const int vec_per_row = H / 8;
+  for (int v = it; v < kSmallRouterTokens * vec_per_row; v += 256) {
+    const int t = v / vec_per_row, i = (v - t * vec_per_row) * 8;
+    *reinterpret_cast<uint4*>(xs + t * H + i) =
+        (t0 + t < T) ? __ldg(reinterpret_cast<const uint4*>(x + size_t(t0 + t) * H + i)) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 template <int RU>
 __global__ void __launch_bounds__(256) router_logits_small_kernel(const uint16_t* __restrict__ x,
                                                                   const uint16_t* __restrict__ wg, int T, int H,
                                                                   int E, float* __restrict__ logits) {
+  extern __shared__ __align__(16) uint16_t xs_dyn[];  // [kSmallRouterTokens][H]
   pdl_wait();
   pdl_launch_dependents();
-  router_logits_item<RU>(x, wg, T, H, E, logits, blockIdx.x, blockIdx.y, threadIdx.x >> 5);
+  uint4 wv[RU];
+  router_item_weights<RU>(wg, H, E, blockIdx.x, threadIdx.x >> 5, wv);
+  stage_router_rows(x, T, H, blockIdx.y, threadIdx.x, xs_dyn);
+  __syncthreads();
+  router_logits_item_xs<RU>(xs_dyn, wv, T, H, E, logits, blockIdx.x, blockIdx.y, threadIdx.x >> 5);
 }
 
 // Top-k over precomputed logits [T, E]: one warp per token. counts has one row of E per

@@ -237,13 +237,14 @@ int run_router_small(const uint16_t* x, const uint16_t* wg, const float* bias, i
   const dim3 grid1(unsigned((E + 7) / 8), unsigned((T + kSmallRouterTokens - 1) / kSmallRouterTokens));
   const dim3 blk(256);
   const int Ti = int(T), Hi = int(H), Ei = int(E);
+  const size_t xs_bytes = sizeof(uint16_t) * size_t(kSmallRouterTokens) * size_t(H);  // <= 32 KB (H <= 4096)
   int rc;
   switch (row_units(Hi)) {
-    case 1: rc = launch_pdl(router_logits_small_kernel<1>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
-    case 2: rc = launch_pdl(router_logits_small_kernel<2>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
-    case 4: rc = launch_pdl(router_logits_small_kernel<4>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
-    case 8: rc = launch_pdl(router_logits_small_kernel<8>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
-    case 16: rc = launch_pdl(router_logits_small_kernel<16>, grid1, blk, 0, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 1: rc = launch_pdl(router_logits_small_kernel<1>, grid1, blk, xs_bytes, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 2: rc = launch_pdl(router_logits_small_kernel<2>, grid1, blk, xs_bytes, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 4: rc = launch_pdl(router_logits_small_kernel<4>, grid1, blk, xs_bytes, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 8: rc = launch_pdl(router_logits_small_kernel<8>, grid1, blk, xs_bytes, stream, x, wg, Ti, Hi, Ei, logits); break;
+    case 16: rc = launch_pdl(router_logits_small_kernel<16>, grid1, blk, xs_bytes, stream, x, wg, Ti, Hi, Ei, logits); break;
     default: return W8A8_ERR_UNSUPPORTED;
   }
   if (rc != W8A8_OK) return rc;
@@ -326,9 +327,8 @@ int launch_group_quant(dim3 grid, size_t smem, cudaStream_t s, const uint16_t* x
 }
 
 // The fused short-batch front end (front.cuh): one cooperative launch of up to one CTA per SM
-// (all resident at once, which its grid barriers need). Rows of up to 2048 values keep the
-// router's per-lane slices in registers at 512 threads per CTA.
-constexpr int64_t kFrontMaxH = 2048;
+// (all resident at once, which its grid barriers need), for rows of at most kFrontMaxH values
+// (the router's token rows are staged in shared memory, the weight slices kept in registers).
 template <int RU, int PER>
 int launch_front_t(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int H, int E, int k, int renorm,
                    float* logits, unsigned* sync, int* ids, float* w, int* tile_counts, int* offsets, int* perm,
