@@ -69,7 +69,8 @@ struct GemmParams {
   int renorm;
   float* topk_w;
   int* tile_counts;            // expert histogram rows (nullptr: none); zeroed before the launch
-  int tile_count_stride;       // elements between the rows of consecutive token tiles (0: one row)
+  int tile_count_stride;       // elements between the rows of consecutive 128-token chunks (0: one row)
+  int router_rows;             // router: tokens per tile (64 or 128; the A map's box height)
 };
 
 template <int NA, int NB, int EPI>
@@ -121,11 +122,13 @@ template <int EPI, int NB>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* mt_prefix, const int* goff, int tile) {
   Tile c;
   if constexpr (EPI == kEpiRouter) {
+    // router_rows tokens per tile (the MMA keeps M = 128: lanes past them compute values that
+    // nobody reads); the histogram row is the tile's 128-token chunk
     c.g = 0;
     c.cb = 0;
-    c.tt = tile;
-    c.tok0 = tile * kBM;
-    c.rows = min(kBM, p.M - c.tok0);
+    c.tok0 = tile * p.router_rows;
+    c.tt = c.tok0 / kBM;
+    c.rows = min(p.router_rows, p.M - c.tok0);
     c.a_row = c.tok0;
     c.b_row = 0;
     c.nb = p.nb_fixed;
@@ -321,8 +324,9 @@ __device__ __forceinline__ void epilogue_router(const GemmParams& p, const Tile&
   const int E = p.n_valid;
   const int k = p.topk;
   const float* __restrict__ bias = p.bias;
-  // 1. TMEM -> shared memory, transposed (with 16 experts the lower warp copies them all)
-  if (NB >= 32 || half == 0) {
+  // 1. TMEM -> shared memory, transposed (with 16 experts the lower warp copies them all; lane
+  //    quarters past the tile's tokens are skipped)
+  if ((NB >= 32 || half == 0) && lane_row - int(threadIdx.x & 31) < c.rows) {
     const int c0 = NB >= 32 ? half * SPAN : 0;
 #pragma unroll
     for (int c16 = 0; c16 < SPAN; c16 += 16) {
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     *abort_flag = 0;
     mt_prefix[0] = 0;
     if (!(EPI != kEpiRouter && p.group_offsets != nullptr))
-      mt_prefix[1] = (EPI == kEpiRouter) ? (p.M + kBM - 1) / kBM : (p.M + NB - 1) / NB;
+      mt_prefix[1] = (EPI == kEpiRouter) ? (p.M + p.router_rows - 1) / p.router_rows : (p.M + NB - 1) / NB;
     tma_prefetch_map(&p.tmA);
     tma_prefetch_map(&p.tmB);
     tma_prefetch_map(&p.tmB2);
@@ -435,7 +439,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
-      const uint32_t bytes = uint32_t(NA * Cfg::kABytes + c.nb * kKBlockBytes);
+      const uint32_t a_bytes = (EPI == kEpiRouter) ? uint32_t(p.router_rows * kKBlockBytes) : uint32_t(Cfg::kABytes);
+      const uint32_t bytes = uint32_t(NA * a_bytes + c.nb * kKBlockBytes);
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
         if (elect_one()) {

@@ -263,8 +263,11 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
                int renorm, int* ids, float* w, int* counts, int64_t count_stride, float* logits,
                cudaStream_t stream) {
   const int nb = router_bn(E);
+  // 64 tokens per tile: the top-k epilogue, the larger part of the kernel, spreads over twice
+  // as many CTAs (64 -> 128 of them for 8192 tokens)
+  constexpr int kRouterRows = 64;
   GemmParams p{};
-  if (!make_kmajor_map(&p.tmA, x, true, H, T, 128) || !make_kmajor_map(&p.tmB, wg, true, H, E, kBBoxRows) ||
+  if (!make_kmajor_map(&p.tmA, x, true, H, T, kRouterRows) || !make_kmajor_map(&p.tmB, wg, true, H, E, kBBoxRows) ||
       !make_kmajor_map(&p.tmB2, wg, true, H, E, uint32_t(nb)))
     return W8A8_ERR_UNSUPPORTED;
   const int64_t C = (T + kChunk - 1) / kChunk;
@@ -289,7 +292,8 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
   p.topk_w = w;
   p.tile_counts = counts;
   p.tile_count_stride = int(count_stride);
-  const int tiles = int(C);
+  p.router_rows = kRouterRows;
+  const int tiles = int((T + kRouterRows - 1) / kRouterRows);
   switch (nb) {
     case 16: return launch_gemm<1, 16, kEpiRouter, kKindBF16>(p, tiles, stream);
     case 32: return launch_gemm<1, 32, kEpiRouter, kKindBF16>(p, tiles, stream);
