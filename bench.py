@@ -423,8 +423,8 @@ def run_linear(args, wl, rank, dist):
 # kernels, the fused short-batch front end and the dense W4A8 GEMM); reported only while those
 # sources are unchanged (null otherwise, since the counters no longer describe the kernel).
 GATE_UP_TRAFFIC = {
-    "qwen3-30b-a3b-decode": (391_960_576 + 5_193_216, "32fc4aef4460e32870654577b19b540dabb6da25"),
-    "qwen3-30b-a3b-prefill": (541_549_568 + 90_793_984, "32fc4aef4460e32870654577b19b540dabb6da25"),
+    "qwen3-30b-a3b-decode": (391_960_576 + 5_193_216, "3f41d6b0e52cfb0ce400f8b802937efd3d00cde6"),
+    "qwen3-30b-a3b-prefill": (541_549_568 + 90_793_984, "3f41d6b0e52cfb0ce400f8b802937efd3d00cde6"),
 }
 
 

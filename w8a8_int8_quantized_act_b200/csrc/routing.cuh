@@ -177,73 +177,15 @@ __device__ __forceinline__ void warp_topk_tokens(Logit logit, int nt, int E, int
 }
 
 // Router logits on the CUDA cores for short batches: logits[t, e] = sum_h x[t, h] * wg[e, h] in
-// fp32 (bf16 inputs). Block = 8 warps; warp w takes expert blockIdx.x * 8 + w and the
-// kSmallRouterTokens tokens of blockIdx.y together (all their loads in flight at once, one
-// accumulator per token and vector slot); each lane holds its 1/32 of the expert's row
-// (H <= 256 * RU) in registers.
+// fp32 (bf16 inputs). A work item is 8 experts x kSmallRouterTokens tokens for 8 warps: warp w8
+// takes expert eg * 8 + w8 and tokens tg * kSmallRouterTokens .. + kSmallRouterTokens - 1, with
+// its 1/32 of the expert's row (H <= 256 * RU) in registers and one accumulator per token and
+// vector slot. The item's token rows sit in shared memory (xs: [kSmallRouterTokens][H] bf16, rows
+// past T zero), read from global memory once per item instead of once per warp. Two steps:
+// router_item_weights loads the warp's expert row (issue it before staging the token rows, so
+// that both loads are in flight together); router_logits_item_xs computes and stores the logits.
 constexpr int kSmallRouterTokens = 4;
 
-// One work item of the short-batch router: the calling warp (w8 = its index among the item's 8
-// warps) computes the logits of expert eg * 8 + w8 for tokens tg * kSmallRouterTokens ..
-// + kSmallRouterTokens - 1.
-template <int RU>
-__device__ __forceinline__ void router_logits_item(const uint16_t* __restrict__ x, const uint16_t* __restrict__ wg,
-                                                   int T, int H, int E, float* __restrict__ logits, int eg, int tg,
-                                                   int w8) {
-  constexpr int TT = kSmallRouterTokens;
-  const int lane = threadIdx.x & 31;
-  const int e = eg * 8 + w8;
-  if (e >= E) return;
-  const int t0 = tg * TT;
-  uint4 wv[RU];
-  uint4 xv[TT][RU];
-#pragma unroll
-  for (int u = 0; u < RU; ++u) {
-    const int i = lane * 8 + u * 256;
-    wv[u] = (i < H) ? __ldg(reinterpret_cast<const uint4*>(wg + size_t(e) * H + i)) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int t = 0; t < TT; ++t)
-      xv[t][u] = (i < H && t0 + t < T) ? __ldg(reinterpret_cast<const uint4*>(x + size_t(t0 + t) * H + i))
-                                       : make_uint4(0, 0, 0, 0);
-  }
-  float acc[TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    float part[RU];
-#pragma unroll
-    for (int u = 0; u < RU; ++u) {
-      const uint32_t a[4] = {xv[t][u].x, xv[t][u].y, xv[t][u].z, xv[t][u].w};
-      const uint32_t b[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
-      float s2 = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        s2 = fmaf(bf16_lo(a[j]), bf16_lo(b[j]), s2);
-        s2 = fmaf(bf16_hi(a[j]), bf16_hi(b[j]), s2);
-      }
-      part[u] = s2;
-    }
-    float sum = 0.0f;
-#pragma unroll
-    for (int u = 0; u < RU; ++u) sum += part[u];
-    acc[t] = sum;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-  if (lane < TT && t0 + lane < T) {
-    float v = acc[0];
-#pragma unroll
-    for (int t = 1; t < TT; ++t) v = (lane == t) ? acc[t] : v;
-    logits[size_t(t0 + lane) * E + e] = v;
-  }
-}
-
-// Same work item in two steps, with the item's kSmallRouterTokens token rows in shared memory
-// (xs: [kSmallRouterTokens][H] bf16, rows past T zero), so that each row is read from global
-// memory once per item instead of once per warp: router_item_weights loads the warp's expert
-// row (issue it before staging the token rows, so that both loads are in flight together),
-// router_logits_item_xs computes and stores the logits.
 template <int RU>
 __device__ __forceinline__ void router_item_weights(const uint16_t* __restrict__ wg, int H, int E, int eg, int w8,
                                                     uint4 (&wv)[RU]) {
