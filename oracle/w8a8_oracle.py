@@ -309,15 +309,24 @@ def gated_activation(acc_gu: np.ndarray, s_row: np.ndarray, s_gu: np.ndarray) ->
     return f32_to_bf16(silu(g) * u)
 
 
-def combine(o_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
-    """y[t] = bf16(sum_j w[t, j] * o[t, j]): fp32 fused multiply-adds in slot order from 0."""
+def combine_acc(o_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """The fp32 accumulator of the weighted combine: acc = 0, then for j = 0 .. k-1 in slot
+    order acc = fma(w[t, j], o[t, j], acc), one rounding per slot."""
     o = bf16_to_f32(o_bits)
     T, k, H = o.shape
     acc = np.zeros((T, H), np.float32)
     w = np.asarray(w, np.float32)
     for j in range(k):
         acc = fma32(np.broadcast_to(w[:, j:j + 1], (T, H)), o[:, j, :], acc)
-    return f32_to_bf16(acc)
+    return acc
+
+
+def combine(o_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """y[t] = bf16(sum_j w[t, j] * o[t, j]): the fma chain of ``combine_acc``, rounded to bf16.
+
+    Section 三 3.1 of the Qwen3-30B-A3B-2507 w8a8 page: the selected experts' outputs are
+    weighted by the router and summed."""
+    return f32_to_bf16(combine_acc(o_bits, w))
 
 
 # --------------------------------------------------------------------------------------

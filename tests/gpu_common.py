@@ -81,10 +81,38 @@ def check_grouping(ids: np.ndarray, perm: np.ndarray, offsets: np.ndarray, E: in
     np.testing.assert_array_equal(perm, ref_perm)
 
 
+def check_topk_valid(ids: np.ndarray, w: np.ndarray, r, k: int, renorm: bool, tol: float = 1e-4):
+    """Every token's routing is a valid top-k of the oracle's probabilities, near ties included.
+
+    Several expert sets are correct where the k-th and (k+1)-th probabilities lie within `tol`
+    of each other, so for every token this checks what is unique: the k ids are distinct and in
+    range; each chosen expert has p >= p_(k) - tol and each rejected one p <= p_(k+1) + tol; the
+    weights equal the oracle's probabilities of the chosen experts (renormalised over them when
+    `renorm`), rtol 2e-4 / atol 2e-6; and the slots are in descending order of weight."""
+    T, E = r.probs.shape
+    assert ids.shape == (T, k) and w.shape == (T, k)
+    assert np.all((ids >= 0) & (ids < E))
+    srt = -np.sort(-r.probs, axis=1)
+    pk = srt[:, k - 1]
+    pk1 = srt[:, k] if k < E else np.full(T, -np.inf)
+    for t in range(T):
+        chosen = ids[t]
+        assert len(set(chosen.tolist())) == k, (t, chosen)
+        p = r.probs[t]
+        assert np.all(p[chosen] >= pk[t] - tol), (t, chosen)
+        rejected = np.setdiff1d(np.arange(E), chosen)
+        if rejected.size:
+            assert p[rejected].max() <= pk1[t] + tol, (t, chosen)
+        ref = p[chosen] / p[chosen].sum() if renorm else p[chosen]
+        np.testing.assert_allclose(w[t], ref, rtol=2e-4, atol=2e-6, err_msg=f"token {t}")
+        assert np.all(np.diff(w[t]) <= 2e-6), (t, w[t])
+
+
 def check_routing(run: MoERun, ids: np.ndarray, w: np.ndarray, tokens: np.ndarray | None = None,
                   gap: float = 1e-4):
-    """Expert sets equal wherever the k-th/(k+1)-th probability gap exceeds `gap`; weights of
-    identical sets within fp32 rounding of the oracle's float64 softmax."""
+    """Expert sets equal wherever the k-th/(k+1)-th probability gap exceeds `gap`; every token,
+    near ties included, a valid top-k with the oracle's weights (check_topk_valid). Returns the
+    mask of tokens whose routing is unambiguous."""
     wl = run.wl
     x = run.inp.x if tokens is None else run.inp.x[tokens]
     r = O.route(x, run.inp.wg, run.inp.bias, wl.k, wl.renorm)
@@ -93,7 +121,7 @@ def check_routing(run: MoERun, ids: np.ndarray, w: np.ndarray, tokens: np.ndarra
     np.testing.assert_array_equal(np.sort(gi[clear], 1), np.sort(r.ids[clear], 1))
     same = np.all(gi == r.ids, axis=1)
     assert same.mean() > 0.9
-    np.testing.assert_allclose(gw[same], r.weights[same], rtol=2e-4, atol=2e-6)
+    check_topk_valid(gi, gw, r, wl.k, wl.renorm, gap)
     return clear
 
 
