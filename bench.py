@@ -2,17 +2,24 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
 
-A step is one whole forward (router, grouping + quantisation, gate_up GEMM, requantisation,
-down GEMM, combine) over one batch of synthetic tokens. Default workload: the Qwen3-30B-A3B
-shaped decode layer (64 tokens, hidden 2048, 128 experts, top-8, intermediate 768).
+A step is one whole forward (router, grouping + quantisation, gate_up GEMM with the fused
+dequant and SiLU * up, requantisation of h, down GEMM, combine) over one batch of synthetic
+tokens. The
+headline workload is the largest single-GPU layer: the Qwen3-235B-A22B shaped MoE layer (4096
+tokens, hidden 4096, 128 experts, top-8, intermediate 1536). With no --workload the same line
+also carries the other workloads as sub-results (the Qwen3-30B-A3B decode, prefill and skewed
+prefill layers, the dense W4A8 linear and the dense W8A8 linears), each with its own timing,
+roofline, end-to-end figure and CPU-oracle baseline. --workload NAME times one workload alone.
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and a device
 synchronisation on both sides, timed with CUDA events on the launching stream; the maximum
-over ranks is reported. Each step streams the touched experts' weights (about 597 MB for the
-decode layer), more than the 126 MB L2, so no step is served from L2 by the previous one.
+over ranks is reported. Every step streams more than the 126 MB L2 (the touched experts'
+weights of the MoE layers, 32 rotating weight copies for the dense linears), so no step is
+served from L2 by the previous one.
 
 Multi-GPU (torchrun): replicas. Every rank holds the full layer and runs its own batch of the
 same size; nothing is exchanged on the data path (tokens are independent), so scaling is weak.
+Only the headline workload is timed with more than one rank.
 
 --impl reference times the CPU oracle on this host on a bounded sample of the same workload.
 """
@@ -35,14 +42,23 @@ if ROOT not in sys.path:
 METRIC = "W8A8 MoE layer tokens/s on 1 B200; INT8 TOPS and HBM GB/s vs peak"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet dense INT8 tensor throughput (the 9 POPS figure NVIDIA quotes is with 2:4
+# sparsity); fractions are also given against 2 x the measured bf16 GEMM rate (the nominal
+# int8:bf16 ratio applied to this machine's measured peak)
+INT8_DATASHEET_TOPS = 4500.0
+
+HEADLINE = "qwen3-235b-a22b"
+SUB_MOE = ("qwen3-30b-a3b-decode", "qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed")
+SUB_LINEAR = ("qwen3-1.7b-mlp-w4a8", "qwen3-1.7b-mlp-w8a8", "qwen3-30b-a3b-q-proj-w8a8",
+              "qwen3-30b-a3b-k-proj-w8a8", "qwen3-30b-a3b-o-proj-w8a8")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="qwen3-30b-a3b-decode")
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None, help="time one workload alone (default: headline + sub-results)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0)
@@ -117,7 +133,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- CPU oracle leg
 def cpu_oracle_rate(wl, n_tokens: int, min_seconds: float = 10.0, max_seconds: float = 30.0):
-    """Times the oracle (as it stands) on `n_tokens` tokens of the workload; tokens/s."""
+    """Times the oracle (as it stands) on `n_tokens` tokens of the MoE workload; tokens/s."""
     from oracle import w8a8_oracle as O
     from w8a8_int8_quantized_act_b200 import synth
 
@@ -134,6 +150,30 @@ def cpu_oracle_rate(wl, n_tokens: int, min_seconds: float = 10.0, max_seconds: f
     reps = 0
     while True:
         O.moe_forward(x, wg, bias, wgu_q, s_gu, wd_q, s_d, wl.k, wl.renorm)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or (reps >= 1 and el * (reps + 1) / reps > max_seconds):
+            break
+    return n_tokens * reps / el, reps, el
+
+
+def cpu_oracle_linear_rate(wl, n_tokens: int, min_seconds: float = 5.0, max_seconds: float = 15.0):
+    """Times the oracle's dense linear (as it stands) on `n_tokens` rows of the workload; tokens/s."""
+    from oracle import w8a8_oracle as O
+    from w8a8_int8_quantized_act_b200 import synth
+
+    x = synth.activations(wl.M, wl.K, wl.n_outlier, wl.seed)[:n_tokens]
+    w = synth.dense_weight(wl.N, wl.K, wl.seed)
+    if wl.fmt == "int4":
+        packed, sw = O.quantize_weight_int4_per_group(w, wl.group)
+        fwd = lambda: O.linear_w4a8(x, packed, sw, wl.group)  # noqa: E731
+    else:
+        wq, sw = O.quantize_weight_per_channel(w)
+        fwd = lambda: O.linear_w8a8(x, wq, sw)  # noqa: E731
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        fwd()
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or (reps >= 1 and el * (reps + 1) / reps > max_seconds):
@@ -159,16 +199,33 @@ def default_sample_tokens(wl) -> int:
 
 # ---------------------------------------------------------------------------- algorithmic work
 def algorithmic(wl, counts: np.ndarray):
-    """Algorithmic ops and bytes of one layer forward, and bytes of the gate_up launch."""
+    """Algorithmic ops and bytes of one layer forward, and of its gate_up and down launches.
+
+    Bytes are what the method must move: the touched experts' int8 weights and fp32 scales, x
+    in and y out, the bf16 router weight. The implementation's own intermediates (token codes,
+    h, o) are not counted."""
     touched = int((counts > 0).sum())
     A = wl.T * wl.k
     ops = 2 * A * (2 * wl.I * wl.H + wl.H * wl.I) + 2 * wl.T * wl.H * wl.E
     w_bytes = touched * (3 * wl.I * wl.H + 4 * (2 * wl.I + wl.H))
     io_bytes = 2 * wl.T * wl.H * 2 + 2 * wl.E * wl.H
-    gate_up_bytes = touched * (2 * wl.I * wl.H + 4 * 2 * wl.I) + A * wl.H + A * wl.I * 2
-    down_bytes = touched * (wl.H * wl.I + 4 * wl.H) + A * wl.I + A * wl.H * 2
+    gate_up_bytes = touched * (2 * wl.I * wl.H + 4 * 2 * wl.I)
+    down_bytes = touched * (wl.H * wl.I + 4 * wl.H)
     return dict(ops=ops, bytes=w_bytes + io_bytes, touched=touched, gate_up_bytes=gate_up_bytes,
                 down_bytes=down_bytes, gate_up_ops=2 * A * 2 * wl.I * wl.H, down_ops=2 * A * wl.H * wl.I)
+
+
+def moe_launches(wl) -> int:
+    """Kernels of this library one forward launches (memsets not counted): the fused front end
+    for T <= 128 and H <= 2048, else the router (two kernels for T <= 512) and the grouping;
+    then gate_up, the requantisation of h, down and the combine."""
+    if wl.T <= 128 and wl.H <= 2048:
+        front = 1
+    elif wl.T <= 512:
+        front = 3
+    else:
+        front = 2
+    return front + 4
 
 
 # ---------------------------------------------------------------------------- native arm
@@ -192,27 +249,37 @@ def whole_job_rate(world: int, units_per_rank_step: int, steps: int, ms: float) 
     return world * units_per_rank_step * steps / (ms / 1e3)
 
 
-def run_native(args, wl, rank, world, dist):
+class MoELayer:
+    """One layer's device weights (quantised by the library), shared by workloads of one shape."""
+
+    def __init__(self, wl, dev):
+        import torch
+
+        from w8a8_int8_quantized_act_b200 import binding as B
+        from w8a8_int8_quantized_act_b200 import synth
+
+        self.key = (wl.H, wl.E, wl.I, wl.seed)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
+        self.wg = bf(synth.router_weight(wl.E, wl.H, wl.seed))
+        self.wgu_q, self.s_gu = B.w8a8_quantize_weight_per_channel(bf(synth.expert_gate_up(wl.E, wl.I, wl.H,
+                                                                                            wl.seed)))
+        self.wd_q, self.s_d = B.w8a8_quantize_weight_per_channel(bf(synth.expert_down(wl.E, wl.H, wl.I, wl.seed)))
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def run_moe(args, wl, layer, rank, dist, dev):
     import torch
 
     from w8a8_int8_quantized_act_b200 import binding as B
     from w8a8_int8_quantized_act_b200 import synth
 
-    local = int(os.environ.get("LOCAL_RANK", 0))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    B.lib()
+    local = dev.index
     # every rank: its own batch of wl.T tokens (seeded by rank), the full layer's weights
     x_host = synth.activations(wl.T, wl.H, wl.n_outlier, rank_seed(wl.seed, rank))
-    inp = synth.moe_inputs(wl)
-    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
-    x = bf(x_host)
-    wg = bf(inp.wg)
-    bias = torch.from_numpy(inp.bias).to(dev) if inp.bias is not None else None
-    wgu_q, s_gu = B.w8a8_quantize_weight_per_channel(bf(inp.wgu))
-    wd_q, s_d = B.w8a8_quantize_weight_per_channel(bf(inp.wd))
-    del inp
-    torch.cuda.empty_cache()
+    x = torch.from_numpy(x_host).view(torch.bfloat16).to(dev)
+    bias = torch.from_numpy(synth.router_bias(wl.E, wl.seed)).to(dev) if wl.skewed else None
+    wg, wgu_q, s_gu, wd_q, s_d = layer.wg, layer.wgu_q, layer.s_gu, layer.wd_q, layer.s_d
     ws = torch.empty(B.w8a8_moe_workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I), dtype=torch.uint8, device=dev)
     y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -225,7 +292,7 @@ def run_native(args, wl, rank, world, dist):
     B.w8a8_check_status()
     counts = np.diff(B.moe_intermediates(ws, wl.T, wl.H, wl.E, wl.k, wl.I)["offsets"].cpu().numpy())
 
-    # ---- timed region 1 (the headline): K replays of the forward captured in a CUDA graph
+    # ---- timed region (the figure reported): K replays of the forward captured in a CUDA graph
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step()
@@ -238,7 +305,7 @@ def run_native(args, wl, rank, world, dist):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start.record(stream)
-        for i in range(args.steps):
+        for _ in range(args.steps):
             graph.replay()
         stop.record(stream)
         torch.cuda.synchronize()
@@ -247,7 +314,7 @@ def run_native(args, wl, rank, world, dist):
     B.w8a8_check_status()
     ms = start.elapsed_time(stop)
 
-    # ---- timed region 2: K direct calls recording events at the stage boundaries, for the
+    # ---- second pass: K direct calls recording events at the stage boundaries, for the
     # per-kernel durations (the dominant kernel's roofline figure comes from here)
     nst = 7
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
@@ -282,6 +349,7 @@ def run_native(args, wl, rank, world, dist):
     B.w8a8_check_status()
 
     ms, e2e_ms = max_over_ranks(dist, [ms, e2e_ms], dev)
+    del ws, y, x
     return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, stage_ms=stage_ms, counts=counts,
                 clocks=clk.summary(), h2d=wl.T * wl.H * 2, d2h=wl.T * wl.H * 2)
 
@@ -335,32 +403,35 @@ def pipelined_e2e(n, x_pin, y_shape, run, dev):
     return start.elapsed_time(end)
 
 
-
-def run_linear(args, wl, rank, dist):
-    """Dense W4A8 linear (x [M, K] bf16 -> y [M, N] bf16) through w8a8_linear."""
+def run_linear(args, wl, rank, dist, dev):
+    """Dense W4A8 / W8A8 linear (x [M, K] bf16 -> y [M, N] bf16) through w8a8_linear."""
     import torch
 
     from w8a8_int8_quantized_act_b200 import binding as B
     from w8a8_int8_quantized_act_b200 import synth
 
-    local = int(os.environ.get("LOCAL_RANK", 0))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    B.lib()
+    local = dev.index
     x_host = synth.activations(wl.M, wl.K, wl.n_outlier, rank_seed(wl.seed, rank))
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
     x = bf(x_host)
-    packed, sw = B.w8a8_quantize_weight_int4_per_group(bf(synth.dense_weight(wl.N, wl.K, wl.seed)), wl.group)
-    fmt = B.W8A8_W_INT4_PER_GROUP
-    ws = torch.empty(B.w8a8_linear_workspace_size(wl.M, wl.K, wl.N, fmt, wl.group), dtype=torch.uint8, device=dev)
+    w = bf(synth.dense_weight(wl.N, wl.K, wl.seed))
+    if wl.fmt == "int4":
+        wq, sw = B.w8a8_quantize_weight_int4_per_group(w, wl.group)
+        fmt, group = B.W8A8_W_INT4_PER_GROUP, wl.group
+    else:
+        wq, sw = B.w8a8_quantize_weight_per_channel(w)
+        fmt, group = B.W8A8_W_INT8_PER_CHANNEL, 128
+    del w
+    ws = torch.empty(B.w8a8_linear_workspace_size(wl.M, wl.K, wl.N, fmt, group), dtype=torch.uint8, device=dev)
     y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
-    # rotate over weight copies so every step reads its weights from HBM, not from L2
-    copies = [(packed, sw)] + [(packed.clone(), sw.clone()) for _ in range(31)]
+    # rotate over weight copies (more than the L2 together) so every step reads its weights from HBM
+    n_copies = max(2, min(32, -(-256 * 2 ** 20 // (wq.numel() * wq.element_size()))))
+    copies = [(wq, sw)] + [(wq.clone(), sw.clone()) for _ in range(n_copies - 1)]
     stream = torch.cuda.current_stream()
 
     def step(i):
         pk, s_ = copies[i % len(copies)]
-        B.w8a8_linear(x, pk, s_, fmt, wl.group, workspace=ws, y=y)
+        B.w8a8_linear(x, pk, s_, fmt, group, workspace=ws, y=y)
 
     for i in range(args.warmup):
         step(i)
@@ -386,16 +457,9 @@ def run_linear(args, wl, rank, dist):
         torch.cuda.synchronize()
     B.w8a8_check_status()
     ms = start.elapsed_time(stop)
-    # the GEMM alone (dominant kernel): the quantisation is a separate entry point
-    xq, sx = B.w8a8_quant_act_per_token(x)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    direct_ms = e0.elapsed_time(e1)
+    # the GEMM launch alone (the dominant kernel): the quantised activations are made once, then
+    # K GEMM launches are timed with events on the launching stream
+    gemm_ms = time_linear_gemm(B, x, copies, fmt, group, wl, args.steps, stream)
     # end to end with host buffers (copies inside the timed region)
     x_pin = torch.from_numpy(x_host).view(torch.bfloat16).pin_memory()
     n_e2e = max(1, min(args.steps, 200))
@@ -405,7 +469,7 @@ def run_linear(args, wl, rank, dist):
     def run_e2e(xd, yd, st):
         pk, s_ = copies[e2e_i[0] % len(copies)]
         e2e_i[0] += 1
-        B.w8a8_linear(xd, pk, s_, fmt, wl.group, workspace=e2e_ws, y=yd, stream=st)
+        B.w8a8_linear(xd, pk, s_, fmt, group, workspace=e2e_ws, y=yd, stream=st)
 
     pipelined_e2e(3, x_pin, (wl.M, wl.N), run_e2e, dev)  # warm-up
     if dist is not None:
@@ -413,175 +477,304 @@ def run_linear(args, wl, rank, dist):
     e2e_ms = pipelined_e2e(n_e2e, x_pin, (wl.M, wl.N), run_e2e, dev)
     B.w8a8_check_status()
     ms, e2e_ms = max_over_ranks(dist, [ms, e2e_ms], dev)
-    return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=n_e2e, direct_ms=direct_ms, clocks=clk.summary(),
-                h2d=wl.M * wl.K * 2, d2h=wl.M * wl.N * 2)
+    return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=n_e2e, gemm_ms=gemm_ms, clocks=clk.summary(),
+                h2d=wl.M * wl.K * 2, d2h=wl.M * wl.N * 2,
+                weight_bytes=wq.numel() * wq.element_size() + sw.numel() * 4)
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one gate_up launch, from one ncu
-# capture of the bench's own workload, with the sha1 of the CUDA sources the gate_up GEMMs are built
-# from (every csrc file but those holding only other kernels: the quantisation / grouping / combine
-# kernels, the fused short-batch front end and the dense W4A8 GEMM); reported only while those
-# sources are unchanged (null otherwise, since the counters no longer describe the kernel).
-GATE_UP_TRAFFIC = {
-    "qwen3-30b-a3b-decode": (391_960_576 + 5_193_216, "3f41d6b0e52cfb0ce400f8b802937efd3d00cde6"),
-    "qwen3-30b-a3b-prefill": (541_549_568 + 90_793_984, "3f41d6b0e52cfb0ce400f8b802937efd3d00cde6"),
+def time_linear_gemm(B, x, copies, fmt, group, wl, steps, stream):
+    """Mean duration (ms) of the linear's GEMM launch alone: the activations are quantised once,
+    then K launches of w8a8_linear_prequant are timed with CUDA events on `stream`."""
+    import torch
+
+    xq, sx = B.w8a8_quant_act_per_token(x)
+    y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=x.device)
+    for i in range(3):
+        pk, s_ = copies[i % len(copies)]
+        B.w8a8_linear_prequant(xq, sx, pk, s_, fmt, group, y=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        pk, s_ = copies[i % len(copies)]
+        B.w8a8_linear_prequant(xq, sx, pk, s_, fmt, group, y=y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    B.w8a8_check_status()
+    return e0.elapsed_time(e1) / steps
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant kernel,
+# from one ncu capture of that workload, with the sha1 of the CUDA sources the kernel is built from;
+# reported only while those sources are unchanged (null otherwise: the counters no longer describe
+# the kernel). Keys: workload name.
+MEASURED_TRAFFIC = {}
+TRAFFIC_SOURCES = {  # csrc files each dominant kernel is built from
+    "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh", "w8a8.cu"),
+    "w4a8": ("gemm.cuh", "gemm_w4a8.cuh", "gemm_w4a8_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh", "w8a8.cu"),
+    "w8a8": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh", "w8a8.cu"),
 }
 
 
-def csrc_sha1():
+def csrc_sha1(kind: str) -> str:
     import hashlib
-    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "w8a8_int8_quantized_act_b200", "csrc")
+    d = os.path.join(ROOT, "w8a8_int8_quantized_act_b200", "csrc")
     h = hashlib.sha1()
-    for name in sorted(os.listdir(d)):
-        if name in ("elementwise.cuh", "front.cuh", "gemm_w4a8.cuh"):
-            continue
-        with open(os.path.join(d, name), "rb") as f:
-            h.update(f.read())
+    for name in sorted(TRAFFIC_SOURCES[kind]):
+        path = os.path.join(d, name)
+        if os.path.exists(path):
+            with open(path, "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
     return h.hexdigest()
 
 
-def measured_traffic(workload):
-    entry = GATE_UP_TRAFFIC.get(workload)
-    if entry is None or entry[1] != csrc_sha1():
+def measured_traffic(workload: str, kind: str):
+    entry = MEASURED_TRAFFIC.get(workload)
+    if entry is None or entry[1] != csrc_sha1(kind):
         return None
     return entry[0]
 
 
-def main_linear(args, wl, world, rank, peaks, peak_kind):
-    dist = None
-    if world > 1:
-        import datetime
+def tensor_fracs(ops: float, seconds: float, peaks) -> dict:
+    tops = ops / seconds / 1e12
+    derived = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    return {"tops": tops, "frac_of_2x_measured_bf16": tops / derived, "peak_2x_measured_bf16": derived,
+            "frac_of_datasheet": tops / INT8_DATASHEET_TOPS, "peak_datasheet": INT8_DATASHEET_TOPS}
 
-        import torch.distributed as dist_mod
 
-        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        dist = dist_mod
-    res = run_linear(args, wl, rank, dist)
-    if dist is not None:
-        dist.destroy_process_group()
-    if rank != 0:
-        return
-    K = args.steps
+def roofline_entry(ops: float, nbytes: float, seconds: float, peaks, peak_kind, traffic, kernel: str) -> dict:
+    """Roofline of one kernel launch: bound by whichever of its tensor time (at 2 x the measured
+    bf16 rate) and its HBM time (at the measured copy bandwidth) is longer."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tf = tensor_fracs(ops, seconds, peaks)
+    t_ops = ops / (tf["peak_2x_measured_bf16"] * 1e12)
+    t_bytes = nbytes / (hbm * 1e9)
+    gbs = nbytes / seconds / 1e9
+    if t_ops >= t_bytes:
+        roof = {"bound": "tensor", "achieved": tf["tops"], "peak": tf["peak_2x_measured_bf16"], "unit": "TOPS",
+                "frac": tf["frac_of_2x_measured_bf16"],
+                "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8:bf16 ratio)"}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "peak_source": f"{peak_kind} HBM copy GB/s"}
+    roof.update({"traffic": traffic, "traffic_unit": "bytes per launch", "kernel": kernel,
+                 "alg_ops": ops, "alg_bytes": nbytes, "launch_ms": seconds * 1e3,
+                 "tensor": tf, "hbm": {"gbs": gbs, "frac": gbs / hbm, "peak": hbm}})
+    return roof
+
+
+def moe_result(wl, res, K, world, peaks, peak_kind):
+    ms_step = res["ms"] / K
+    alg = algorithmic(wl, res["counts"])
+    st = dict(zip(("router", "group_quant", "gate_up", "requant", "down", "combine"), res["stage_ms"].tolist()))
+    gu_s = st["gate_up"] / 1e3
+    roof = roofline_entry(alg["gate_up_ops"], alg["gate_up_bytes"], gu_s, peaks, peak_kind,
+                          measured_traffic(wl.name, "gate_up"),
+                          "gate_up grouped INT8 GEMM (tcgen05 kind::i8) with the dequant + SiLU*up epilogue")
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    t = ms_step / 1e3
+    layer_tf = tensor_fracs(alg["ops"], t, peaks)
+    t_ops = alg["ops"] / (layer_tf["peak_2x_measured_bf16"] * 1e12)
+    t_bytes = alg["bytes"] / (hbm * 1e9)
+    return {
+        "value": whole_job_rate(world, wl.T, K, res["ms"]), "unit": UNIT, "ms_per_step": ms_step,
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
+                   "skewed_router": wl.skewed, "tokens_per_step_per_gpu": wl.T},
+        "roofline": roof,
+        "layer": {"tops": layer_tf["tops"], "gbs": alg["bytes"] / t / 1e9, "hbm_frac": alg["bytes"] / t / 1e9 / hbm,
+                  "tensor_frac_of_2x_measured_bf16": layer_tf["frac_of_2x_measured_bf16"],
+                  "tensor_frac_of_datasheet": layer_tf["frac_of_datasheet"],
+                  "roofline_frac": max(t_ops, t_bytes) / t,
+                  "roofline_bound": "tensor" if t_ops >= t_bytes else "hbm",
+                  "alg_bytes": alg["bytes"], "alg_ops": alg["ops"], "touched_experts": alg["touched"]},
+        "stage_ms": st,
+        "e2e": {"value": whole_job_rate(world, wl.T, res["e2e_steps"], res["e2e_ms"]), "unit": UNIT,
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "overlap": E2E_OVERLAP},
+        "gpu_launches": moe_launches(wl) * K,
+        "clocks": res["clocks"],
+    }
+
+
+def linear_result(wl, res, K, world, peaks, peak_kind):
     ms_step = res["ms"] / K
     ops = 2.0 * wl.M * wl.N * wl.K
-    int8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = ops / (ms_step / 1e3) / 1e12
-    out = {
-        "metric": METRIC, "value": whole_job_rate(world, wl.M, K, res["ms"]), "unit": UNIT, "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8 (int4 weights unpacked to int8)", "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "group": wl.group,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "32 rotating weight copies (201 MB > L2): each step reads its weights from HBM",
-                   "timing": "CUDA graphs of quantise + GEMM, replayed K times"},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
-                     "frac": achieved / int8_peak, "traffic": None,
-                     "kernel": "w4a8_gemm_kernel (tcgen05 kind::i8, int4 unpacked in shared memory) + x quantisation",
-                     "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8:bf16 ratio)"},
-        "direct_call_ms_per_step": res["direct_ms"] / K,
+    nbytes = res["weight_bytes"] + wl.M * wl.K * 2 + wl.M * wl.N * 2
+    kind = "w4a8" if wl.fmt == "int4" else "w8a8"
+    kernel = ("W4A8 GEMM (tcgen05 kind::i8, int4 unpacked to int8 in shared memory, per-group fp32 scaling)"
+              if wl.fmt == "int4" else "W8A8 GEMM (tcgen05 kind::i8, per-token x per-channel dequant epilogue)")
+    roof = roofline_entry(ops, nbytes, res["gemm_ms"] / 1e3, peaks, peak_kind, measured_traffic(wl.name, kind), kernel)
+    step_tf = tensor_fracs(ops, ms_step / 1e3, peaks)
+    return {
+        "value": whole_job_rate(world, wl.M, K, res["ms"]), "unit": UNIT, "ms_per_step": ms_step,
+        "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "weights": wl.fmt,
+                   "group": wl.group if wl.fmt == "int4" else None},
+        "roofline": roof,
+        "step": {"tops": step_tf["tops"], "tensor_frac_of_2x_measured_bf16": step_tf["frac_of_2x_measured_bf16"],
+                 "tensor_frac_of_datasheet": step_tf["frac_of_datasheet"],
+                 "note": "step = per-token activation quantisation + GEMM"},
         "e2e": {"value": whole_job_rate(world, wl.M, res["e2e_steps"], res["e2e_ms"]), "unit": UNIT,
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "overlap": E2E_OVERLAP},
-        "gpu_launches": 2 * K, "clocks": res["clocks"],
+        "gpu_launches": 2 * K,
+        "clocks": res["clocks"],
     }
-    print(json.dumps(out))
+
+
+def moe_cpu_baseline(wl, sample, min_s, max_s):
+    rate, reps, el = cpu_oracle_rate(wl, sample, min_s, max_s)
+    return {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{sample} of the workload's {wl.T} tokens per oracle forward, {reps} forwards in {el:.1f} s"}
+
+
+def linear_cpu_baseline(wl, sample, min_s, max_s):
+    rate, reps, el = cpu_oracle_linear_rate(wl, sample, min_s, max_s)
+    return {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{sample} of the workload's {wl.M} rows per oracle call, {reps} calls in {el:.1f} s"}
+
+
+def int8_gemm_probe(dev, steps=20, n=8192):
+    """Rate of this library's plain int8 GEMM (w8a8_gemm_s8s8s32) on an n x n x n problem: the
+    build's own measured tcgen05 kind::i8 throughput, for context next to the peaks."""
+    import torch
+
+    from w8a8_int8_quantized_act_b200 import binding as B
+
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    c = torch.empty((n, n), dtype=torch.int32, device=dev)
+    for _ in range(3):
+        B.w8a8_gemm_s8s8s32(a, b, c)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        B.w8a8_gemm_s8s8s32(a, b, c)
+    e1.record()
+    torch.cuda.synchronize()
+    B.w8a8_check_status()
+    ms = e0.elapsed_time(e1) / steps
+    del a, b, c
+    torch.cuda.empty_cache()
+    return {"shape": [n, n, n], "ms": ms, "tops": 2.0 * n ** 3 / (ms / 1e3) / 1e12}
+
+
+def top_line(metric_res, name, args, world):
+    out = {"metric": METRIC, "value": metric_res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": metric_res["ms_per_step"], "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic"}
+    cfg = dict(metric_res["config"])
+    cfg.update({"parallelism": f"replicas x{world}",
+                "l2": "inputs larger than L2: each step streams more than 126 MB of int8 weights",
+                "timing": "CUDA graph of one step, replayed K times; stage / GEMM times from a second pass"})
+    out["config"] = cfg
+    for key in ("roofline", "layer", "step", "stage_ms", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
+        if key in metric_res:
+            out[key] = metric_res[key]
+    return out
+
+
+def init_dist(world):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist_mod
+
+    dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist_mod
 
 
 def main():
     args = parse()
     from w8a8_int8_quantized_act_b200 import synth
 
-    if args.workload in synth.LINEAR_WORKLOADS:
-        world = int(os.environ.get("WORLD_SIZE", "1"))
-        rank = int(os.environ.get("RANK", "0"))
-        peaks, peak_kind = load_peaks()
-        if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable": "the CPU-oracle reference arm covers the MoE "
-                              "workloads; run it with the default workload"}))
-            return
-        return main_linear(args, synth.LINEAR_WORKLOADS[args.workload], world, rank, peaks, peak_kind)
-    wl = synth.MOE_WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     peaks, peak_kind = load_peaks()
-    sample = args.cpu_sample_tokens or default_sample_tokens(wl)
+    name = args.workload or HEADLINE
+    single = args.workload is not None
 
     if args.impl == "reference":
         if rank != 0:
             return
-        rate, reps, el = cpu_oracle_rate(wl, sample, min_seconds=min(30.0, 2.0 * max(1, args.steps)),
-                                         max_seconds=120.0)
-        cores = blas_threads()
-        samp = f"{sample} of the workload's {wl.T} tokens per step, {reps} oracle forwards in {el:.1f} s"
+        if name in synth.LINEAR_WORKLOADS:
+            wl = synth.LINEAR_WORKLOADS[name]
+            sample = args.cpu_sample_tokens or 16
+            base = linear_cpu_baseline(wl, sample, min(30.0, 2.0 * max(1, args.steps)), 120.0)
+            cfg = {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "weights": wl.fmt}
+        else:
+            wl = synth.MOE_WORKLOADS[name]
+            sample = args.cpu_sample_tokens or default_sample_tokens(wl)
+            base = moe_cpu_baseline(wl, sample, min(30.0, 2.0 * max(1, args.steps)), 120.0)
+            cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I}
         print(json.dumps({
-            "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+            "impl": "reference", "metric": METRIC, "value": base["value"], "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I},
-            "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": samp},
-            "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic", "config": cfg,
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
         return
 
-    dist = None
-    if world > 1:
-        import datetime
+    import torch
 
-        import torch.distributed as dist_mod
+    from w8a8_int8_quantized_act_b200 import binding as B
 
-        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        dist = dist_mod
-    res = run_native(args, wl, rank, world, dist)
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B.lib()
+    dist = init_dist(world)
+    K = args.steps
+
+    def run_one(wname, layer_cache):
+        if wname in synth.LINEAR_WORKLOADS:
+            wl = synth.LINEAR_WORKLOADS[wname]
+            res = run_linear(args, wl, rank, dist, dev)
+            return wl, linear_result(wl, res, K, world, peaks, peak_kind)
+        wl = synth.MOE_WORKLOADS[wname]
+        key = (wl.H, wl.E, wl.I, wl.seed)
+        if layer_cache.get("key") != key:
+            layer_cache.clear()
+            torch.cuda.empty_cache()
+            layer_cache["key"], layer_cache["layer"] = key, MoELayer(wl, dev)
+        res = run_moe(args, wl, layer_cache["layer"], rank, dist, dev)
+        return wl, moe_result(wl, res, K, world, peaks, peak_kind)
+
+    cache = {}
+    wl, head = run_one(name, cache)
+    subs = {}
+    probe = None
+    if not single and world == 1:
+        for wname in SUB_MOE + SUB_LINEAR:
+            _, subs[wname] = run_one(wname, cache)
+        cache.clear()
+        torch.cuda.empty_cache()
+        probe = int8_gemm_probe(dev)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
-
-    K = args.steps
-    ms_step = res["ms"] / K
-    value = whole_job_rate(world, wl.T, K, res["ms"])
-    e2e_value = whole_job_rate(world, wl.T, res["e2e_steps"], res["e2e_ms"])
-    alg = algorithmic(wl, res["counts"])
-    st = dict(zip(("router", "group_quant", "gate_up", "requant", "down", "combine"), res["stage_ms"].tolist()))
-    # dominant kernel: the gate_up GEMM (largest share of every step)
-    prefill_like = wl.T * wl.k >= 4096
-    gu_s = st["gate_up"] / 1e3
-    if prefill_like:
-        int8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-        achieved = alg["gate_up_ops"] / gu_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
-                "frac": achieved / int8_peak, "traffic": measured_traffic(wl.name), "traffic_unit": "bytes per launch",
-                "kernel": "gate_up grouped INT8 GEMM (tcgen05 kind::i8)",
-                "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8:bf16 ratio)"}
-    else:
-        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-        achieved = alg["gate_up_bytes"] / gu_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": measured_traffic(wl.name), "traffic_unit": "bytes per launch",
-                "kernel": "gate_up grouped INT8 GEMM (tcgen05 kind::i8)",
-                "peak_source": f"{peak_kind} HBM copy GB/s"}
-    out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8", "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
-                   "tokens_per_step_per_gpu": wl.T, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: each step streams the touched experts' int8 weights",
-                   "timing": "CUDA graph of one forward, replayed K times; stage times from a second pass"},
-        "roofline": roof,
-        "layer": {"tops": alg["ops"] / (ms_step / 1e3) / 1e12, "gbs": alg["bytes"] / (ms_step / 1e3) / 1e9,
-                  "hbm_frac": alg["bytes"] / (ms_step / 1e3) / 1e9 / float(peaks.get("hbm_gbs", 6650.0)),
-                  "alg_bytes": alg["bytes"], "alg_ops": alg["ops"], "touched_experts": alg["touched"]},
-        "stage_ms": st,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
-                "d2h_bytes_per_step": res["d2h"], "overlap": E2E_OVERLAP},
-        "gpu_launches": (5 if (wl.T <= 128 and wl.H <= 2048) else (7 if wl.T <= 512 else 6)) * K,
-        "clocks": res["clocks"],
-    }
-    if not args.no_cpu_baseline:
-        rate, reps, el = cpu_oracle_rate(wl, sample)
-        out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                               "sample": f"{sample} tokens of the workload per oracle forward, {reps} forwards "
-                                         f"in {el:.1f} s"}
+    if not args.no_cpu_baseline and world == 1:
+        if name in synth.LINEAR_WORKLOADS:
+            head["cpu_baseline"] = linear_cpu_baseline(wl, args.cpu_sample_tokens or 16, 10.0, 30.0)
+        else:
+            head["cpu_baseline"] = moe_cpu_baseline(wl, args.cpu_sample_tokens or default_sample_tokens(wl), 10.0,
+                                                    30.0)
+        for wname, sub in subs.items():
+            if wname in synth.LINEAR_WORKLOADS:
+                sub["cpu_baseline"] = linear_cpu_baseline(synth.LINEAR_WORKLOADS[wname], 16, 4.0, 12.0)
+            else:
+                swl = synth.MOE_WORKLOADS[wname]
+                sub["cpu_baseline"] = moe_cpu_baseline(swl, default_sample_tokens(swl), 4.0, 12.0)
+    out = top_line(head, name, args, world)
+    if name in synth.LINEAR_WORKLOADS:
+        out["dtype"] = "int8 (int4 weights unpacked to int8)" if wl.fmt == "int4" else "int8"
+    if subs:
+        out["sub_results"] = subs
+    if probe is not None:
+        out["int8_gemm_probe"] = probe
     print(json.dumps(out))
 
 

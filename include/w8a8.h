@@ -17,7 +17,8 @@
  *     gate_proj and up_proj of an expert concatenated along the output dimension into
  *     gate_up_proj; down_proj kept separate.
  *
- * Conventions for every entry point:
+ * Each declaration below names the passage that defines its operation. Conventions for every
+ * entry point:
  *   - Pointers are device memory owned by the caller unless stated otherwise; the library
  *     never allocates, frees or retains them. bf16 tensors are passed as their raw 16-bit
  *     patterns (w8a8_bf16). All tensors are row-major and contiguous.
@@ -66,6 +67,9 @@ const char* w8a8_status_string(int status);
 int w8a8_check_status(w8a8_stream stream);
 
 /* Static per-output-channel int8 weight quantisation (offline weight preparation).
+ * Defined by: "Qwen3.6-35B-A3B-w8a8量化配置深度解读：config.json与recipe.yaml关键参数解析", block
+ * config_groups.group_0.weights (num_bits 8, strategy channel, symmetric, dynamic false, min-max
+ * observer); "Qwen3-30B-A3B-Instruct-2507-quantized.w8a8" explainer, section 二.
  *   w      bf16 [G, N, K]   G blocks (experts) of nn.Linear weights [out = N, in = K]
  *   q      int8 [G, N, K]   codes clamp(rne(w / scale), -127, 127)
  *   scale  fp32 [G, N]      max |w[g, n, :]| / 127 (0 for an all-zero row)
@@ -74,6 +78,8 @@ int w8a8_quantize_weight_per_channel(const w8a8_bf16* w, int64_t G, int64_t N, i
                                      float* scale, w8a8_stream stream);
 
 /* Symmetric int4 weight quantisation with one scale per `group` consecutive K values.
+ * Defined by: "Qwen3-1.7B-W4A8-V1" explainer, section "4bit 权重", items 1 (group_size 128) and 2
+ * (two's-complement codes packed two per byte).
  *   w       bf16 [N, K]
  *   packed  uint8 [N, K/2]   byte i = code(2i) & 0xF | (code(2i+1) & 0xF) << 4, codes in [-7, 7]
  *   scale   fp32 [N, K/group] max |w| over the group / 7
@@ -82,6 +88,9 @@ int w8a8_quantize_weight_int4_per_group(const w8a8_bf16* w, int64_t N, int64_t K
                                         float* scale, w8a8_stream stream);
 
 /* Dynamic per-token symmetric int8 activation quantisation.
+ * Defined by: the group_0.input_activations block of the Qwen3.6-35B-A3B-w8a8 config page
+ * (num_bits 8, strategy token, symmetric, dynamic true); "Qwen3-1.7B-W4A8-V1" explainer,
+ * section "8bit 激活" (each token's scale computed online).
  *   x      bf16 [T, K]
  *   q      int8 [T, K]   clamp(rne(x / scale), -127, 127)
  *   scale  fp32 [T]      max |x[t, :]| / 127 (0 for an all-zero token)
@@ -89,7 +98,11 @@ int w8a8_quantize_weight_int4_per_group(const w8a8_bf16* w, int64_t N, int64_t K
 int w8a8_quant_act_per_token(const w8a8_bf16* x, int64_t T, int64_t K, int8_t* q, float* scale,
                              w8a8_stream stream);
 
-/* BF16 router (never quantised): logits = x . wg^T (+ bias) accumulated in fp32 on the tensor
+/* Defined by: "Qwen3-30B-A3B-Instruct-2507-quantized.w8a8" explainer, section 三 3.1 (mlp.gate
+ * maps the hidden state to one score per expert, softmax, top-8) and the recipe's ignore list
+ * (re:.*mlp.gate$: the gate stays bf16); "Qwen3-235B-A22B-quantized.w8a8" model table (128
+ * experts, 8 per token).
+ * BF16 router (never quantised): logits = x . wg^T (+ bias) accumulated in fp32 on the tensor
  * cores, softmax over the E experts, top-k by descending probability (equal values: lower
  * expert first), weights renormalised over the k selected experts when renorm != 0.
  *   x              bf16 [T, H]
@@ -126,11 +139,15 @@ int w8a8_moe_workspace_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I,
 /* Workspace bytes w8a8_moe_forward needs for this shape (0 if the shape is rejected). */
 size_t w8a8_moe_workspace_size(int64_t T, int64_t H, int64_t E, int k, int64_t I);
 
-/* W8A8 MoE expert-FFN forward of one Qwen3-MoE layer:
+/* Defined by: the group_0 block of the Qwen3.6-35B-A3B-w8a8 config page (int8 per-channel
+ * static weights, int8 per-token dynamic activations for every expert Linear, gate_proj,
+ * up_proj and down_proj alike); "Qwen3-Next-80B-A3B-Instruct 在 AMCT 中的 MoE 混合注意力量化适配实战",
+ * section 二 2.2 (gate_proj and up_proj concatenated into gate_up_proj); the router as above.
+ * W8A8 MoE expert-FFN forward of one Qwen3-MoE layer:
  *   route (bf16) -> per-token int8 x -> grouped int8 gate_up GEMM (int32) -> dequant
  *   ((acc * s_x) * s_gu), SiLU(gate) * up -> bf16 h -> per-row int8 requantisation of h ->
  *   grouped int8 down GEMM -> dequant ((acc * s_h) * s_d) -> bf16 o -> y[t] = bf16(sum_j
- *   w[t,j] * o[t,j]) (fp32 products and sums in slot order).
+ *   w[t,j] * o[t,j]) (one fp32 fused multiply-add per slot, in slot order from 0).
  *   x     bf16 [T, H];  wg bf16 [E, H];  bias fp32 [E] or NULL
  *   wgu   int8 [E, 2I, H]  packed gate_up: rows 0..I-1 gate_proj, rows I..2I-1 up_proj
  *   s_gu  fp32 [E, 2I]     per-channel scales of wgu
@@ -170,7 +187,10 @@ int w8a8_moe_forward_profiled(const w8a8_bf16* x, const w8a8_bf16* wg, const flo
  *     anything is enqueued; that covers decode-sized batches (up to about 240 tokens of the
  *     Qwen3-30B-A3B shaped layer, about 120 of the Qwen3-235B-A22B shaped one), not prefill.
  *   - The first call on a device looks the buffer's address up on that device (the device
- *     must be current). Make that first call before any stream capture begins.
+ *     must be current) and caches it with the device's context; a call in a different context
+ *     of that device (after a device reset) looks it up again. Make the first call on a device
+ *     before any stream capture begins. Devices with an index of 64 or more are not covered:
+ *     the call returns W8A8_ERR_UNSUPPORTED there.
  *   - All calls on one device share the one buffer; each call overwrites it and resets what
  *     must start at zero. Calls whose work overlaps on the GPU (different streams without
  *     ordering between them) race on the buffer: serialise them, e.g. on one stream. The
@@ -183,7 +203,10 @@ int w8a8_moe_forward_noalloc(const w8a8_bf16* x, const w8a8_bf16* wg, const floa
 /* Workspace bytes w8a8_linear needs (0 if the shape is rejected). */
 size_t w8a8_linear_workspace_size(int64_t M, int64_t K, int64_t N, int w_format, int group);
 
-/* Dense W8A8 / W4A8 linear: y = x . W^T with per-token dynamic int8 x.
+/* Defined by: the group_0 block of the Qwen3.6-35B-A3B-w8a8 config page (int8 formats);
+ * "Qwen3-235B-A22B-quantized.w8a8" shard contents (q/k/v/o projections in INT8); the
+ * "Qwen3-1.7B-W4A8-V1" explainer, sections "4bit 权重" and "8bit 激活" (int4 format).
+ * Dense W8A8 / W4A8 linear: y = x . W^T with per-token dynamic int8 x.
  *   W8A8_W_INT8_PER_CHANNEL: w int8 [N, K], sw fp32 [N]; y = bf16(((float)acc * s_x) * sw[n]).
  *   W8A8_W_INT4_PER_GROUP:   w uint8 [N, K/2] (packing as above), sw fp32 [N, K/group];
  *     y = bf16(acc_f * s_x) with acc_f = sum over groups g in order of (float)acc_g * sw[n, g],
@@ -193,7 +216,15 @@ size_t w8a8_linear_workspace_size(int64_t M, int64_t K, int64_t N, int w_format,
 int w8a8_linear(const w8a8_bf16* x, const void* w, const float* sw, int w_format, int group, int64_t M,
                 int64_t K, int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream);
 
-/* Exact integer GEMM on the tensor cores: c[m, n] = sum_k a[m, k] * b[n, k] in int32.
+/* The GEMM of w8a8_linear on activations already quantised per token (for example by
+ * w8a8_quant_act_per_token, or by a producer that emits int8 codes directly):
+ *   xq int8 [M, K], sx fp32 [M] (per-token scales); w, sw, w_format, group, y as w8a8_linear.
+ * Same shape rules and results as w8a8_linear given the same xq and sx; needs no workspace. */
+int w8a8_linear_prequant(const int8_t* xq, const float* sx, const void* w, const float* sw, int w_format, int group,
+                         int64_t M, int64_t K, int64_t N, w8a8_bf16* y, w8a8_stream stream);
+
+/* Exact integer GEMM on the tensor cores: c[m, n] = sum_k a[m, k] * b[n, k] in int32: the
+ * int8 x int8 product every W8A8 Linear of the group_0 scheme accumulates before its scales.
  *   a int8 [M, K], b int8 [N, K], c int32 [M, N];  K % 128 == 0, N % 128 == 0. */
 int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
                       w8a8_stream stream);
@@ -216,7 +247,11 @@ int w8a8_debug_ex2_approx_ulp(uint32_t first_bits, uint32_t count, unsigned int*
 
 /* Test hook for the bounded waits: launches one CTA that waits on an mbarrier phase nothing
  * completes; after `timeout_ns` the wait gives up and sets the device error word, which the
- * next w8a8_check_status() reports as W8A8_ERR_DEVICE. The context stays usable. */
+ * next w8a8_check_status() reports as W8A8_ERR_DEVICE. The context stays usable.
+ * Every wait inside the library's kernels is bounded the same way: a single wait (an mbarrier
+ * phase, a grid barrier) that has not completed 2 s after it began (or the number of
+ * milliseconds in the environment variable W8A8_WAIT_TIMEOUT_MS, read once per process) gives
+ * up. The bound applies to each wait on its own, not to the lifetime of a kernel. */
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream);
 
 #ifdef __cplusplus

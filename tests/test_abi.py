@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.w8a8_version() == 100
+    assert lib.w8a8_version() == 200
     for st in range(-5, 1):
         assert B.status_string(st) not in ("", "unknown status")
 

@@ -61,6 +61,7 @@ SIGNATURES = {
                                         _int, _c_p, _c_p]),
     "w8a8_linear_workspace_size": (_size, [_i64, _i64, _i64, _int, _int]),
     "w8a8_linear": (_int, [_c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _size, _c_p, _c_p]),
+    "w8a8_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_gemm_s8s8s32": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
     "w8a8_debug_rcp_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
@@ -287,6 +288,19 @@ def w8a8_linear(x, w, sw, w_format: int = W8A8_W_INT8_PER_CHANNEL, group: int = 
     y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
     _check(lib().w8a8_linear(_ptr(x), _ptr(w), _ptr(sw), w_format, group, M, K, N, _ptr(workspace),
                              workspace.numel(), _ptr(y), _stream(stream)), "w8a8_linear")
+    return y
+
+
+def w8a8_linear_prequant(xq, sx, w, sw, w_format: int = W8A8_W_INT8_PER_CHANNEL, group: int = 128, y=None,
+                         stream=None):
+    """The dense linear's GEMM on per-token int8 activations xq [M, K] with scales sx [M]."""
+    if xq.dtype != torch.int8 or sx.dtype != torch.float32:
+        raise TypeError("expected int8 codes and fp32 scales")
+    M, K = xq.shape
+    N = w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if y is None else y
+    _check(lib().w8a8_linear_prequant(_ptr(xq), _ptr(sx), _ptr(w), _ptr(sw), w_format, group, M, K, N, _ptr(y),
+                                      _stream(stream)), "w8a8_linear_prequant")
     return y
 
 

@@ -237,7 +237,7 @@ __global__ void wait_timeout_probe_kernel(uint64_t timeout_ns) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const WaitCtx wc{&abort_flag, globaltimer_ns() + timeout_ns};
+    const WaitCtx wc{&abort_flag, timeout_ns};
     mbar_wait(&bar, 0, wc);
   }
 }

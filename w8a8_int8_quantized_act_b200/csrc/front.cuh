@@ -29,13 +29,15 @@ constexpr int kFrontWarps = kFrontThreads / 32;
 
 // Arrival number `round` (1, 2, ...) of every CTA on *count (zeroed before the launch): waits
 // until all `nctas` CTAs have arrived `round` times. Needs every CTA resident at once (a
-// cooperative launch). Bounded by `deadline`: past it the error word is raised and false returned.
-__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned nctas, unsigned round, uint64_t deadline,
+// cooperative launch). Bounded: a CTA that has waited longer than `timeout_ns` raises the error
+// word and returns false.
+__device__ __forceinline__ bool grid_barrier(unsigned* count, unsigned nctas, unsigned round, uint64_t timeout_ns,
                                              int* ok_smem) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     atomicAdd(count, 1u);
+    const uint64_t deadline = globaltimer_ns() + timeout_ns;
     int ok = 1;
     while (true) {
       unsigned v;
@@ -70,7 +72,6 @@ __global__ void __launch_bounds__(kFrontThreads) front_small_kernel(
 
   pdl_wait();
   pdl_launch_dependents();
-  const uint64_t deadline = globaltimer_ns() + timeout_ns;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x;
 
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(kFrontThreads) front_small_kernel(
     router_logits_item_xs<RU>(xrows[hf], wv, T, H, E, logits, item - tg * neg, tg, warp & 7);
     asm volatile("bar.sync %0, 256;" ::"r"(1 + hf) : "memory");  // the rows are rewritten by the next item
   }
-  if (!grid_barrier(sync_count, unsigned(G), 1u, deadline, &ok_smem)) return;
+  if (!grid_barrier(sync_count, unsigned(G), 1u, timeout_ns, &ok_smem)) return;
 
   // phase 2: top-k, one warp per token, spread over the CTAs first (token t on warp t / G of
   // CTA t % G), so that no SM sub-partition interleaves several tokens' selections (logits
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(kFrontThreads) front_small_kernel(
     warp_topk_token<PER>([&](int e) { return __ldcg(row + e); }, E, k, renorm != 0, bias, ids + size_t(t) * k,
                          w + size_t(t) * k, nullptr);
   }
-  if (!grid_barrier(sync_count, unsigned(G), 2u, deadline, &ok_smem)) return;
+  if (!grid_barrier(sync_count, unsigned(G), 2u, timeout_ns, &ok_smem)) return;
 
   // phase 3: counting sort by expert, stable by token, in every CTA
   for (int i = threadIdx.x; i < 4 * E; i += kFrontThreads) mask[i] = 0u;

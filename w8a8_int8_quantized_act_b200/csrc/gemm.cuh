@@ -379,7 +379,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const WaitCtx wc{abort_flag, globaltimer_ns() + p.timeout_ns};
+  const WaitCtx wc{abort_flag, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     if (lane == 0 && *abort_flag) {
       // let every load already issued land before the CTA's shared memory goes away
       volatile int no_abort = 0;
-      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      const WaitCtx dw{&no_abort, 100000000ull};
       for (int s = 0; s < STAGES; ++s)
         if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
     }
@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
       // before TMEM is released
       tc_commit(drain);
       volatile int no_abort = 0;
-      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      const WaitCtx dw{&no_abort, 100000000ull};
       mbar_wait(drain, 0, dw);
     }
     __syncwarp();

@@ -286,7 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
   const bool leader = rank == 0;
   const int cluster = int(cluster_index());
   const int nclusters = int(cluster_count());
-  const WaitCtx wc{abort_flag, globaltimer_ns() + p.timeout_ns};
+  const WaitCtx wc{abort_flag, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
@@ -392,7 +392,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
       // let every load already issued land before the CTA's shared memory goes away: rank 0
       // sees both ranks' bytes on its barriers; rank 1 cannot observe them and waits 1 ms
       volatile int no_abort = 0;
-      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      const WaitCtx dw{&no_abort, 100000000ull};
       if (leader) {
         for (int s = 0; s < STAGES; ++s)
           if (issued_mask & (1u << s)) mbar_wait(full + s, (issued_parity >> s) & 1u, dw);
@@ -461,7 +461,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
         // before TMEM is released
         tc_commit_pair(smem_addr(drain));
         volatile int no_abort = 0;
-        const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+        const WaitCtx dw{&no_abort, 100000000ull};
         mbar_wait(drain, 0, dw);
       }
     }

@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const WaitCtx wc{abort_flag, globaltimer_ns() + p.timeout_ns};
+  const WaitCtx wc{abort_flag, p.timeout_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < XS; ++s) { mbar_init(xfull + s, 1); mbar_init(xempty + s, 1); }
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
     }
     if (lane == 0 && *abort_flag) {  // loads still in flight land before the CTA exits
       volatile int no_abort = 0;
-      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      const WaitCtx dw{&no_abort, 100000000ull};
       for (int s = 0; s < XS; ++s)
         if (x_issued & (1u << s)) mbar_wait(xfull + s, (x_parity >> s) & 1u, dw);
       for (int s = 0; s < WS; ++s)
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
     if (lane == 0 && *abort_flag && issued_any) {
       tc_commit(drain);
       volatile int no_abort = 0;
-      const WaitCtx dw{&no_abort, globaltimer_ns() + 100000000ull};
+      const WaitCtx dw{&no_abort, 100000000ull};
       mbar_wait(drain, 0, dw);
     }
     __syncwarp();

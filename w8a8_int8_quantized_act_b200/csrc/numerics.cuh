@@ -153,7 +153,9 @@ __device__ __forceinline__ float dequant(int32_t acc, float s_row, float s_col) 
 // exactly as __float2int_rn for |y| < 2^22, and the low byte of r's bit pattern is that integer
 // as an int8 code (|y| <= 127 * (1 + 2^-22) here, so no clamp is needed). d = y - rint(y) is
 // exact; |d| >= 0.5 - 3e-5 is the same near-tie test as sym_code_fast, and a vector holding such a
-// value takes the true divide for all eight.
+// value takes the true divide for all eight. A row whose amax is below about 2^-121 has a
+// subnormal scale whose reciprocal overflows to +inf: y is then +-inf or NaN, d is NaN, and the
+// test is written so that NaN also counts as unsure and takes the true divide.
 __device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv) {
   if (s == 0.0f) return make_uint2(0u, 0u);
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
@@ -168,7 +170,7 @@ __device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv) {
       const float y = __fmul_rn(x, inv);
       const float r = __fadd_rn(y, kMagic);
       const float d = __fsub_rn(y, __fsub_rn(r, kMagic));
-      unsure |= fabsf(d) >= 0.49997f;
+      unsure |= !(fabsf(d) < 0.49997f);
       c[2 * j + h] = __float_as_uint(r);
     }
   }

@@ -1,7 +1,9 @@
 // Thin wrappers over the sm_100a instructions the kernels use: mbarriers, TMA tile loads,
 // and the tcgen05 tensor-core family (TMEM allocation, MMA, commit, TMEM loads, fences).
-// Every wait on an mbarrier is bounded by a %globaltimer deadline; a wait that runs out
-// raises the CTA's abort flag and the library's device error word instead of hanging.
+// Every wait on an mbarrier is bounded: a wait that has not completed `timeout` nanoseconds
+// (by %globaltimer) after it began raises the CTA's abort flag and the library's device error
+// word instead of hanging. The bound is per wait, so a long-running CTA whose waits each
+// complete in time is never cut short.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -75,21 +77,24 @@ __device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, 
   return ok != 0;
 }
 
-// Bounded wait context: the CTA-wide abort flag (shared memory) and the absolute deadline.
+// Bounded wait context: the CTA-wide abort flag (shared memory) and the longest time, in
+// nanoseconds, that any single wait may take.
 struct WaitCtx {
   volatile int* abort;
-  uint64_t deadline;
+  uint64_t timeout;
 };
 
 // Waits for the phase of `bar` with parity `parity` to complete. Returns false (without
-// waiting further) when the CTA is aborting or when the deadline passes; the latter sets the
-// abort flag and the device error word.
+// waiting further) when the CTA is aborting or when the wait has lasted longer than
+// w.timeout; the latter sets the abort flag and the device error word. The deadline is taken
+// when the phase is first found incomplete, so the fast path reads no timer.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_test(bar, parity)) return true;
+  const uint64_t deadline = globaltimer_ns() + w.timeout;
   while (true) {
     if (mbar_test_sleep(bar, parity, 20000u)) return true;
     if (*w.abort) return false;
-    if (globaltimer_ns() > w.deadline) {
+    if (globaltimer_ns() > deadline) {
       *w.abort = 1;
       atomicOr(&g_error_word, kErrWaitTimeout);
       return false;

@@ -16,7 +16,7 @@
 namespace w8a8 {
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0
 
 cudaStream_t as_stream(w8a8_stream s) { return static_cast<cudaStream_t>(s); }
 
@@ -391,9 +391,9 @@ constexpr int64_t kPairMinRows = 128;
 // CTA pairs.
 bool small_token_blocks(int64_t A, int64_t E) { return A <= 32 * E; }
 
-// CTAs per 128-token chunk of the grouping kernel: enough warps for every token of a small
-// batch, fewer for long ones (each CTA re-derives its chunk's positions).
-int group_quant_splits(int64_t T) { return T <= 1024 ? 8 : 8; }
+// CTAs per 128-token chunk of the grouping kernel (each re-derives the chunk's positions and
+// quantises every 8th token of the chunk).
+int group_quant_splits() { return 8; }
 
 }  // namespace
 }  // namespace w8a8
@@ -555,7 +555,7 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     // 2. group assignments by expert and quantise every token once into its sorted rows
     const size_t gq_smem = sizeof(int) * (2 * E + 2 * kChunk * k + 4 * E);
     mark(ev, 1, s);
-    rc = launch_group_quant(dim3(C, group_quant_splits(T)), gq_smem, s, x, ids, tile_counts, int(T), int(H),
+    rc = launch_group_quant(dim3(C, group_quant_splits()), gq_smem, s, x, ids, tile_counts, int(T), int(H),
                             int(E), k, offsets, perm, sx, sx_sorted, xq);
     if (rc != W8A8_OK) return rc;
   }
@@ -693,21 +693,53 @@ namespace {
 constexpr size_t kNoallocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
+constexpr int kNoallocMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {nullptr};
+struct NoallocSlot {
+  void* ptr;      // device address of g_noalloc_scratch
+  void* context;  // the CUDA context that address belongs to
+};
+NoallocSlot g_noalloc_slot[kNoallocMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (first call per device looks it
-// up with that device current); nullptr if the lookup fails.
-void* noalloc_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The calling thread's current CUDA context (nullptr if none is bound yet or the query fails).
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of g_noalloc_scratch on the current device. The address is looked up with
+// cudaGetSymbolAddress, with that device current, the first time a device is used, and cached
+// together with the context it was found in. If the current context differs later (the device
+// was reset and the library's module loaded again, possibly at another address), it is looked
+// up again. Returns W8A8_OK, W8A8_ERR_UNSUPPORTED for a device index the cache does not cover,
+// or W8A8_ERR_LAUNCH if the runtime cannot give the address.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W8A8_ERR_LAUNCH;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return W8A8_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  void* ctx = current_context();
+  if (slot.ptr == nullptr || ctx == nullptr || ctx != slot.context) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return W8A8_ERR_LAUNCH;
+    slot.ptr = p;
+    slot.context = current_context();  // bound by now: the lookup made the device's context current
   }
-  return g_noalloc_ptr[dev];
+  *out = slot.ptr;
+  return W8A8_OK;
 }
 
 }  // namespace
@@ -724,8 +756,9 @@ int w8a8_moe_forward_noalloc(const w8a8_bf16* x, const w8a8_bf16* wg, const floa
   w8a8_moe_ws_layout L;
   fill_layout(T, H, E, k, I, &L);
   if (L.total > kNoallocScratchBytes) return W8A8_ERR_UNSUPPORTED;
-  void* scratch = noalloc_scratch();
-  if (scratch == nullptr) return W8A8_ERR_LAUNCH;
+  void* scratch = nullptr;
+  const int sst = noalloc_scratch(&scratch);
+  if (sst != W8A8_OK) return sst;
   return moe_forward_impl(x, wg, bias, wgu, s_gu, wd, s_d, T, H, E, k, I, renorm, scratch, kNoallocScratchBytes, y,
                           stream, nullptr);
 }
@@ -747,30 +780,20 @@ size_t w8a8_linear_workspace_size(int64_t M, int64_t K, int64_t N, int w_format,
   return align256(size_t(Mp) * K) + align256(sizeof(float) * Mp) + 256;
 }
 
-int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_format, int group, int64_t M, int64_t K,
-                int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream) {
-  if (M < 0 || K <= 0 || N <= 0) return W8A8_ERR_ARG;
-  const size_t need = w8a8_linear_workspace_size(M, K, N, w_format, group);
-  if (need == 0) return W8A8_ERR_UNSUPPORTED;
-  if (M == 0) return W8A8_OK;
-  if (!x || !wq || !sw || !workspace || !y) return W8A8_ERR_ARG;
-  if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
-  if (!aligned16(x) || !aligned16(wq) || !aligned16(y) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return W8A8_ERR_UNSUPPORTED;
-  if (w_format == W8A8_W_INT4_PER_GROUP && (K / 128) > (int64_t(1) << 20)) return W8A8_ERR_UNSUPPORTED;
-  if (M >= (int64_t(1) << 30) || N * K >= (int64_t(1) << 40)) return W8A8_ERR_UNSUPPORTED;
-  const int64_t Mp = round_up(M, 128);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int8_t* xq = reinterpret_cast<int8_t*>(ws);
-  float* sx = reinterpret_cast<float*>(ws + align256(size_t(Mp) * K));
-  cudaStream_t s = as_stream(stream);
-  int rc = w8a8_quant_act_per_token(x, M, K, xq, sx, stream);
-  if (rc != W8A8_OK) return rc;
+}  // extern "C"
+
+namespace w8a8 {
+namespace {
+
+// The GEMM of the dense linear on already quantised activations: xq int8 [M, K] (rows past M
+// are read as zeros), sx fp32 [M]. Arguments are checked by the callers.
+int linear_gemm(const int8_t* xq, const float* sx, const void* wq, const float* sw, int w_format, int64_t M,
+                int64_t K, int64_t N, w8a8_bf16* y, cudaStream_t s) {
   if (w_format == W8A8_W_INT4_PER_GROUP) {
     W4A8Params q{};
     if (!make_plain_map(&q.tmW, wq, uint64_t(K / 2), uint64_t(N), 64, 128) ||
         !make_plain_map(&q.tmY, y, uint64_t(N) * 2, uint64_t(M), 256, 128) ||
-        !make_kmajor_map(&q.tmX, xq, false, K, Mp, kBBoxRows) || !make_kmajor_map(&q.tmX2, xq, false, K, Mp, 128))
+        !make_kmajor_map(&q.tmX, xq, false, K, M, kBBoxRows) || !make_kmajor_map(&q.tmX2, xq, false, K, M, 128))
       return W8A8_ERR_UNSUPPORTED;
     q.num_kb = int(K / 128);
     q.n_cb = int(N / 128);
@@ -789,7 +812,7 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
   }
   if (M > kPairMinRows) {
     PairParams q{};
-    if (!make_kmajor_map(&q.tmA, wq, false, K, N, 128) || !make_pair_b_maps(&q, xq, K, Mp))
+    if (!make_kmajor_map(&q.tmA, wq, false, K, N, 128) || !make_pair_b_maps(&q, xq, K, M))
       return W8A8_ERR_UNSUPPORTED;
     q.num_kb = int(K / 128);
     q.n_cb = int((N + 255) / 256);
@@ -804,8 +827,8 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
     return launch_pair<kEpiDense>(q, int((M + kPairNB - 1) / kPairNB) * q.n_cb, s);
   }
   GemmParams p{};
-  if (!make_kmajor_map(&p.tmA, wq, false, K, N, 128) || !make_kmajor_map(&p.tmB, xq, false, K, Mp, kBBoxRows) ||
-      !make_kmajor_map(&p.tmB2, xq, false, K, Mp, 128))
+  if (!make_kmajor_map(&p.tmA, wq, false, K, N, 128) || !make_kmajor_map(&p.tmB, xq, false, K, M, kBBoxRows) ||
+      !make_kmajor_map(&p.tmB2, xq, false, K, M, 128))
     return W8A8_ERR_UNSUPPORTED;
   p.num_kb = int(K / 128);
   p.n_cb = int((N + 255) / 256);
@@ -821,6 +844,50 @@ int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_forma
   p.col_scale = sw;
   const int tiles = int((M + 127) / 128) * p.n_cb;
   return launch_gemm<2, 128, kEpiDense, kKindI8>(p, tiles, s);
+}
+
+// Host-side checks shared by the two dense-linear entry points (everything but the activations).
+int check_linear(const void* wq, const float* sw, int w_format, int group, int64_t M, int64_t K, int64_t N,
+                 const w8a8_bf16* y) {
+  if (M < 0 || K <= 0 || N <= 0) return W8A8_ERR_ARG;
+  if (w8a8_linear_workspace_size(M, K, N, w_format, group) == 0) return W8A8_ERR_UNSUPPORTED;
+  if (M == 0) return W8A8_OK;
+  if (!wq || !sw || !y) return W8A8_ERR_ARG;
+  if (!aligned16(wq) || !aligned16(y)) return W8A8_ERR_UNSUPPORTED;
+  if (w_format == W8A8_W_INT4_PER_GROUP && (K / 128) > (int64_t(1) << 20)) return W8A8_ERR_UNSUPPORTED;
+  if (M >= (int64_t(1) << 30) || N * K >= (int64_t(1) << 40)) return W8A8_ERR_UNSUPPORTED;
+  return W8A8_OK;
+}
+
+}  // namespace
+}  // namespace w8a8
+
+extern "C" {
+
+int w8a8_linear(const w8a8_bf16* x, const void* wq, const float* sw, int w_format, int group, int64_t M, int64_t K,
+                int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream) {
+  int rc = check_linear(wq, sw, w_format, group, M, K, N, y);
+  if (rc != W8A8_OK || M == 0) return rc;
+  const size_t need = w8a8_linear_workspace_size(M, K, N, w_format, group);
+  if (!x || !workspace) return W8A8_ERR_ARG;
+  if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return W8A8_ERR_UNSUPPORTED;
+  const int64_t Mp = round_up(M, 128);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(ws + align256(size_t(Mp) * K));
+  rc = w8a8_quant_act_per_token(x, M, K, xq, sx, stream);
+  if (rc != W8A8_OK) return rc;
+  return linear_gemm(xq, sx, wq, sw, w_format, M, K, N, y, as_stream(stream));
+}
+
+int w8a8_linear_prequant(const int8_t* xq, const float* sx, const void* wq, const float* sw, int w_format,
+                         int group, int64_t M, int64_t K, int64_t N, w8a8_bf16* y, w8a8_stream stream) {
+  const int rc = check_linear(wq, sw, w_format, group, M, K, N, y);
+  if (rc != W8A8_OK || M == 0) return rc;
+  if (!xq || !sx) return W8A8_ERR_ARG;
+  if (!aligned16(xq)) return W8A8_ERR_UNSUPPORTED;
+  return linear_gemm(xq, sx, wq, sw, w_format, M, K, N, y, as_stream(stream));
 }
 
 int w8a8_gemm_s8s8s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,

@@ -18,7 +18,8 @@ Recipe (the same for every workload):
   gate_proj, rows ``I..2I-1`` are up_proj, the packed layout of the AMCT Qwen3-Next case
   study, section 2.2) and ``down`` ``[E, H, I]``.
 * Skewed router: a bias of +2 on 8 experts drawn without replacement, 0 elsewhere.
-* Dense W4A8 linear: ``W ~ N(0, 0.02)`` with shape ``[N, K]``, activations as above.
+* Dense linears (W4A8 and W8A8): ``W ~ N(0, 0.02)`` with shape ``[N, K]``, activations as
+  above.
 """
 from __future__ import annotations
 
@@ -57,7 +58,8 @@ class MoEWorkload:
 
 @dataclass(frozen=True)
 class LinearWorkload:
-    """Dense linear workload: x [M, K] times W [N, K]^T, int4 weights in groups of ``group``."""
+    """Dense linear workload: x [M, K] times W [N, K]^T; weights int4 in groups of ``group``
+    along K (``fmt`` "int4") or int8 per output channel (``fmt`` "int8")."""
 
     name: str
     M: int
@@ -66,6 +68,7 @@ class LinearWorkload:
     group: int
     n_outlier: int
     seed: int = 0
+    fmt: str = "int4"
 
 
 MOE_WORKLOADS = {
@@ -82,8 +85,16 @@ MOE_WORKLOADS = {
 
 LINEAR_WORKLOADS = {
     w.name: w
-    for w in (LinearWorkload("qwen3-1.7b-mlp-w4a8", M=2048, K=2048, N=6144, group=128,
-                             n_outlier=20),)
+    for w in (
+        LinearWorkload("qwen3-1.7b-mlp-w4a8", M=2048, K=2048, N=6144, group=128, n_outlier=20),
+        # the same MLP shape with int8 per-channel weights, and the Qwen3-30B-A3B attention
+        # projections (hidden 2048, 32 query heads and 4 key/value heads of 128): q_proj
+        # 2048 -> 4096, k_proj / v_proj 2048 -> 512, o_proj 4096 -> 2048
+        LinearWorkload("qwen3-1.7b-mlp-w8a8", M=2048, K=2048, N=6144, group=0, n_outlier=20, fmt="int8"),
+        LinearWorkload("qwen3-30b-a3b-q-proj-w8a8", M=2048, K=2048, N=4096, group=0, n_outlier=20, fmt="int8"),
+        LinearWorkload("qwen3-30b-a3b-k-proj-w8a8", M=2048, K=2048, N=512, group=0, n_outlier=20, fmt="int8"),
+        LinearWorkload("qwen3-30b-a3b-o-proj-w8a8", M=2048, K=4096, N=2048, group=0, n_outlier=41, fmt="int8"),
+    )
 }
 
 
