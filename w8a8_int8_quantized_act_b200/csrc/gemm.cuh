@@ -71,16 +71,27 @@ struct GemmParams {
   int* tile_counts;            // expert histogram rows (nullptr: none); zeroed before the launch
   int tile_count_stride;       // elements between the rows of consecutive 128-token chunks (0: one row)
   int router_rows;             // router: tokens per tile (64 or 128; the A map's box height)
+  // down with the requantisation of h fused into the B operand (template QKB > 0): the bf16 rows
+  // of h [rows, K] the CTA quantises itself, and where the tiles of channel block 0 leave the
+  // codes and scales (hq [rows, K], s_h [rows])
+  const uint16_t* qb_h;
+  int8_t* qb_hq;
+  float* qb_s;
 };
 
-template <int NA, int NB, int EPI>
+// QKB > 0 (down GEMM of short token lists): the B operand of a tile is not loaded by TMA but made
+// by the CTA itself from bf16 h, QKB K-blocks at most, into one of two resident buffers.
+template <int NA, int NB, int EPI, int QKB = 0>
 struct GemmCfg {
   static constexpr int kABytes = kBM * kKBlockBytes;
   static constexpr int kBBytes = NB * kKBlockBytes;
-  static constexpr int kStageBytes = NA * kABytes + kBBytes;
+  static constexpr int kStageBytes = NA * kABytes + (QKB > 0 ? 0 : kBBytes);
   // router: logits of one tile transposed to [expert][token] (row pitch 129 floats, so both the
-  // per-token writes and the per-expert reads are free of bank conflicts)
-  static constexpr int kXBytes = (EPI == kEpiRouter) ? NB * 129 * 4 : 0;
+  // per-token writes and the per-expert reads are free of bank conflicts); resident B: two
+  // buffers of QKB 128-byte-swizzled K-blocks of NB rows, then their row scales
+  static constexpr int kQBBufBytes = QKB * NB * kKBlockBytes;
+  static constexpr int kXBytes = (EPI == kEpiRouter) ? NB * 129 * 4 : (QKB > 0 ? 2 * kQBBufBytes + 2 * NB * 4 : 0);
+  static_assert(QKB == 0 || (NB * kKBlockBytes) % 1024 == 0, "resident K-blocks sit on 1 KB boundaries");
   static constexpr int kStagesRaw = (196 * 1024 - kXBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   static constexpr int kAccCols = NA * NB;  // TMEM columns of one accumulator set
@@ -206,9 +217,11 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, uint32_t (
 // ---------------------------------------------------------------------------- epilogues
 // Expert GEMM epilogues: thread = one channel (TMEM lane), columns = the tile's token rows.
 // The two epilogue warps of a lane quarter take alternate 16-column chunks.
+// tile_scale (down with a resident B): the tile's row scales in shared memory, indexed by the
+// row's position in the tile; nullptr: p.row_scale in global memory, indexed by sorted row.
 template <int EPI, int NB>
 __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Tile& c, uint32_t t_lane, int lane_ch,
-                                                  int half) {
+                                                  int half, const float* tile_scale = nullptr) {
   const int ch = c.cb * p.a_cb_step + lane_ch;  // channel within the group
   const size_t ldo = size_t(p.ldo);
   const float* __restrict__ row_scale = p.row_scale;
@@ -268,7 +281,7 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
       int orow[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        srow[j] = (j < nj) ? __ldg(row_scale + row0 + j) : 0.0f;
+        srow[j] = (j < nj) ? (tile_scale != nullptr ? tile_scale[j0 + j] : __ldg(row_scale + row0 + j)) : 0.0f;
         orow[j] = (EPI == kEpiDown) ? ((j < nj) ? __ldg(row_map + row0 + j) : 0) : row0 + j;
       }
       tmem_ld16x2(t_lane + j0, t_lane + NB + j0, r, r1);
@@ -356,16 +369,20 @@ __device__ __forceinline__ void epilogue_router(const GemmParams& p, const Tile&
   xphase ^= 1u;
 }
 
-template <int NA, int NB, int EPI, int KIND>
+template <int NA, int NB, int EPI, int KIND, int QKB = 0>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
-  using Cfg = GemmCfg<NA, NB, EPI>;
+  using Cfg = GemmCfg<NA, NB, EPI, QKB>;
   constexpr int STAGES = Cfg::kStages;
   constexpr int KB_ELEMS = (KIND == kKindI8) ? 128 : 64;
   constexpr uint32_t IDESC0 = (KIND == kKindI8) ? idesc_s8s8s32(0) : idesc_bf16f32(0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes);
+  // QKB: the two resident B buffers (1 KB aligned after the stages) and their row scales [2][NB]
+  uint8_t* qb_buf = smem + STAGES * Cfg::kStageBytes;
+  float* qb_scale = reinterpret_cast<float*>(qb_buf + 2 * Cfg::kQBBufBytes);
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::kStageBytes + (QKB > 0 ? Cfg::kXBytes : 0));
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -376,6 +393,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   int* goff = mt_prefix + (kMaxGroups + 1);
   float* xs = reinterpret_cast<float*>(goff + (kMaxGroups + 1));  // router: [NB][129] logits
   uint64_t* xbar = drain + 1;  // router: all epilogue threads, two phases per tile
+  uint64_t* bready = drain + 2;  // QKB: resident B buffer [2] written (all epilogue threads)
+  uint64_t* bfree = drain + 4;   // QKB: resident B buffer [2] read by the tile's MMAs (commit)
+  uint64_t* ebar = drain + 6;    // QKB: all epilogue threads done with a tile's row scales
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -386,6 +406,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, kEpiWarps * 32); }
     mbar_init(drain, 1);
     mbar_init(xbar, 32 * kEpiWarps);
+    for (int b = 0; b < 2; ++b) { mbar_init(bready + b, 32 * kEpiWarps); mbar_init(bfree + b, 1); }
+    mbar_init(ebar, 32 * kEpiWarps);
     fence_mbar_init();
     *abort_flag = 0;
     mt_prefix[0] = 0;
@@ -440,7 +462,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
       const uint32_t a_bytes = (EPI == kEpiRouter) ? uint32_t(p.router_rows * kKBlockBytes) : uint32_t(Cfg::kABytes);
-      const uint32_t bytes = uint32_t(NA * a_bytes + c.nb * kKBlockBytes);
+      const uint32_t bytes = uint32_t(NA * a_bytes + (QKB > 0 ? 0 : c.nb * kKBlockBytes));
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
         if (elect_one()) {
@@ -450,11 +472,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
           tma_load_2d(st, &p.tmA, full + stage, x, c.a_row);
           if (NA == 2) tma_load_2d(st + Cfg::kABytes, &p.tmA, full + stage, x, c.a_row + p.a_second_offset);
           uint8_t* sb = st + NA * Cfg::kABytes;
-          if (c.nb == NB) {
-            tma_load_2d(sb, &p.tmB2, full + stage, x, c.b_row);
-          } else {
-            for (int b = 0; b < c.nb; b += kBBoxRows)
-              tma_load_2d(sb + b * kKBlockBytes, &p.tmB, full + stage, x, c.b_row + b);
+          if constexpr (QKB == 0) {
+            if (c.nb == NB) {
+              tma_load_2d(sb, &p.tmB2, full + stage, x, c.b_row);
+            } else {
+              for (int b = 0; b < c.nb; b += kBBoxRows)
+                tma_load_2d(sb + b * kKBlockBytes, &p.tmB, full + stage, x, c.b_row + b);
+            }
           }
         }
         __syncwarp();
@@ -477,16 +501,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     // start-address field, which cannot carry: shared memory ends below 256 KB); one elected
     // lane issues every MMA and commit.
     const uint64_t adesc0 = sw128_kmajor_desc(smem_addr(smem));
+    const uint64_t qdesc0 = sw128_kmajor_desc(smem_addr(qb_buf));
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int local_tile = 0;
     bool issued_any = false;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++local_tile) {
       const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
       const uint32_t idesc = IDESC0 | (uint32_t(c.nb >> 3) << 17);
+      const int qb = local_tile & 1;
       if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) break;
+      if constexpr (QKB > 0) {
+        // the tile's resident B (written by the epilogue warps, fenced for the async proxy)
+        if (!mbar_wait_warp(bready + qb, uint32_t(local_tile >> 1) & 1u, wc)) break;
+      }
       tc_fence_after();
       const uint32_t d0 = tmem_base + uint32_t(acc * Cfg::kAccCols);
       for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -494,7 +525,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         if (!mbar_wait_warp(full + stage, phase, wc)) { ok = false; break; }
         if (elect_one()) {
           const uint64_t ad = adesc0 + uint64_t(stage * (Cfg::kStageBytes >> 4));
-          const uint64_t bd = ad + uint64_t(NA * (Cfg::kABytes >> 4));
+          const uint64_t bd = (QKB > 0) ? qdesc0 + uint64_t((qb * Cfg::kQBBufBytes + kb * NB * kKBlockBytes) >> 4)
+                                        : ad + uint64_t(NA * (Cfg::kABytes >> 4));
 #pragma unroll
           for (int kk = 0; kk < kKBlockBytes / 32; ++kk) {
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
@@ -510,7 +542,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      if (elect_one()) tc_commit(tfull + acc);
+      if (elect_one()) {
+        tc_commit(tfull + acc);
+        if constexpr (QKB > 0) tc_commit(bfree + qb);  // the resident B may be rewritten
+      }
       __syncwarp();
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
@@ -531,19 +566,64 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t xphase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    // Resident B (QKB > 0): the epilogue warps quantise each tile's bf16 h rows into one of two
+    // shared-memory buffers, warp w taking rows w, w + 8, ...: the row maximum, the scale and the
+    // codes exactly as the per-row requantisation kernel computes them (quant_row_warp), written as
+    // 128-byte swizzled K-blocks; the tiles of channel block 0 also leave the codes and scales in
+    // global memory (hq, s_h). A tile's buffer is made two tiles ahead, once the MMAs of the tile
+    // that last used it have completed and every epilogue thread is done with its row scales.
+    auto make_b = [&](const Tile& t, int b) {
+      if constexpr (QKB > 0) {
+        const int K = p.num_kb * kKBlockBytes;
+        uint8_t* buf = qb_buf + b * Cfg::kQBBufBytes;
+        for (int r = warp - 2; r < t.rows; r += kEpiWarps) {
+          const float sc = quant_row_warp<QKB / 2>(p.qb_h + size_t(t.tok0 + r) * K, K, [&](int i, uint2 v) {
+            const int kb = i >> 7, ch16 = (i & 127) >> 4, hv = (i >> 3) & 1;
+            *reinterpret_cast<uint2*>(buf + kb * (NB * kKBlockBytes) + r * kKBlockBytes + ((ch16 ^ (r & 7)) << 4) +
+                                      hv * 8) = v;
+            if (t.cb == 0) *reinterpret_cast<uint2*>(p.qb_hq + size_t(t.tok0 + r) * K + i) = v;
+          });
+          if (lane == 0) {
+            qb_scale[b * NB + r] = sc;
+            if (t.cb == 0) p.qb_s[t.tok0 + r] = sc;
+          }
+        }
+        fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
+        mbar_arrive(bready + b);
+      }
+    };
+    if constexpr (QKB > 0) {
+      for (int i = 0; i < 2; ++i) {
+        const int tl = int(blockIdx.x) + i * int(gridDim.x);
+        if (tl < total_tiles) make_b(decode_tile<EPI, NB>(p, mt_prefix, goff, tl), i);
+      }
+    }
+    uint32_t ephase = 0;
+    int local_tile = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++local_tile) {
       const Tile c = decode_tile<EPI, NB>(p, mt_prefix, goff, tile);
       if (!mbar_wait(tfull + acc, acc_phase, wc)) break;
       tc_fence_after();
       const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * Cfg::kAccCols);
+      const int qb = local_tile & 1;
       if constexpr (EPI == kEpiRouter) {
         epilogue_router<NB>(p, c, t_lane, lane_idx, half, warp - 2, xs, xbar, xphase, wc);
       } else {
-        epilogue_channels<EPI, NB>(p, c, t_lane, lane_idx, half);
+        epilogue_channels<EPI, NB>(p, c, t_lane, lane_idx, half, QKB > 0 ? qb_scale + qb * NB : nullptr);
       }
       tc_fence_before();
       mbar_arrive(tempty + acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if constexpr (QKB > 0) {
+        const int t2 = tile + 2 * int(gridDim.x);
+        if (t2 < total_tiles) {
+          mbar_arrive(ebar);  // every epilogue thread is done with this tile's row scales
+          if (!mbar_wait(ebar, ephase, wc)) break;
+          ephase ^= 1u;
+          if (!mbar_wait(bfree + qb, uint32_t(local_tile >> 1) & 1u, wc)) break;
+          make_b(decode_tile<EPI, NB>(p, mt_prefix, goff, t2), qb);
+        }
+      }
     }
   }
 

@@ -141,9 +141,6 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   return uint64_t(__float_as_uint(lo)) | (uint64_t(__float_as_uint(hi)) << 32);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 template <int NB, int CV, int EW>
 __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)

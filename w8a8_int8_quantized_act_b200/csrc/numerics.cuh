@@ -156,23 +156,31 @@ __device__ __forceinline__ float dequant(int32_t acc, float s_row, float s_col) 
 // value takes the true divide for all eight. A row whose amax is below about 2^-121 has a
 // subnormal scale whose reciprocal overflows to +inf: y is then +-inf or NaN, d is NaN, and the
 // test is written so that NaN also counts as unsure and takes the true divide.
+// The products and sums run two values at a time (packed f32x2 operations, each lane rounded to
+// nearest like the scalar operation, subnormals kept).
 __device__ __forceinline__ uint2 quant8(const uint4 v, float s, float inv) {
   if (s == 0.0f) return make_uint2(0u, 0u);
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t inv2 = (uint64_t(__float_as_uint(inv)) << 32) | __float_as_uint(inv);
+  const uint64_t mag2 = (uint64_t(0x4B400000u) << 32) | 0x4B400000u;  // 1.5 * 2^23 in both halves
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   uint32_t c[8];
   bool unsure = false;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const float x = h ? bf16_hi(w[j]) : bf16_lo(w[j]);
-      const float y = __fmul_rn(x, inv);
-      const float r = __fadd_rn(y, kMagic);
-      const float d = __fsub_rn(y, __fsub_rn(r, kMagic));
-      unsure |= !(fabsf(d) < 0.49997f);
-      c[2 * j + h] = __float_as_uint(r);
-    }
+    uint32_t r0, r1, d0, d1;
+    asm("{\n\t.reg .b64 x, y, r, t, d;\n\t"
+        "mov.b64 x, {%4, %5};\n\t"
+        "mul.rn.f32x2 y, x, %6;\n\t"
+        "add.rn.f32x2 r, y, %7;\n\t"
+        "sub.rn.f32x2 t, r, %7;\n\t"
+        "sub.rn.f32x2 d, y, t;\n\t"
+        "mov.b64 {%0, %1}, r;\n\t"
+        "mov.b64 {%2, %3}, d;\n\t}"
+        : "=r"(r0), "=r"(r1), "=r"(d0), "=r"(d1)
+        : "r"(w[j] << 16), "r"(w[j] & 0xFFFF0000u), "l"(inv2), "l"(mag2));
+    unsure |= !(fabsf(__uint_as_float(d0)) < 0.49997f) || !(fabsf(__uint_as_float(d1)) < 0.49997f);
+    c[2 * j] = r0;
+    c[2 * j + 1] = r1;
   }
   if (unsure) {
 #pragma unroll

@@ -125,10 +125,10 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaS
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? W8A8_OK : W8A8_ERR_LAUNCH;
 }
 
-template <int NA, int NB, int EPI, int KIND>
+template <int NA, int NB, int EPI, int KIND, int QKB = 0>
 int launch_gemm(const GemmParams& p, int max_tiles, cudaStream_t stream) {
-  using Cfg = GemmCfg<NA, NB, EPI>;
-  auto kern = gemm_tc_kernel<NA, NB, EPI, KIND>;
+  using Cfg = GemmCfg<NA, NB, EPI, QKB>;
+  auto kern = gemm_tc_kernel<NA, NB, EPI, KIND, QKB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cfg::kSmemBytes)) !=
       cudaSuccess)
     return W8A8_ERR_LAUNCH;
@@ -195,6 +195,10 @@ int check_moe_shape(int64_t T, int64_t H, int64_t E, int k, int64_t I) {
   if (E * 2 * I >= (int64_t(1) << 31) || E * H >= (int64_t(1) << 31)) return W8A8_ERR_UNSUPPORTED;
   return W8A8_OK;
 }
+
+// Token block of the expert GEMMs: 32 rows when experts see few tokens (decode), else 256 on
+// CTA pairs.
+bool small_token_blocks(int64_t A, int64_t E) { return A <= 32 * E; }
 
 void fill_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_layout* L) {
   const int64_t A = T * k;
@@ -387,9 +391,6 @@ int max_token_blocks(int64_t A, int64_t E, int nb) { return int((A + nb - 1) / n
 // Dense GEMMs with more token rows than this run on CTA pairs.
 constexpr int64_t kPairMinRows = 128;
 
-// Token block of the expert GEMMs: 32 rows when experts see few tokens (decode), else 256 on
-// CTA pairs.
-bool small_token_blocks(int64_t A, int64_t E) { return A <= 32 * E; }
 
 // CTAs per 128-token chunk of the grouping kernel (each re-derives the chunk's positions and
 // quantises every 8th token of the chunk).
@@ -536,6 +537,9 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   const int C = int((T + kChunk - 1) / kChunk);
   int rc;
 
+  // Few rows per expert (decode): the expert GEMMs run one CTA per tile of <= 32 sorted rows;
+  // otherwise CTA pairs on tiles of <= 256 rows.
+  const bool small = small_token_blocks(A, E);
   if (T <= kFrontMaxT && H <= kFrontMaxH) {
     // 1+2. short batch: routing, grouping and quantisation in one cooperative launch
     mark(ev, 0, s);
@@ -561,9 +565,7 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   }
 
   // 3. grouped gate_up GEMM (weights on M, tokens on N) with the dequant + SiLU(gate)*up
-  //    epilogue -> h. Few rows per expert (decode): one CTA per tile of <= 32 rows; otherwise
-  //    CTA pairs on tiles of <= 256 rows.
-  const bool small = small_token_blocks(A, E);
+  //    epilogue -> h
   if (small) {
     GemmParams p{};
     if (!make_kmajor_map(&p.tmA, wgu, false, H, uint64_t(E) * 2 * I, 128) ||
@@ -608,11 +610,12 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     if ((rc = launch_pair<kEpiGateUp>(p, tiles, s)) != W8A8_OK) return rc;
   }
 
-  // 4. per-row requantisation of h
-  {
-    mark(ev, 3, s);
-    if ((rc = launch_quant_rows(h, A, int(I), hq, s_h, s)) != W8A8_OK) return rc;
-  }
+  // 4. per-row requantisation of h: inside the down GEMM for short token lists with rows of up
+  //    to 1024 values (each CTA quantises its tile's rows into shared memory), else a launch of
+  //    its own
+  const bool rq_in_down = small && I <= 1024;
+  mark(ev, 3, s);
+  if (!rq_in_down && (rc = launch_quant_rows(h, A, int(I), hq, s_h, s)) != W8A8_OK) return rc;
 
   // 5. grouped down GEMM with the dequant epilogue -> o in slot order
   if (small) {
@@ -637,7 +640,15 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     p.row_map = perm;
     const int tiles = max_token_blocks(A, E, 32) * p.n_cb;
     mark(ev, 4, s);
-    if ((rc = launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s)) != W8A8_OK) return rc;
+    if (rq_in_down) {
+      p.qb_h = h;
+      p.qb_hq = hq;
+      p.qb_s = s_h;
+      rc = launch_gemm<2, 32, kEpiDown, kKindI8, 8>(p, tiles, s);
+    } else {
+      rc = launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s);
+    }
+    if (rc != W8A8_OK) return rc;
   } else {
     PairParams p{};
     if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(E) * H, 128) || !make_pair_b_maps(&p, hq, I, Ap))
