@@ -44,6 +44,13 @@ Readings where the pages are silent (each one is fixed identically on the GPU si
   K-groups g in order.
 * fma(a, b, c) is the fp32 fused multiply-add: a*b + c rounded once. numpy has none, so
   ``fma32`` computes it exactly from float64 arithmetic (see there).
+* Shared expert (the Qwen3-Next / Qwen3.6 layers): the shared expert is a dense gated MLP
+  quantised W8A8 like the routed experts (the AMCT Qwen3-Next page, section 二 2.2: the shared
+  expert is a dense activated path, quantised directly); its gate ``shared_expert_gate`` is a
+  bf16 Linear [H] -> 1 kept out of quantisation (the ignore list of the Qwen3.6-35B-A3B recipe).
+  The pages do not give the combination: it is read as y = routed + sigmoid(x . w_sg) * shared,
+  the shared output entering the combine's fma chain after the k routed slots with weight
+  g = sigmoid(z), z the gate logit (float64 here), sigmoid(z) = 1 / (1 + exp(-z)).
 """
 from __future__ import annotations
 
@@ -321,6 +328,21 @@ def combine_acc(o_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
     return acc
 
 
+def combine_acc_with_shared(o_bits: np.ndarray, w: np.ndarray, o_shared_bits: np.ndarray, g: np.ndarray
+                            ) -> np.ndarray:
+    """The combine's fp32 accumulator extended by the shared expert: acc over the k routed slots
+    as in ``combine_acc``, then acc = fma(g[t], o_shared[t], acc), one rounding."""
+    acc = combine_acc(o_bits, w)
+    o_s = bf16_to_f32(o_shared_bits)
+    g = np.asarray(g, np.float32)
+    return fma32(np.broadcast_to(g[:, None], o_s.shape), o_s, acc)
+
+
+def combine_with_shared(o_bits: np.ndarray, w: np.ndarray, o_shared_bits: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """y[t] = bf16(``combine_acc_with_shared``)."""
+    return f32_to_bf16(combine_acc_with_shared(o_bits, w, o_shared_bits, g))
+
+
 def combine(o_bits: np.ndarray, w: np.ndarray) -> np.ndarray:
     """y[t] = bf16(sum_j w[t, j] * o[t, j]): the fma chain of ``combine_acc``, rounded to bf16.
 
@@ -398,6 +420,39 @@ def moe_forward(x_bits, wg_bits, bias, wgu_q, s_gu, wd_q, s_d, k: int, renorm: b
         out.update(h=h.reshape(T, k, I), hq=hq.reshape(T, k, I), s_h=s_h.reshape(T, k))
     if r is not None:
         out["routing"] = r
+    return out
+
+
+def shared_gate(x_bits, wsg_bits) -> np.ndarray:
+    """g[t] = sigmoid(x[t] . w_sg) in float64: the bf16 shared_expert_gate, never quantised
+    (ignore list of the Qwen3.6-35B-A3B recipe)."""
+    z = bf16_to_f32(x_bits).astype(np.float64) @ bf16_to_f32(wsg_bits).astype(np.float64).reshape(-1)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def shared_expert(x_bits, wgu_q, s_gu, wd_q, s_d) -> dict:
+    """The shared expert as a dense W8A8 gated MLP (every token): per-token int8 x, int32 GEMM
+    with the packed gate|up weight, dequant, SiLU(gate) * up -> bf16 h, per-row requantisation,
+    int32 GEMM with the down weight, dequant -> bf16 o. The same arithmetic as one routed expert
+    that every token selects."""
+    xq, sx = quant_act_per_token(np.asarray(x_bits, np.uint16))
+    h = gated_activation(int_gemm(xq, wgu_q), sx, s_gu)
+    hq, s_h = symmetric_quantize_rows(bf16_to_f32(h), Q_MAX_INT8)
+    o = f32_to_bf16(dequant(int_gemm(hq, wd_q), s_h, s_d))
+    return dict(xq=xq, sx=sx, h=h, hq=hq, s_h=s_h, o=o)
+
+
+def moe_forward_shared(x_bits, wg_bits, bias, wgu_q, s_gu, wd_q, s_d, k: int, wsg_bits, sh_gu_q, sh_s_gu, sh_d_q,
+                       sh_s_d, renorm: bool = True, routing: tuple | None = None, gate: np.ndarray | None = None
+                       ) -> dict:
+    """MoE layer with a shared expert: the routed forward of ``moe_forward``, the shared expert on
+    every token, and y = bf16(fma(g, o_shared, routed fma chain)). ``gate`` replaces the oracle's
+    own float64 sigmoid gate (the GPU's fp32 gate can be fed in, like the routing)."""
+    out = moe_forward(x_bits, wg_bits, bias, wgu_q, s_gu, wd_q, s_d, k, renorm, routing)
+    sh = shared_expert(x_bits, sh_gu_q, sh_s_gu, sh_d_q, sh_s_d)
+    g64 = shared_gate(x_bits, wsg_bits)
+    g = np.asarray(g64 if gate is None else gate, np.float32)
+    out.update(shared=sh, gate=g64, y=combine_with_shared(out["o"], out["weights"], sh["o"], g))
     return out
 
 
