@@ -161,6 +161,47 @@ int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
                      int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
                      w8a8_stream stream);
 
+/* Workspace of w8a8_moe_forward_shared: the routed layer's regions (as w8a8_moe_ws_layout gives
+ * them for the same T, H, E, k, I) followed by the shared expert's (every region 256-byte aligned):
+ *   xq int8 [T, H] and sx fp32 [T] (per-token codes and scales of x, token order);
+ *   h bf16 [T, Is] (SiLU(gate) * up); s_h fp32 [T]; hq int8 [T, Is]; o bf16 [T, H];
+ *   gate fp32 [T] (sigmoid of the shared_expert_gate logit). */
+typedef struct {
+  w8a8_moe_ws_layout routed;
+  size_t xq, sx, h, s_h, hq, o, gate;
+  size_t total;
+} w8a8_moe_shared_ws_layout;
+
+/* Fills *layout for the shape (Is: the shared expert's intermediate size, a multiple of 128).
+ * Returns W8A8_ERR_ARG / W8A8_ERR_UNSUPPORTED on bad shapes. */
+int w8a8_moe_shared_workspace_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, int64_t Is,
+                                     w8a8_moe_shared_ws_layout* layout);
+
+/* Workspace bytes w8a8_moe_forward_shared needs for this shape (0 if the shape is rejected). */
+size_t w8a8_moe_shared_workspace_size(int64_t T, int64_t H, int64_t E, int k, int64_t I, int64_t Is);
+
+/* Defined by: "Qwen3-Next-80B-A3B-Instruct 在 AMCT 中的 MoE 混合注意力量化适配实战", section 二 2.2
+ * (the shared expert is a dense path, quantised W8A8 directly, next to the packed routed experts);
+ * the ignore list of the Qwen3.6-35B-A3B-w8a8 recipe (shared_expert_gate stays bf16). The pages
+ * do not give how the two paths combine; the library reads it as y = routed + sigmoid(x . w_sg) *
+ * shared.
+ * MoE layer with a shared expert: the routed forward of w8a8_moe_forward, plus on every token
+ *   g = sigmoid(x . w_sg) (bf16 inputs, fp32 sum, fp32 sigmoid), the shared expert as a dense W8A8
+ *   gated MLP (per-token int8 x, int8 gate_up, dequant, SiLU(gate) * up -> bf16 h, per-row int8
+ *   requantisation, int8 down, dequant -> bf16 o_s), and
+ *   y[t] = bf16(fma(g[t], o_s[t], acc_t)), acc_t the fp32 accumulator of the routed combine.
+ *   wsg    bf16 [H]        shared_expert_gate (nn.Linear H -> 1)
+ *   wgu_s  int8 [2Is, H]   packed gate|up of the shared expert; s_gu_s fp32 [2Is]
+ *   wd_s   int8 [H, Is];   s_d_s fp32 [H]
+ *   workspace  at least w8a8_moe_shared_workspace_size() bytes, 256-byte aligned; it keeps the
+ *              intermediates listed in w8a8_moe_shared_ws_layout after the call.
+ * The other arguments and rules are those of w8a8_moe_forward; Is % 128 == 0. */
+int w8a8_moe_forward_shared(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                            const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E,
+                            int k, int64_t I, int renorm, const w8a8_bf16* wsg, const int8_t* wgu_s,
+                            const float* s_gu_s, const int8_t* wd_s, const float* s_d_s, int64_t Is, void* workspace,
+                            size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream);
+
 /* w8a8_moe_forward that also records caller-created CUDA events (cudaEvent_t, may be NULL
  * entries) on `stream` at the stage boundaries, for per-kernel timing:
  *   [0] before the router, [1] before grouping + quantisation, [2] before the gate_up GEMM,

@@ -42,6 +42,11 @@ class _Layout(ctypes.Structure):
                  "s_h", "hq", "o", "logits", "sync", "total")]
 
 
+class _SharedLayout(ctypes.Structure):
+    _fields_ = [("routed", _Layout)] + [(n, ctypes.c_size_t) for n in
+                                        ("xq", "sx", "h", "s_h", "hq", "o", "gate", "total")]
+
+
 # (name, restype, argtypes) of every exported entry point
 SIGNATURES = {
     "w8a8_version": (_int, []),
@@ -59,6 +64,10 @@ SIGNATURES = {
                                          _int, _c_p, _size, _c_p, _c_p, ctypes.POINTER(_c_p)]),
     "w8a8_moe_forward_noalloc": (_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _i64,
                                         _int, _c_p, _c_p]),
+    "w8a8_moe_shared_workspace_layout": (_int, [_i64, _i64, _i64, _int, _i64, _i64, ctypes.POINTER(_SharedLayout)]),
+    "w8a8_moe_shared_workspace_size": (_size, [_i64, _i64, _i64, _int, _i64, _i64]),
+    "w8a8_moe_forward_shared": (_int, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _i64, _int,
+                                       _c_p, _c_p, _c_p, _c_p, _c_p, _i64, _c_p, _size, _c_p, _c_p]),
     "w8a8_linear_workspace_size": (_size, [_i64, _i64, _i64, _int, _int]),
     "w8a8_linear": (_int, [_c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _size, _c_p, _c_p]),
     "w8a8_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _c_p]),
@@ -207,6 +216,58 @@ def w8a8_moe_forward(x, wg, wgu, s_gu, wd, s_d, k: int, renorm: bool = True, bia
                                   T, H, E, k, I, int(renorm), _ptr(workspace), workspace.numel(), _ptr(y),
                                   _stream(stream)), "w8a8_moe_forward")
     return y
+
+
+def w8a8_moe_shared_workspace_layout(T: int, H: int, E: int, k: int, I: int, Is: int) -> dict:
+    L = _SharedLayout()
+    _check(lib().w8a8_moe_shared_workspace_layout(T, H, E, k, I, Is, ctypes.byref(L)),
+           "w8a8_moe_shared_workspace_layout")
+    out = {name: getattr(L, name) for name, _ in _SharedLayout._fields_ if name != "routed"}
+    out["routed"] = {name: getattr(L.routed, name) for name, _ in _Layout._fields_}
+    return out
+
+
+def w8a8_moe_shared_workspace_size(T: int, H: int, E: int, k: int, I: int, Is: int) -> int:
+    return lib().w8a8_moe_shared_workspace_size(T, H, E, k, I, Is)
+
+
+def w8a8_moe_forward_shared(x, wg, wgu, s_gu, wd, s_d, k: int, wsg, wgu_s, s_gu_s, wd_s, s_d_s, renorm: bool = True,
+                            bias=None, workspace=None, y=None, stream=None):
+    """MoE layer with a shared expert; returns y bf16 [T, H] (workspace keeps the intermediates)."""
+    _bf16(x), _bf16(wg), _bf16(wsg)
+    T, H = x.shape
+    E, twoI, _ = wgu.shape
+    I = twoI // 2
+    Is = wgu_s.shape[0] // 2
+    ws_bytes = w8a8_moe_shared_workspace_size(T, H, E, k, I, Is)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(lib().w8a8_moe_forward_shared(_ptr(x), _ptr(wg), _ptr(bias), _ptr(wgu), _ptr(s_gu), _ptr(wd), _ptr(s_d),
+                                         T, H, E, k, I, int(renorm), _ptr(wsg), _ptr(wgu_s), _ptr(s_gu_s), _ptr(wd_s),
+                                         _ptr(s_d_s), Is, _ptr(workspace), workspace.numel(), _ptr(y),
+                                         _stream(stream)), "w8a8_moe_forward_shared")
+    return y
+
+
+def moe_shared_intermediates(workspace: torch.Tensor, T: int, H: int, E: int, k: int, I: int, Is: int) -> dict:
+    """Views of the intermediates w8a8_moe_forward_shared leaves in its workspace: the routed ones
+    (as moe_intermediates) and the shared expert's under the key "shared"."""
+    L = w8a8_moe_shared_workspace_layout(T, H, E, k, I, Is)
+
+    def view(name, dtype, shape):
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return workspace[L[name]:L[name] + nbytes].view(dtype).view(*shape)
+
+    out = moe_intermediates(workspace, T, H, E, k, I)
+    out["shared"] = dict(xq=view("xq", torch.int8, (T, H)), sx=view("sx", torch.float32, (T,)),
+                         h=view("h", torch.bfloat16, (T, Is)), s_h=view("s_h", torch.float32, (T,)),
+                         hq=view("hq", torch.int8, (T, Is)), o=view("o", torch.bfloat16, (T, H)),
+                         gate=view("gate", torch.float32, (T,)))
+    return out
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

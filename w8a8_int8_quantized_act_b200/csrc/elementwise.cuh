@@ -162,9 +162,13 @@ __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
 }
 
 // y[t, :] = bf16(sum_j w[t, j] * o[t, j, :]): fp32 fused multiply-adds in slot order from 0.
+// With a shared expert (o_shared != nullptr) one more fused multiply-add follows the k slots:
+// acc = fma(g[t], o_shared[t, :], acc).
 // One CTA per token, 8 columns per thread, no atomics: every y element has one writer.
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ o, const float* __restrict__ w,
-                                                      int T, int H, int k, uint16_t* __restrict__ y) {
+                                                      int T, int H, int k, uint16_t* __restrict__ y,
+                                                      const uint16_t* __restrict__ o_shared,
+                                                      const float* __restrict__ g) {
   pdl_wait();
   pdl_launch_dependents();
   const int t = blockIdx.x;
@@ -183,6 +187,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
         acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(u[i]), acc[2 * i + 1]);
       }
     }
+    if (o_shared != nullptr) {
+      const float gt = __ldg(g + t);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(o_shared + size_t(t) * H + c));
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fmaf_rn(gt, bf16_lo(u[i]), acc[2 * i]);
+        acc[2 * i + 1] = __fmaf_rn(gt, bf16_hi(u[i]), acc[2 * i + 1]);
+      }
+    }
     uint4 out;
     out.x = pack_bf16(acc[0], acc[1]);
     out.y = pack_bf16(acc[2], acc[3]);
@@ -190,6 +204,34 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
     out.w = pack_bf16(acc[6], acc[7]);
     *reinterpret_cast<uint4*>(y + size_t(t) * H + c) = out;
   }
+}
+
+// Gate of the shared expert (bf16 shared_expert_gate, never quantised): g[t] = sigmoid(z),
+// z = sum_h x[t, h] * w_sg[h] in fp32 (bf16 inputs; each lane fma-accumulates its 8-value vectors,
+// then a warp butterfly sum), sigmoid(z) = 1 / (1 + exp(-z)) with the layer's exponential and a
+// true divide. One warp per token; H a multiple of 8.
+__global__ void __launch_bounds__(kRowWarps * 32) shared_gate_kernel(const uint16_t* __restrict__ x,
+                                                                     const uint16_t* __restrict__ wsg, int T, int H,
+                                                                     float* __restrict__ g) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int t = int(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  float z = 0.0f;
+  for (int i = lane * 8; i < H; i += 256) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * H + i));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(wsg + i));
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      z = __fmaf_rn(bf16_lo(av[j]), bf16_lo(bv[j]), z);
+      z = __fmaf_rn(bf16_hi(av[j]), bf16_hi(bv[j]), z);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, o));
+  if (lane == 0) g[t] = __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_cw(-z)));
 }
 
 // Largest distance, in units in the last place, between rcp.approx.ftz.f32(d) and the correctly

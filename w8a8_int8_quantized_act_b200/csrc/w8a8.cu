@@ -227,6 +227,25 @@ void fill_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, w8a8_moe_ws_
   L->total = off;
 }
 
+// Shared-expert regions after the routed layer's (the routed offsets are those of fill_layout).
+void fill_shared_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, int64_t Is, w8a8_moe_shared_ws_layout* L) {
+  fill_layout(T, H, E, k, I, &L->routed);
+  size_t off = L->routed.total;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L->xq = take(size_t(T) * H);
+  L->sx = take(sizeof(float) * T);
+  L->h = take(size_t(T) * Is * 2);
+  L->s_h = take(sizeof(float) * T);
+  L->hq = take(size_t(T) * Is);
+  L->o = take(size_t(T) * H * 2);
+  L->gate = take(sizeof(float) * T);
+  L->total = off;
+}
+
 // Router: tcgen05 bf16 GEMM with the softmax / top-k epilogue. tile_counts is zeroed here.
 // counts: expert histogram rows (nullptr: none) with `count_stride` elements between the rows of
 // consecutive 128-token tiles (0: every tile adds into one row of E counters).
@@ -504,20 +523,83 @@ inline void mark(void* const* events, int i, cudaStream_t s) {
   if (events != nullptr && events[i] != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
 }
 
+int linear_gemm(const int8_t* xq, const float* sx, const void* wq, const float* sw, int w_format, int64_t M,
+                int64_t K, int64_t N, w8a8_bf16* y, cudaStream_t s);
+
+// The shared expert of a layer (bf16 gate [H], packed int8 gate_up [2Is, H] with its scales,
+// int8 down [H, Is] with its scales).
+struct SharedExpert {
+  const w8a8_bf16* wsg;
+  const int8_t* wgu;
+  const float* s_gu;
+  const int8_t* wd;
+  const float* s_d;
+  int64_t Is;
+};
+
+// Dense gate_up GEMM of every token (one group of T rows in token order) with the dequant +
+// SiLU(gate)*up epilogue: h [T, Is] from xq [T, H], sx [T] and the packed weight [2Is, H].
+int dense_gate_up(const int8_t* xq, const float* sx, const int8_t* wgu, const float* s_gu, int64_t T, int64_t H,
+                  int64_t Is, uint16_t* h, cudaStream_t s) {
+  if (T > kPairMinRows) {
+    PairParams p{};
+    if (!make_gate_up_pair_map(&p.tmA, wgu, H, Is, 1) || !make_pair_b_maps(&p, xq, H, T)) return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(H / 128);
+    p.n_cb = int(Is / 128);
+    p.num_groups = 1;
+    p.M = int(T);
+    p.a_rows_per_group = int(2 * Is);
+    p.n_channels = int(Is);
+    p.timeout_ns = wait_timeout_ns();
+    p.out = h;
+    p.ldo = int(Is);
+    p.row_scale = sx;
+    p.col_scale = s_gu;
+    p.col_scale_stride = int(2 * Is);
+    p.up_offset = int(Is);
+    return launch_pair<kEpiGateUp>(p, int((T + kPairNB - 1) / kPairNB) * p.n_cb, s);
+  }
+  GemmParams p{};
+  if (!make_kmajor_map(&p.tmA, wgu, false, H, uint64_t(2 * Is), 128) ||
+      !make_kmajor_map(&p.tmB, xq, false, H, T, kBBoxRows) || !make_kmajor_map(&p.tmB2, xq, false, H, T, 32))
+    return W8A8_ERR_UNSUPPORTED;
+  p.num_kb = int(H / 128);
+  p.n_cb = int(Is / 128);
+  p.num_groups = 1;
+  p.M = int(T);
+  p.a_rows_per_group = int(2 * Is);
+  p.a_second_offset = int(Is);
+  p.a_cb_step = 128;
+  p.timeout_ns = wait_timeout_ns();
+  p.out = h;
+  p.ldo = int(Is);
+  p.row_scale = sx;
+  p.col_scale = s_gu;
+  p.col_scale_stride = int(2 * Is);
+  p.up_offset = int(Is);
+  return launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, int((T + 31) / 32) * p.n_cb, s);
+}
+
 int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
                      const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E, int k,
                      int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
-                     w8a8_stream stream, void* const* ev) {
+                     w8a8_stream stream, void* const* ev, const SharedExpert* sh = nullptr) {
   const int st = check_moe_shape(T, H, E, k, I);
   if (st != W8A8_OK) return st;
+  if (sh != nullptr && (sh->Is <= 0 || sh->Is % 128 || 2 * sh->Is * H >= (int64_t(1) << 31)))
+    return sh->Is <= 0 ? W8A8_ERR_ARG : W8A8_ERR_UNSUPPORTED;
   if (T == 0) return W8A8_OK;
   if (!x || !wg || !wgu || !s_gu || !wd || !s_d || !workspace || !y) return W8A8_ERR_ARG;
+  if (sh != nullptr && (!sh->wsg || !sh->wgu || !sh->s_gu || !sh->wd || !sh->s_d)) return W8A8_ERR_ARG;
   if (!aligned16(x) || !aligned16(wg) || !aligned16(wgu) || !aligned16(wd) || !aligned16(y) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return W8A8_ERR_UNSUPPORTED;
-  w8a8_moe_ws_layout L;
-  fill_layout(T, H, E, k, I, &L);
-  if (workspace_bytes < L.total) return W8A8_ERR_WORKSPACE;
+  if (sh != nullptr && (!aligned16(sh->wsg) || !aligned16(sh->wgu) || !aligned16(sh->wd))) return W8A8_ERR_UNSUPPORTED;
+  w8a8_moe_shared_ws_layout SL;
+  if (sh != nullptr) fill_shared_layout(T, H, E, k, I, sh->Is, &SL);
+  else fill_layout(T, H, E, k, I, &SL.routed);
+  const w8a8_moe_ws_layout& L = SL.routed;
+  if (workspace_bytes < (sh != nullptr ? SL.total : L.total)) return W8A8_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* ids = reinterpret_cast<int*>(ws + L.topk_ids);
   float* w = reinterpret_cast<float*>(ws + L.topk_w);
@@ -671,9 +753,32 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
     if ((rc = launch_pair<kEpiDown>(p, tiles, s)) != W8A8_OK) return rc;
   }
 
-  // 6. scatter-free weighted combine
+  // 5b. the shared expert (every token): its bf16 gate, per-token int8 x, the dense gate_up GEMM
+  //     with the SiLU*up epilogue, the requantisation of its h, the dense down GEMM
+  uint16_t* o_sh = nullptr;
+  float* gate = nullptr;
+  if (sh != nullptr) {
+    int8_t* sxq = reinterpret_cast<int8_t*>(ws + SL.xq);
+    float* ssx = reinterpret_cast<float*>(ws + SL.sx);
+    uint16_t* sh_h = reinterpret_cast<uint16_t*>(ws + SL.h);
+    float* sh_sh = reinterpret_cast<float*>(ws + SL.s_h);
+    int8_t* sh_hq = reinterpret_cast<int8_t*>(ws + SL.hq);
+    o_sh = reinterpret_cast<uint16_t*>(ws + SL.o);
+    gate = reinterpret_cast<float*>(ws + SL.gate);
+    if ((rc = launch_pdl(shared_gate_kernel, dim3(unsigned((T + kRowWarps - 1) / kRowWarps)), dim3(kRowWarps * 32), 0,
+                         s, x, sh->wsg, int(T), int(H), gate)) != W8A8_OK)
+      return rc;
+    if ((rc = launch_quant_rows(x, T, int(H), sxq, ssx, s)) != W8A8_OK) return rc;
+    if ((rc = dense_gate_up(sxq, ssx, sh->wgu, sh->s_gu, T, H, sh->Is, sh_h, s)) != W8A8_OK) return rc;
+    if ((rc = launch_quant_rows(sh_h, T, int(sh->Is), sh_hq, sh_sh, s)) != W8A8_OK) return rc;
+    if ((rc = linear_gemm(sh_hq, sh_sh, sh->wd, sh->s_d, W8A8_W_INT8_PER_CHANNEL, T, sh->Is, H, o_sh, s)) != W8A8_OK)
+      return rc;
+  }
+
+  // 6. scatter-free weighted combine (and the gated shared expert after the k slots)
   mark(ev, 5, s);
-  rc = launch_pdl(combine_kernel, dim3(unsigned(T)), dim3(256), 0, s, o, w, int(T), int(H), k, y);
+  rc = launch_pdl(combine_kernel, dim3(unsigned(T)), dim3(256), 0, s, o, w, int(T), int(H), k, y,
+                  static_cast<const uint16_t*>(o_sh), static_cast<const float*>(gate));
   mark(ev, 6, s);
   return rc;
 }
@@ -682,6 +787,32 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
 }  // namespace w8a8
 
 extern "C" {
+
+int w8a8_moe_shared_workspace_layout(int64_t T, int64_t H, int64_t E, int k, int64_t I, int64_t Is,
+                                     w8a8_moe_shared_ws_layout* layout) {
+  if (!layout) return W8A8_ERR_ARG;
+  const int st = check_moe_shape(T, H, E, k, I);
+  if (st != W8A8_OK) return st;
+  if (Is <= 0) return W8A8_ERR_ARG;
+  if (Is % 128 || 2 * Is * H >= (int64_t(1) << 31)) return W8A8_ERR_UNSUPPORTED;
+  fill_shared_layout(T, H, E, k, I, Is, layout);
+  return W8A8_OK;
+}
+
+size_t w8a8_moe_shared_workspace_size(int64_t T, int64_t H, int64_t E, int k, int64_t I, int64_t Is) {
+  w8a8_moe_shared_ws_layout L;
+  return w8a8_moe_shared_workspace_layout(T, H, E, k, I, Is, &L) == W8A8_OK ? L.total : 0;
+}
+
+int w8a8_moe_forward_shared(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
+                            const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E,
+                            int k, int64_t I, int renorm, const w8a8_bf16* wsg, const int8_t* wgu_s,
+                            const float* s_gu_s, const int8_t* wd_s, const float* s_d_s, int64_t Is, void* workspace,
+                            size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream) {
+  const SharedExpert sh{wsg, wgu_s, s_gu_s, wd_s, s_d_s, Is};
+  return moe_forward_impl(x, wg, bias, wgu, s_gu, wd, s_d, T, H, E, k, I, renorm, workspace, workspace_bytes, y,
+                          stream, nullptr, &sh);
+}
 
 int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
                      const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E, int k,

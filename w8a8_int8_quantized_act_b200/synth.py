@@ -20,6 +20,8 @@ Recipe (the same for every workload):
 * Skewed router: a bias of +2 on 8 experts drawn without replacement, 0 elsewhere.
 * Dense linears (W4A8 and W8A8): ``W ~ N(0, 0.02)`` with shape ``[N, K]``, activations as
   above.
+* Shared expert: gate ``w_sg [H]``, packed gate|up ``[2Is, H]`` and down ``[H, Is]``, all
+  ``N(0, 0.02)``.
 """
 from __future__ import annotations
 
@@ -31,7 +33,7 @@ import numpy as np
 import torch
 
 # Tensor-kind stream ids (part of the Philox key).
-_X, _OUTLIER, _WG, _BIAS, _WGU, _WD, _WDENSE = 1, 2, 3, 4, 5, 6, 7
+_X, _OUTLIER, _WG, _BIAS, _WGU, _WD, _WDENSE, _WSG, _WSGU, _WSD = 1, 2, 3, 4, 5, 6, 7, 8, 9, 10
 _ROWS_PER_CHUNK = 256
 
 
@@ -175,6 +177,13 @@ def expert_down(E: int, H: int, I: int, seed: int = 0, experts=None) -> np.ndarr
     ids = range(E) if experts is None else [int(e) for e in experts]
     parts = _parallel(lambda e: _normal_bf16(seed, _WD, e, (H, I), 0.02), ids)
     return np.stack(parts) if parts else np.zeros((0, H, I), np.uint16)
+
+
+def shared_expert_weights(H: int, Is: int, seed: int = 0):
+    """Shared expert of a layer as bf16 bits: gate w_sg [H] (shared_expert_gate, N(0, 0.02)),
+    packed gate|up [2Is, H] and down [H, Is], N(0, 0.02)."""
+    return (_normal_bf16(seed, _WSG, 0, (H,), 0.02), _normal_bf16(seed, _WSGU, 0, (2 * Is, H), 0.02),
+            _normal_bf16(seed, _WSD, 0, (H, Is), 0.02))
 
 
 def dense_weight(N: int, K: int, seed: int = 0) -> np.ndarray:
