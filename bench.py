@@ -48,7 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 INT8_DATASHEET_TOPS = 4500.0
 
 HEADLINE = "qwen3-235b-a22b"
-SUB_MOE = ("qwen3-30b-a3b-decode", "qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed")
+SUB_MOE = ("qwen3-30b-a3b-decode", "qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed",
+           "qwen3-30b-a3b-prefill-shared")
 SUB_LINEAR = ("qwen3-1.7b-mlp-w4a8", "qwen3-1.7b-mlp-w8a8", "qwen3-30b-a3b-q-proj-w8a8",
               "qwen3-30b-a3b-k-proj-w8a8", "qwen3-30b-a3b-o-proj-w8a8")
 
@@ -85,7 +86,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -146,10 +147,16 @@ def cpu_oracle_rate(wl, n_tokens: int, min_seconds: float = 10.0, max_seconds: f
     dq, ds = O.quantize_weight_per_channel(synth.expert_down(wl.E, wl.H, wl.I, wl.seed, experts=touched))
     d = lambda a: {int(e): a[i] for i, e in enumerate(touched)}  # noqa: E731
     wgu_q, s_gu, wd_q, s_d = d(gq), d(gs), d(dq), d(ds)
+    if wl.shared_I:
+        wsg, sgu, sd = synth.shared_expert_weights(wl.H, wl.shared_I, wl.seed)
+        shared = (wsg, *O.quantize_weight_per_channel(sgu), *O.quantize_weight_per_channel(sd))
+        fwd = lambda: O.moe_forward_shared(x, wg, bias, wgu_q, s_gu, wd_q, s_d, wl.k, *shared, renorm=wl.renorm)  # noqa: E731
+    else:
+        fwd = lambda: O.moe_forward(x, wg, bias, wgu_q, s_gu, wd_q, s_d, wl.k, wl.renorm)  # noqa: E731
     t0 = time.perf_counter()
     reps = 0
     while True:
-        O.moe_forward(x, wg, bias, wgu_q, s_gu, wd_q, s_d, wl.k, wl.renorm)
+        fwd()
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or (reps >= 1 and el * (reps + 1) / reps > max_seconds):
@@ -209,6 +216,9 @@ def algorithmic(wl, counts: np.ndarray):
     ops = 2 * A * (2 * wl.I * wl.H + wl.H * wl.I) + 2 * wl.T * wl.H * wl.E
     w_bytes = touched * (3 * wl.I * wl.H + 4 * (2 * wl.I + wl.H))
     io_bytes = 2 * wl.T * wl.H * 2 + 2 * wl.E * wl.H
+    if wl.shared_I:  # the shared expert on every token, its weights and its bf16 gate
+        ops += 2 * wl.T * 3 * wl.shared_I * wl.H + 2 * wl.T * wl.H
+        w_bytes += 3 * wl.shared_I * wl.H + 4 * (2 * wl.shared_I + wl.H) + 2 * wl.H
     gate_up_bytes = touched * (2 * wl.I * wl.H + 4 * 2 * wl.I)
     down_bytes = touched * (wl.H * wl.I + 4 * wl.H)
     return dict(ops=ops, bytes=w_bytes + io_bytes, touched=touched, gate_up_bytes=gate_up_bytes,
@@ -225,7 +235,9 @@ def moe_launches(wl) -> int:
         front = 3
     else:
         front = 2
-    return front + 4
+    small = wl.T * wl.k <= 32 * wl.E
+    routed = front + (3 if (small and wl.I <= 1024) else 4)  # requantisation inside the short-batch down GEMM
+    return routed + (5 if wl.shared_I else 0)  # shared expert: gate, quantise, gate_up, requantise, down
 
 
 # ---------------------------------------------------------------------------- native arm
@@ -258,12 +270,18 @@ class MoELayer:
         from w8a8_int8_quantized_act_b200 import binding as B
         from w8a8_int8_quantized_act_b200 import synth
 
-        self.key = (wl.H, wl.E, wl.I, wl.seed)
+        self.key = (wl.H, wl.E, wl.I, wl.seed, wl.shared_I)
         bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
         self.wg = bf(synth.router_weight(wl.E, wl.H, wl.seed))
         self.wgu_q, self.s_gu = B.w8a8_quantize_weight_per_channel(bf(synth.expert_gate_up(wl.E, wl.I, wl.H,
                                                                                             wl.seed)))
         self.wd_q, self.s_d = B.w8a8_quantize_weight_per_channel(bf(synth.expert_down(wl.E, wl.H, wl.I, wl.seed)))
+        self.shared = None
+        if wl.shared_I:
+            wsg, sgu, sd = synth.shared_expert_weights(wl.H, wl.shared_I, wl.seed)
+            gq, gs = B.w8a8_quantize_weight_per_channel(bf(sgu[None]))
+            dq, ds = B.w8a8_quantize_weight_per_channel(bf(sd[None]))
+            self.shared = (bf(wsg), gq[0], gs[0], dq[0], ds[0])
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
@@ -280,12 +298,23 @@ def run_moe(args, wl, layer, rank, dist, dev):
     x = torch.from_numpy(x_host).view(torch.bfloat16).to(dev)
     bias = torch.from_numpy(synth.router_bias(wl.E, wl.seed)).to(dev) if wl.skewed else None
     wg, wgu_q, s_gu, wd_q, s_d = layer.wg, layer.wgu_q, layer.s_gu, layer.wd_q, layer.s_d
-    ws = torch.empty(B.w8a8_moe_workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I), dtype=torch.uint8, device=dev)
+    sh = layer.shared
+    ws_bytes = (B.w8a8_moe_shared_workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I, wl.shared_I) if sh is not None
+                else B.w8a8_moe_workspace_size(wl.T, wl.H, wl.E, wl.k, wl.I))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
+    def forward(xd, yd, st=None):
+        if sh is None:
+            B.w8a8_moe_forward(xd, wg, wgu_q, s_gu, wd_q, s_d, wl.k, renorm=wl.renorm, bias=bias, workspace=ws, y=yd,
+                               stream=st)
+        else:
+            B.w8a8_moe_forward_shared(xd, wg, wgu_q, s_gu, wd_q, s_d, wl.k, *sh, renorm=wl.renorm, bias=bias,
+                                      workspace=ws, y=yd, stream=st)
+
     def step():
-        B.w8a8_moe_forward(x, wg, wgu_q, s_gu, wd_q, s_d, wl.k, renorm=wl.renorm, bias=bias, workspace=ws, y=y)
+        forward(x, y)
 
     for _ in range(args.warmup):
         step()
@@ -315,7 +344,8 @@ def run_moe(args, wl, layer, rank, dist, dev):
     ms = start.elapsed_time(stop)
 
     # ---- second pass: K direct calls recording events at the stage boundaries, for the
-    # per-kernel durations (the dominant kernel's roofline figure comes from here)
+    # per-kernel durations (the dominant kernel's roofline figure comes from here); with a shared
+    # expert this pass times the routed layer alone (the same routed kernels)
     nst = 7
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
     for row in ev:  # torch creates the CUDA event on its first record
@@ -339,8 +369,7 @@ def run_moe(args, wl, layer, rank, dist, dev):
     e2e_steps = max(1, min(args.steps, 500))
 
     def run_e2e(xd, yd, st):
-        B.w8a8_moe_forward(xd, wg, wgu_q, s_gu, wd_q, s_d, wl.k, renorm=wl.renorm, bias=bias, workspace=ws, y=yd,
-                           stream=st)
+        forward(xd, yd, st)
 
     pipelined_e2e(3, x_pin, (wl.T, wl.H), run_e2e, dev)  # warm-up
     if dist is not None:
@@ -512,6 +541,10 @@ MEASURED_TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the gate_up launch of the
     # Qwen3-235B-A22B-shaped layer (1 pass, full workload): 1905.0 MB read + 97.5 MB written
     "qwen3-235b-a22b": (1_905_008_128 + 97_517_312, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
+    # the same two metrics on the gate_up launch of the 30B-shaped layers: decode (T = 64)
+    # 392.0 MB read + 3.6 MB written; prefill (T = 8192) 538.6 MB read + 88.7 MB written
+    "qwen3-30b-a3b-decode": (391_984_896 + 3_580_160, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
+    "qwen3-30b-a3b-prefill": (538_649_344 + 88_734_976, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
 }
 TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
@@ -584,7 +617,7 @@ def moe_result(wl, res, K, world, peaks, peak_kind):
     return {
         "value": whole_job_rate(world, wl.T, K, res["ms"]), "unit": UNIT, "ms_per_step": ms_step,
         "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "I": wl.I,
-                   "skewed_router": wl.skewed, "tokens_per_step_per_gpu": wl.T},
+                   "skewed_router": wl.skewed, "shared_expert_I": wl.shared_I, "tokens_per_step_per_gpu": wl.T},
         "roofline": roof,
         "layer": {"tops": layer_tf["tops"], "gbs": alg["bytes"] / t / 1e9, "hbm_frac": alg["bytes"] / t / 1e9 / hbm,
                   "tensor_frac_of_2x_measured_bf16": layer_tf["frac_of_2x_measured_bf16"],
@@ -738,7 +771,7 @@ def main():
             res = run_linear(args, wl, rank, dist, dev)
             return wl, linear_result(wl, res, K, world, peaks, peak_kind)
         wl = synth.MOE_WORKLOADS[wname]
-        key = (wl.H, wl.E, wl.I, wl.seed)
+        key = (wl.H, wl.E, wl.I, wl.seed, wl.shared_I)
         if layer_cache.get("key") != key:
             layer_cache.clear()
             torch.cuda.empty_cache()

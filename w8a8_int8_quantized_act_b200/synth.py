@@ -51,6 +51,7 @@ class MoEWorkload:
     skewed: bool = False
     renorm: bool = True
     seed: int = 0
+    shared_I: int = 0  # intermediate size of a shared expert (0: none)
 
     @property
     def A(self) -> int:
@@ -82,6 +83,10 @@ MOE_WORKLOADS = {
         MoEWorkload("qwen3-30b-a3b-prefill-skewed", T=8192, H=2048, E=128, k=8, I=768,
                     n_outlier=20, skewed=True),
         MoEWorkload("qwen3-235b-a22b", T=4096, H=4096, E=128, k=8, I=1536, n_outlier=41),
+        # the 30B-shaped prefill layer with one shared expert as wide as a routed one (the
+        # shared-expert path of the Qwen3-Next / Qwen3.6 layers on a supported expert count)
+        MoEWorkload("qwen3-30b-a3b-prefill-shared", T=8192, H=2048, E=128, k=8, I=768, n_outlier=20,
+                    shared_I=768),
     )
 }
 
