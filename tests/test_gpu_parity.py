@@ -238,9 +238,12 @@ def test_linear_w8a8_exact(M, K, N):
 
 
 # (1000, 1024, 6144): 384 tiles, several per CTA, the last token tile ragged (104 rows), so the
-# shared-memory output tile is handed between bulk stores and its store clips rows past M.
+# shared-memory output tile is handed between bulk stores and its store clips rows past M;
+# (200, 512, 384): four groups, the scales of a channel in one 16-byte load and none read past the
+# row; (300, 1152, 512): 9 groups, so the scales are read one by one; (257, 256, 256): a last
+# token tile of one row.
 @pytest.mark.parametrize("M,K,N", [(1, 128, 128), (200, 512, 384), (77, 1024, 256), (1000, 1024, 6144),
-                                   (2048, 2048, 6144)])
+                                   (2048, 2048, 6144), (300, 1152, 512), (257, 256, 256), (600, 1024, 384)])
 def test_linear_w4a8_exact(M, K, N):
     x = synth.activations(M, K, max(1, K // 100), seed=M + 1)
     w = synth.dense_weight(N, K, seed=N + 1)
@@ -270,9 +273,10 @@ def test_linear_prequant_matches_linear(fmt, M, K, N):
     np.testing.assert_array_equal(G.host(y2), G.host(y))
 
 
-def test_linear_w4a8_extreme_codes():
+@pytest.mark.parametrize("M,N", [(130, 128), (520, 256)])
+def test_linear_w4a8_extreme_codes(M, N):
     # every nibble pattern the quantiser can produce, including -7 and +7 everywhere
-    M, K, N = 130, 256, 128
+    K = 256
     x = O.f32_to_bf16(np.where(np.arange(M * K).reshape(M, K) % 3 == 0, -127.0, 127.0).astype(np.float32))
     wv = np.tile(np.array([7, -7, 1, -1, 0, 3, -3, 5], np.float32), (N, K // 8))
     w = O.f32_to_bf16(wv * np.float32(0.01))
@@ -282,9 +286,10 @@ def test_linear_w4a8_extreme_codes():
     np.testing.assert_array_equal(G.host(y), O.linear_w4a8(x, op, os_, 128))
 
 
-def test_linear_w4a8_largest_group_sums():
+@pytest.mark.parametrize("M", [96, 700])
+def test_linear_w4a8_largest_group_sums(M):
     # every group partial at the largest magnitude the codes allow, 127 * 7 * 128, with both signs
-    M, K, N = 96, 384, 256
+    K, N = 384, 256
     sign = np.where(np.arange(M) % 2 == 1, -1.0, 1.0).astype(np.float32)
     x = O.f32_to_bf16(np.repeat((sign * (1.0 + 0.01 * np.arange(M)))[:, None], K, axis=1).astype(np.float32))
     w = O.f32_to_bf16(np.full((N, K), 0.07, np.float32) * np.where(np.arange(N) % 3 == 0, -1.0, 1.0)[:, None]

@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(W4Cfg<NB, CV, EW>::kThreads, 1)
 #pragma unroll
       for (int j = 0; j < CW; ++j) accf[j] = 0.0f;
       float4 s_cur = load_s4(swr, 0);
-      float4 s_nxt = load_s4(swr, 4);
+      float4 s_nxt = nkb > 4 ? load_s4(swr, 4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);  // no read past the row
       // the s_x of the warp's tokens, needed only at the tile's end: loaded now
       float sxr[CW / 32];
 #pragma unroll
