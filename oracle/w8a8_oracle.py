@@ -1,4 +1,4 @@
-"""CPU oracle for the W8A8 INT8 MoE expert-FFN forward and the dense W8A8/W4A8 linear.
+"""CPU oracle for the W8A8 INT8 MoE expert-FFN forward and the dense W8A8/W4A8/MXFP8 linear.
 
 TEST INFRASTRUCTURE. This module is the slow, plain statement of what the GPU path must
 compute. Only the test-suite, the smoke check and the CPU-baseline leg of the benchmark
@@ -51,6 +51,11 @@ Readings where the pages are silent (each one is fixed identically on the GPU si
   The pages do not give the combination: it is read as y = routed + sigmoid(x . w_sg) * shared,
   the shared output entering the combine's fma chain after the k routed slots with weight
   g = sigmoid(z), z the gate logit (float64 here), sigmoid(z) = 1 / (1 + exp(-z)).
+* MXFP8 A8W8 (the AMCT Qwen3-Next page, section 六, names "MXFP A8w8" and nothing more): the OCP
+  Microscaling FP8 format, blocks of 32 values along K with one E8M0 power-of-two scale and E4M3
+  elements; E = floor(log2 amax) - 8, elements rounded to nearest even and saturated at 448. The
+  layer's product is the exact sum of the dequantised products; the GPU's fp32 sum of the same
+  products is checked within the summation bound (see ``linear_mxfp8``).
 """
 from __future__ import annotations
 
@@ -510,3 +515,98 @@ def linear_w4a8(x_bits, packed, s_w, group: int = 128) -> np.ndarray:
         acc_g = int_gemm(xq[:, ks], wq[:, ks]).astype(np.float32)
         acc_f = fma32(acc_g, np.broadcast_to(s_w[None, :, g], acc_g.shape), acc_f)
     return f32_to_bf16(acc_f * sx[:, None])
+
+
+# --------------------------------------------------------------------------------------
+# MXFP8 A8W8 (the "MXFP A8w8" row of the accuracy table, section 六 of the AMCT Qwen3-Next page)
+# --------------------------------------------------------------------------------------
+# The page names the format only. It is read as the OCP Microscaling (MX) FP8 format: blocks of
+# 32 consecutive values along K share one power-of-two scale X = 2**E stored as an E8M0 byte
+# (E + 127), and every element is an FP8 E4M3 value (1 sign, 4 exponent bits with bias 7, 3
+# mantissa bits; exponent field 0 holds the subnormals m/8 * 2**-6; 0x7F and 0xFF are NaN; no
+# infinities; the largest magnitude is 1.75 * 2**8 = 448). Activations are quantised per token
+# (dynamic), weights per output channel (static), both along K.
+#   E = floor(log2(max |v| over the block)) - 8, clamped to [-127, 127] (8 is the exponent of
+#       E4M3's largest binade); a block of zeros takes E = -127;
+#   P = E4M3(v / 2**E), rounded to nearest with ties to even, magnitudes above 448 saturating
+#       to 448 (the largest element of a block lands in [256, 512), so values in (448, 512) clip);
+#       the sign of a value that rounds to zero is kept.
+# The product of the layer is y[t, n] = sum_k (P_x[t,k] X_x[t,k/32]) (P_w[n,k] X_w[n,k/32]) in
+# exact arithmetic; a tensor core sums it in fp32 in an order of its own, so the GPU result is
+# checked against this exact value within the fp32 summation bound (``linear_mxfp8``).
+MX_BLOCK = 32
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """float64 value of each E4M3 byte (NaN for 0x7F / 0xFF)."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    return np.where((c & 0x7F) == 0x7F, np.nan, sign * mag)
+
+
+# non-negative finite E4M3 values in increasing order, with their codes
+_E4M3_POS_CODES = np.arange(0x7F, dtype=np.uint8)
+_E4M3_POS_VALUES = e4m3_decode(_E4M3_POS_CODES)
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """E4M3 byte of each finite float64 value: nearest representable magnitude, ties to the even
+    mantissa, saturating at 448; negative values (and -0) carry the sign bit."""
+    v = np.asarray(v, np.float64)
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    # the quantum of the binade that holds a: 2**(e - 3) for e = floor(log2 a) >= -6, and the
+    # subnormal quantum 2**-9 below 2**-6
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = np.maximum(ex - 1, -6)
+    q = np.exp2(e.astype(np.float64) - 3.0)
+    n = np.rint(a / q)                        # a / q is exact; rint rounds halves to even
+    mag = np.minimum(n * q, E4M3_MAX)         # n = 16 is the first value of the next binade
+    idx = np.searchsorted(_E4M3_POS_VALUES, mag)
+    assert np.all(_E4M3_POS_VALUES[idx] == mag)
+    code = _E4M3_POS_CODES[idx]
+    return np.where(np.signbit(v), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def mx_quantize_rows(v_bits: np.ndarray):
+    """MXFP8 codes [R, K] (uint8, E4M3) and scales [R, K/32] (uint8, E8M0) of bf16 rows."""
+    v = bf16_to_f32(v_bits).astype(np.float64)
+    R, K = v.shape
+    assert K % MX_BLOCK == 0
+    blocks = v.reshape(R, K // MX_BLOCK, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=2)
+    _, ex = np.frexp(np.where(amax > 0, amax, 1.0))      # amax in [2**(ex-1), 2**ex)
+    E = np.where(amax > 0, ex - 1 - 8, -127)
+    E = np.clip(E, -127, 127)
+    codes = e4m3_encode(blocks / np.exp2(E.astype(np.float64))[:, :, None])
+    return codes.reshape(R, K), (E + 127).astype(np.uint8)
+
+
+def mx_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """float64 values P * 2**(scale - 127) of MXFP8 rows."""
+    R, K = codes.shape
+    p = e4m3_decode(codes).reshape(R, K // MX_BLOCK, MX_BLOCK)
+    x = np.exp2(np.asarray(scales, np.float64) - 127.0)
+    return (p * x[:, :, None]).reshape(R, K)
+
+
+def linear_mxfp8(x_bits, w_codes, w_scales) -> dict:
+    """Dense MXFP8 A8W8 linear: x quantised per token to MXFP8, then y = A . W^T exactly.
+
+    Returns the token codes and scales, y (float64, the exact sum of the dequantised products
+    up to float64 rounding) and ``bound``: the largest |y_gpu - y| a bf16 result of an fp32
+    summation of the same products in any order can show, (K - 1) * 2**-24 * S (fp32
+    summation) plus 2**-8 times the fp32 result's magnitude (one bf16 rounding), with
+    S = sum_k |A[t,k] W[n,k]|."""
+    xc, xs = mx_quantize_rows(x_bits)
+    A = mx_dequantize(xc, xs)
+    W = mx_dequantize(w_codes, w_scales)
+    y = A @ W.T
+    K = A.shape[1]
+    S = np.abs(A) @ np.abs(W).T
+    summ = (K - 1) * 2.0 ** -24 * S
+    bound = summ + 2.0 ** -8 * (np.abs(y) + summ)
+    return dict(codes=xc, scales=xs, y=y, bound=bound)
