@@ -45,13 +45,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # B200 datasheet dense INT8 tensor throughput (the 9 POPS figure NVIDIA quotes is with 2:4
 # sparsity); fractions are also given against 2 x the measured bf16 GEMM rate (the nominal
 # int8:bf16 ratio applied to this machine's measured peak)
-INT8_DATASHEET_TOPS = 4500.0
+INT8_DATASHEET_TOPS = 4500.0  # B200 dense int8 (and fp8)
+BF16_DATASHEET_TFLOPS = 2250.0  # B200 dense bf16
 
 HEADLINE = "qwen3-235b-a22b"
 SUB_MOE = ("qwen3-30b-a3b-decode", "qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed",
            "qwen3-30b-a3b-prefill-shared")
 SUB_LINEAR = ("qwen3-1.7b-mlp-w4a8", "qwen3-1.7b-mlp-w8a8", "qwen3-30b-a3b-q-proj-w8a8",
-              "qwen3-30b-a3b-k-proj-w8a8", "qwen3-30b-a3b-o-proj-w8a8")
+              "qwen3-30b-a3b-k-proj-w8a8", "qwen3-30b-a3b-o-proj-w8a8", "qwen3-1.7b-mlp-mxfp8")
 
 
 def parse():
@@ -174,6 +175,9 @@ def cpu_oracle_linear_rate(wl, n_tokens: int, min_seconds: float = 5.0, max_seco
     if wl.fmt == "int4":
         packed, sw = O.quantize_weight_int4_per_group(w, wl.group)
         fwd = lambda: O.linear_w4a8(x, packed, sw, wl.group)  # noqa: E731
+    elif wl.fmt == "mxfp8":
+        wc, ws = O.mx_quantize_rows(w)
+        fwd = lambda: O.linear_mxfp8(x, wc, ws)  # noqa: E731
     else:
         wq, sw = O.quantize_weight_per_channel(w)
         fwd = lambda: O.linear_w8a8(x, wq, sw)  # noqa: E731
@@ -444,14 +448,27 @@ def run_linear(args, wl, rank, dist, dev):
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
     x = bf(x_host)
     w = bf(synth.dense_weight(wl.N, wl.K, wl.seed))
+    mx = wl.fmt == "mxfp8"
     if wl.fmt == "int4":
         wq, sw = B.w8a8_quantize_weight_int4_per_group(w, wl.group)
         fmt, group = B.W8A8_W_INT4_PER_GROUP, wl.group
+    elif mx:
+        wq, sw = B.w8a8_mxfp8_quantize(w)  # E4M3 codes [N, K], E8M0 scales [N, K/32]
+        fmt, group = None, 32
     else:
         wq, sw = B.w8a8_quantize_weight_per_channel(w)
         fmt, group = B.W8A8_W_INT8_PER_CHANNEL, 128
     del w
-    ws = torch.empty(B.w8a8_linear_workspace_size(wl.M, wl.K, wl.N, fmt, group), dtype=torch.uint8, device=dev)
+    ws_bytes = (B.w8a8_mxfp8_linear_workspace_size(wl.M, wl.K, wl.N) if mx
+                else B.w8a8_linear_workspace_size(wl.M, wl.K, wl.N, fmt, group))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def linear(xd, pk, s_, wsp, yd, st=None):
+        if mx:
+            B.w8a8_mxfp8_linear(xd, pk, s_, workspace=wsp, y=yd, stream=st)
+        else:
+            B.w8a8_linear(xd, pk, s_, fmt, group, workspace=wsp, y=yd, stream=st)
+
     y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=dev)
     # rotate over weight copies (more than the L2 together) so every step reads its weights from HBM
     n_copies = max(2, min(32, -(-256 * 2 ** 20 // (wq.numel() * wq.element_size()))))
@@ -460,7 +477,7 @@ def run_linear(args, wl, rank, dist, dev):
 
     def step(i):
         pk, s_ = copies[i % len(copies)]
-        B.w8a8_linear(x, pk, s_, fmt, group, workspace=ws, y=y)
+        linear(x, pk, s_, ws, y)
 
     for i in range(args.warmup):
         step(i)
@@ -488,7 +505,10 @@ def run_linear(args, wl, rank, dist, dev):
     ms = start.elapsed_time(stop)
     # the GEMM launch alone (the dominant kernel): the quantised activations are made once, then
     # K GEMM launches are timed with events on the launching stream
-    gemm_ms = time_linear_gemm(B, x, copies, fmt, group, wl, args.steps, stream)
+    if mx:
+        gemm_ms = time_mxfp8_gemm(B, ws, wl, args.steps, stream)
+    else:
+        gemm_ms = time_linear_gemm(B, x, copies, fmt, group, wl, args.steps, stream)
     # end to end with host buffers (copies inside the timed region)
     x_pin = torch.from_numpy(x_host).view(torch.bfloat16).pin_memory()
     n_e2e = max(1, min(args.steps, 200))
@@ -498,7 +518,7 @@ def run_linear(args, wl, rank, dist, dev):
     def run_e2e(xd, yd, st):
         pk, s_ = copies[e2e_i[0] % len(copies)]
         e2e_i[0] += 1
-        B.w8a8_linear(xd, pk, s_, fmt, group, workspace=e2e_ws, y=yd, stream=st)
+        linear(xd, pk, s_, e2e_ws, yd, st)
 
     pipelined_e2e(3, x_pin, (wl.M, wl.N), run_e2e, dev)  # warm-up
     if dist is not None:
@@ -508,7 +528,30 @@ def run_linear(args, wl, rank, dist, dev):
     ms, e2e_ms = max_over_ranks(dist, [ms, e2e_ms], dev)
     return dict(ms=ms, e2e_ms=e2e_ms, e2e_steps=n_e2e, gemm_ms=gemm_ms, clocks=clk.summary(),
                 h2d=wl.M * wl.K * 2, d2h=wl.M * wl.N * 2,
-                weight_bytes=wq.numel() * wq.element_size() + sw.numel() * 4)
+                weight_bytes=wq.numel() * wq.element_size() + sw.numel() * sw.element_size())
+
+
+def time_mxfp8_gemm(B, ws, wl, steps, stream):
+    """Mean duration (ms) of the MXFP8 linear's GEMM launch alone, on the dequantised operands the
+    last w8a8_mxfp8_linear call left in `ws`: K launches of w8a8_mxfp8_linear_dequantized timed
+    with CUDA events on `stream`. (Their weights come from one copy: the 25 MB bf16 operand stays in
+    the L2, which the roofline's HBM side does not assume.)"""
+    import torch
+
+    inter = B.mxfp8_linear_intermediates(ws, wl.M, wl.K, wl.N)
+    a, w = inter["a"].clone(), inter["w"].clone()
+    y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=a.device)
+    for _ in range(3):
+        B.w8a8_mxfp8_linear_dequantized(a, w, y=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        B.w8a8_mxfp8_linear_dequantized(a, w, y=y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    B.w8a8_check_status()
+    return e0.elapsed_time(e1) / steps
 
 
 def time_linear_gemm(B, x, copies, fmt, group, wl, steps, stream):
@@ -550,6 +593,7 @@ TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
     "w4a8": ("gemm.cuh", "gemm_w4a8.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
     "w8a8": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
+    "mxfp8": ("gemm.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
 }
 
 
@@ -633,10 +677,52 @@ def moe_result(wl, res, K, world, peaks, peak_kind):
     }
 
 
+def bf16_roofline_entry(ops: float, nbytes: float, seconds: float, peaks, peak_kind, traffic, kernel: str) -> dict:
+    """Roofline of a kind::f16 (bf16 operand) GEMM launch: tensor time at the measured bf16 rate
+    against HBM time at the measured copy bandwidth; the FP8 datasheet rate is given for context
+    (the rate of the block-scaled FP8 MMA that would run the same MXFP8 product natively)."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tflops = ops / seconds / 1e12
+    gbs = nbytes / seconds / 1e9
+    tensor = {"tflops": tflops, "frac_of_measured_bf16": tflops / bf16, "peak_measured_bf16": bf16,
+              "frac_of_bf16_datasheet": tflops / BF16_DATASHEET_TFLOPS, "peak_bf16_datasheet": BF16_DATASHEET_TFLOPS,
+              "frac_of_fp8_datasheet": tflops / INT8_DATASHEET_TOPS, "peak_fp8_datasheet": INT8_DATASHEET_TOPS}
+    if ops / (bf16 * 1e12) >= nbytes / (hbm * 1e9):
+        roof = {"bound": "tensor", "achieved": tflops, "peak": bf16, "unit": "TFLOP/s", "frac": tflops / bf16,
+                "peak_source": f"{peak_kind} bf16 TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "peak_source": f"{peak_kind} HBM copy GB/s"}
+    roof.update({"traffic": traffic, "traffic_unit": "bytes per launch", "kernel": kernel, "alg_ops": ops,
+                 "alg_bytes": nbytes, "launch_ms": seconds * 1e3, "tensor": tensor,
+                 "hbm": {"gbs": gbs, "frac": gbs / hbm, "peak": hbm}})
+    return roof
+
+
 def linear_result(wl, res, K, world, peaks, peak_kind):
     ms_step = res["ms"] / K
     ops = 2.0 * wl.M * wl.N * wl.K
     nbytes = res["weight_bytes"] + wl.M * wl.K * 2 + wl.M * wl.N * 2
+    if wl.fmt == "mxfp8":
+        roof = bf16_roofline_entry(ops, nbytes, res["gemm_ms"] / 1e3, peaks, peak_kind,
+                                   measured_traffic(wl.name, "mxfp8"),
+                                   "MXFP8 GEMM (operands dequantised exactly to bf16, tcgen05 kind::f16, fp32 sums)")
+        step_tflops = ops / (ms_step / 1e3) / 1e12
+        bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        return {
+            "value": whole_job_rate(world, wl.M, K, res["ms"]), "unit": UNIT, "ms_per_step": ms_step,
+            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "weights": "mxfp8 e4m3 + e8m0",
+                       "block": 32},
+            "roofline": roof,
+            "step": {"tflops": step_tflops, "tensor_frac_of_measured_bf16": step_tflops / bf16,
+                     "note": "step = MXFP8 quantisation of x (with its bf16 dequantisation), dequantisation of w, "
+                             "bf16 GEMM"},
+            "e2e": {"value": whole_job_rate(world, wl.M, res["e2e_steps"], res["e2e_ms"]), "unit": UNIT,
+                    "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "overlap": E2E_OVERLAP},
+            "gpu_launches": 3 * K,
+            "clocks": res["clocks"],
+        }
     kind = "w4a8" if wl.fmt == "int4" else "w8a8"
     kernel = ("W4A8 GEMM (tcgen05 kind::i8, int4 unpacked to int8 in shared memory, per-group fp32 scaling)"
               if wl.fmt == "int4" else "W8A8 GEMM (tcgen05 kind::i8, per-token x per-channel dequant epilogue)")
@@ -807,7 +893,8 @@ def main():
                 sub["cpu_baseline"] = moe_cpu_baseline(swl, default_sample_tokens(swl), 4.0, 12.0)
     out = top_line(head, name, args, world)
     if name in synth.LINEAR_WORKLOADS:
-        out["dtype"] = "int8 (int4 weights unpacked to int8)" if wl.fmt == "int4" else "int8"
+        out["dtype"] = {"int4": "int8 (int4 weights unpacked to int8)", "int8": "int8",
+                        "mxfp8": "mxfp8 (e4m3 x e8m0, dequantised exactly to bf16)"}[wl.fmt]
     if subs:
         out["sub_results"] = subs
     if probe is not None:

@@ -264,6 +264,43 @@ int w8a8_linear(const w8a8_bf16* x, const void* w, const float* sw, int w_format
 int w8a8_linear_prequant(const int8_t* xq, const float* sx, const void* w, const float* sw, int w_format, int group,
                          int64_t M, int64_t K, int64_t N, w8a8_bf16* y, w8a8_stream stream);
 
+/* Defined by: section 六 of "Qwen3-Next-80B-A3B-Instruct 在 AMCT 中的 MoE 混合注意力量化适配实战",
+ * the "MXFP A8w8" row of its accuracy table (the format is named there and nothing more; it is
+ * read as the OCP Microscaling FP8 format).
+ * MXFP8 quantisation of bf16 rows along K, in blocks of 32 consecutive values:
+ *   E = floor(log2(max |v| of the block)) - 8, clamped to [-127, 127] (-127 for a block of zeros);
+ *   scales[r, b] = E + 127 (an E8M0 byte: the block's scale is 2^E);
+ *   codes[r, k] = the FP8 E4M3 byte of v * 2^-E: nearest, ties to even, magnitudes above 448
+ *   saturating to 448, the sign kept when the value rounds to zero.
+ * Used for the weights of a layer (once, per output channel) and, inside w8a8_mxfp8_linear, for
+ * its activations (per token, at every call).
+ *   x bf16 [R, K] (16-byte aligned), codes uint8 [R, K] (8-byte aligned), scales uint8 [R, K/32];
+ *   all device memory owned by the caller. K % 32 == 0 (else W8A8_ERR_UNSUPPORTED). */
+int w8a8_mxfp8_quantize(const w8a8_bf16* x, int64_t R, int64_t K, uint8_t* codes, uint8_t* scales,
+                        w8a8_stream stream);
+
+/* Workspace bytes w8a8_mxfp8_linear needs (0 if the shape is rejected). */
+size_t w8a8_mxfp8_linear_workspace_size(int64_t M, int64_t K, int64_t N);
+
+/* Defined by: the same row of the same table (MXFP8 A8W8: both operands in MXFP8).
+ * Dense MXFP8 A8W8 linear: x is quantised to MXFP8 per token (w8a8_mxfp8_quantize), both
+ * operands are dequantised to P * 2^E (exact in bf16) and multiplied on the tensor cores with fp32
+ * accumulation: y[m, n] = bf16(sum_k A[m, k] W[n, k]), the sum of the exact products taken in the
+ * tensor core's own order (so within (K - 1) * 2^-24 * sum_k |A W| of the exact sum before the
+ * bf16 rounding).
+ *   x bf16 [M, K]; w_codes uint8 [N, K] and w_scales uint8 [N, K/32] from w8a8_mxfp8_quantize;
+ *   workspace of w8a8_mxfp8_linear_workspace_size() bytes (256-byte aligned; it receives x's
+ *   codes at offset 0 and its scales after them, 256-byte aligned); y bf16 [M, N].
+ * K % 64 == 0, N % 128 == 0 (else W8A8_ERR_UNSUPPORTED). */
+int w8a8_mxfp8_linear(const w8a8_bf16* x, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M, int64_t K,
+                      int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream);
+
+/* The GEMM of w8a8_mxfp8_linear on operands already dequantised to bf16 (P * 2^E):
+ *   a bf16 [M, K], w bf16 [N, K], y bf16 [M, N] = bf16(fp32 sum_k a[m, k] w[n, k]) on the tensor
+ *   cores (kind::f16). Same shape rules as w8a8_mxfp8_linear; needs no workspace. */
+int w8a8_mxfp8_linear_dequantized(const w8a8_bf16* a, const w8a8_bf16* w, int64_t M, int64_t K, int64_t N,
+                                  w8a8_bf16* y, w8a8_stream stream);
+
 /* Exact integer GEMM on the tensor cores: c[m, n] = sum_k a[m, k] * b[n, k] in int32: the
  * int8 x int8 product every W8A8 Linear of the group_0 scheme accumulates before its scales.
  *   a int8 [M, K], b int8 [N, K], c int32 [M, N];  K % 128 == 0, N % 128 == 0. */

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.w8a8_version() == 200
+    assert lib.w8a8_version() == 210
     for st in range(-5, 1):
         assert B.status_string(st) not in ("", "unknown status")
 
@@ -56,6 +56,9 @@ def test_workspace_queries_are_host_only(lib):
     assert B.w8a8_moe_workspace_size(64, 2048, 4, 8, 768) == 0  # k > E
     assert B.w8a8_linear_workspace_size(2048, 2048, 6144, 1, 64) == 0  # group != 128
     assert B.w8a8_linear_workspace_size(2048, 2048, 6144, 1, 128) > 0
+    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2048, 6144) >= 2048 * 2048 * (1 + 2) + 6144 * 2048 * 2
+    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2016, 6144) == 0  # K % 64
+    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2048, 6100) == 0  # N % 128
 
 
 def test_argument_checks_reject_before_any_launch(lib):
@@ -74,6 +77,13 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert lib.w8a8_moe_route(None, None, None, 4, 2048, 128, 9, 1, None, None, None, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_quantize_weight_int4_per_group(None, 4, 256, 64, None, None, None) == B.W8A8_ERR_UNSUPPORTED
     assert lib.w8a8_gemm_s8s8s32(None, None, None, 4, 100, 128, None) == B.W8A8_ERR_UNSUPPORTED
+    assert lib.w8a8_mxfp8_quantize(c(16), 4, 48, c(16), c(16), None) == B.W8A8_ERR_UNSUPPORTED  # K % 32
+    assert lib.w8a8_mxfp8_quantize(None, 4, 64, None, None, None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_mxfp8_quantize(None, 0, 64, None, None, None) == B.W8A8_OK  # empty
+    assert lib.w8a8_mxfp8_linear(c(256), c(256), c(256), 8, 128, 256, c(256), 10, c(256), None) == \
+        B.W8A8_ERR_WORKSPACE
+    assert lib.w8a8_mxfp8_linear(c(256), c(256), c(256), 8, 96, 256, c(256), 1 << 20, c(256), None) == \
+        B.W8A8_ERR_UNSUPPORTED  # K % 64
     assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_debug_rcp_approx_ulp(0, 10, c(16), None) == B.W8A8_ERR_ARG  # not a normal input
     assert lib.w8a8_debug_rcp_approx_ulp(0x7E7FFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # reciprocal subnormal

@@ -72,6 +72,10 @@ SIGNATURES = {
     "w8a8_linear": (_int, [_c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _size, _c_p, _c_p]),
     "w8a8_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _int, _int, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_gemm_s8s8s32": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p]),
+    "w8a8_mxfp8_quantize": (_int, [_c_p, _i64, _i64, _c_p, _c_p, _c_p]),
+    "w8a8_mxfp8_linear_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
+    "w8a8_mxfp8_linear": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, ctypes.c_size_t, _c_p, _c_p]),
+    "w8a8_mxfp8_linear_dequantized": (_int, [_c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
     "w8a8_debug_rcp_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
     "w8a8_debug_ex2_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
@@ -363,6 +367,60 @@ def w8a8_linear_prequant(xq, sx, w, sw, w_format: int = W8A8_W_INT8_PER_CHANNEL,
     _check(lib().w8a8_linear_prequant(_ptr(xq), _ptr(sx), _ptr(w), _ptr(sw), w_format, group, M, K, N, _ptr(y),
                                       _stream(stream)), "w8a8_linear_prequant")
     return y
+
+
+def w8a8_mxfp8_quantize(x: torch.Tensor, codes=None, scales=None, stream=None):
+    """x bf16 [R, K] -> (codes uint8 [R, K] (E4M3), scales uint8 [R, K/32] (E8M0))."""
+    _bf16(x)
+    R, K = x.shape
+    codes = torch.empty((R, K), dtype=torch.uint8, device=x.device) if codes is None else codes
+    scales = torch.empty((R, max(K // 32, 1)), dtype=torch.uint8, device=x.device) if scales is None else scales
+    _check(lib().w8a8_mxfp8_quantize(_ptr(x), R, K, _ptr(codes), _ptr(scales), _stream(stream)),
+           "w8a8_mxfp8_quantize")
+    return codes, scales
+
+
+def w8a8_mxfp8_linear_workspace_size(M: int, K: int, N: int) -> int:
+    return int(lib().w8a8_mxfp8_linear_workspace_size(M, K, N))
+
+
+def w8a8_mxfp8_linear(x, w_codes, w_scales, workspace=None, y=None, stream=None):
+    """Dense MXFP8 A8W8 linear: y bf16 [M, N] = x [M, K] . W^T, W given as MXFP8 codes and scales."""
+    _bf16(x)
+    M, K = x.shape
+    N = w_codes.shape[0]
+    ws_bytes = w8a8_mxfp8_linear_workspace_size(M, K, N)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(lib().w8a8_mxfp8_linear(_ptr(x), _ptr(w_codes), _ptr(w_scales), M, K, N, _ptr(workspace),
+                                   workspace.numel(), _ptr(y), _stream(stream)), "w8a8_mxfp8_linear")
+    return y
+
+
+def w8a8_mxfp8_linear_dequantized(a, w, y=None, stream=None):
+    """The GEMM of w8a8_mxfp8_linear on dequantised bf16 operands a [M, K], w [N, K]."""
+    _bf16(a), _bf16(w)
+    M, K = a.shape
+    N = w.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if y is None else y
+    _check(lib().w8a8_mxfp8_linear_dequantized(_ptr(a), _ptr(w), M, K, N, _ptr(y), _stream(stream)),
+           "w8a8_mxfp8_linear_dequantized")
+    return y
+
+
+def mxfp8_linear_intermediates(workspace, M: int, K: int, N: int) -> dict:
+    """What w8a8_mxfp8_linear left in its workspace: x's MXFP8 codes [M, K] and scales [M, K/32],
+    and both dequantised operands, a bf16 [M, K] and w bf16 [N, K]."""
+    a256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
+    codes = workspace[:M * K].view(M, K)
+    off = a256(M * K)
+    scales = workspace[off:off + M * (K // 32)].view(M, K // 32)
+    off += a256(M * (K // 32))
+    a = workspace[off:off + M * K * 2].view(torch.bfloat16).view(M, K)
+    off += a256(M * K * 2)
+    w = workspace[off:off + N * K * 2].view(torch.bfloat16).view(N, K)
+    return dict(codes=codes, scales=scales, a=a, w=w)
 
 
 def w8a8_gemm_s8s8s32(a, b, c=None, stream=None):
