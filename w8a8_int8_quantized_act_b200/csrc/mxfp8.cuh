@@ -27,27 +27,29 @@ __device__ __forceinline__ int bf16_floor_log2(uint32_t mag) {
   return (31 - __clz(int(mag))) - 133;  // a subnormal is m * 2^-133, m its 7-bit mantissa
 }
 
-// E4M3 byte of r: nearest, ties to even, saturating at 448 (cvt.rn.satfinite).
-__device__ __forceinline__ uint32_t e4m3_byte(float r) {
-  return uint32_t(__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3));
-}
-// Exact value of an E4M3 byte (every E4M3 value is an fp16 value).
-__device__ __forceinline__ float e4m3_float(uint32_t c) {
-  const __half_raw h = __nv_cvt_fp8_to_halfraw(__nv_fp8_storage_t(c), __NV_E4M3);
-  return __half2float(__half(h));
+// E4M3 bytes of (lo, hi) in the low and high byte: nearest, ties to even, saturating at 448
+// (cvt.rn.satfinite.e4m3x2).
+__device__ __forceinline__ uint32_t e4m3_pair(float lo, float hi) {
+  return uint32_t(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// Eight elements of one block with the block's exponent E into bf16 values P * 2^E, packed.
-__device__ __forceinline__ uint4 mx_dequant8(uint2 codes, int E) {
+// 2^E as an fp32 value for E in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float pow2_f32(int E) {
+  return E >= -126 ? __int_as_float((E + 127) << 23) : __int_as_float(0x00400000);
+}
+
+// Eight elements of one block with the block's scale 2^E into bf16 values P * 2^E, packed. The
+// E4M3 -> fp16 conversion and the power-of-two product are exact.
+__device__ __forceinline__ uint4 mx_dequant8(uint2 codes, float scale) {
   uint32_t out[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t w = (i < 2) ? codes.x : codes.y;
-    const int sh = (i & 1) * 16;
-    const float a = ldexpf(e4m3_float((w >> sh) & 0xFFu), E);
-    const float b = ldexpf(e4m3_float((w >> (sh + 8)) & 0xFFu), E);
-    out[i] = uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
-             (uint32_t(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
+    const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t((w >> ((i & 1) * 16)) & 0xFFFFu),
+                                                      __NV_E4M3);
+    const float2 f = __half22float2(__half2(h2));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(f.x, scale), __fmul_rn(f.y, scale));
+    out[i] = *reinterpret_cast<const uint32_t*>(&b);
   }
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
@@ -82,15 +84,12 @@ __global__ void __launch_bounds__(kMxWarps * 32) mx_quant_rows_kernel(const uint
   const float inv = __int_as_float((127 - E) << 23);  // 2^-E, exact (E <= 119 for bf16 input)
   uint32_t c[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t lo = e4m3_byte(__fmul_rn(bf16_lo(w[i]), inv));
-    const uint32_t hi = e4m3_byte(__fmul_rn(bf16_hi(w[i]), inv));
-    c[i >> 1] |= (lo | (hi << 8)) << (16 * (i & 1));
-  }
+  for (int i = 0; i < 4; ++i)
+    c[i >> 1] |= e4m3_pair(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv)) << (16 * (i & 1));
   if (!valid) return;
   *reinterpret_cast<uint2*>(codes + r * K + k0) = make_uint2(c[0], c[1]);
   if ((lane & 3) == 0) scales[r * (K / kMxBlock) + k0 / kMxBlock] = uint8_t(E + 127);
-  if (deq != nullptr) *reinterpret_cast<uint4*>(deq + r * K + k0) = mx_dequant8(make_uint2(c[0], c[1]), E);
+  if (deq != nullptr) *reinterpret_cast<uint4*>(deq + r * K + k0) = mx_dequant8(make_uint2(c[0], c[1]), pow2_f32(E));
 }
 
 // The dequantised bf16 values P * 2^(scale - 127) of MXFP8 rows (codes [R, K], scales [R, K / 32]).
@@ -108,7 +107,7 @@ __global__ void __launch_bounds__(kMxWarps * 32) mx_dequant_rows_kernel(const ui
   if (k0 >= K) return;
   const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + r * K + k0));
   const int E = int(__ldg(scales + r * (K / kMxBlock) + k0 / kMxBlock)) - 127;
-  *reinterpret_cast<uint4*>(deq + r * K + k0) = mx_dequant8(c, E);
+  *reinterpret_cast<uint4*>(deq + r * K + k0) = mx_dequant8(c, pow2_f32(E));
 }
 
 }  // namespace w8a8
