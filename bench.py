@@ -46,7 +46,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # sparsity); fractions are also given against 2 x the measured bf16 GEMM rate (the nominal
 # int8:bf16 ratio applied to this machine's measured peak)
 INT8_DATASHEET_TOPS = 4500.0  # B200 dense int8 (and fp8)
-BF16_DATASHEET_TFLOPS = 2250.0  # B200 dense bf16
 
 HEADLINE = "qwen3-235b-a22b"
 SUB_MOE = ("qwen3-30b-a3b-decode", "qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed",
@@ -506,7 +505,7 @@ def run_linear(args, wl, rank, dist, dev):
     # the GEMM launch alone (the dominant kernel): the quantised activations are made once, then
     # K GEMM launches are timed with events on the launching stream
     if mx:
-        gemm_ms = time_mxfp8_gemm(B, ws, wl, args.steps, stream)
+        gemm_ms = time_mxfp8_gemm(B, x, copies, wl, args.steps, stream)
     else:
         gemm_ms = time_linear_gemm(B, x, copies, fmt, group, wl, args.steps, stream)
     # end to end with host buffers (copies inside the timed region)
@@ -531,23 +530,23 @@ def run_linear(args, wl, rank, dist, dev):
                 weight_bytes=wq.numel() * wq.element_size() + sw.numel() * sw.element_size())
 
 
-def time_mxfp8_gemm(B, ws, wl, steps, stream):
-    """Mean duration (ms) of the MXFP8 linear's GEMM launch alone, on the dequantised operands the
-    last w8a8_mxfp8_linear call left in `ws`: K launches of w8a8_mxfp8_linear_dequantized timed
-    with CUDA events on `stream`. (Their weights come from one copy: the 25 MB bf16 operand stays in
-    the L2, which the roofline's HBM side does not assume.)"""
+def time_mxfp8_gemm(B, x, copies, wl, steps, stream):
+    """Mean duration (ms) of the MXFP8 linear's GEMM launch alone: x is quantised to MXFP8 once,
+    then K launches of w8a8_mxfp8_linear_prequant over the rotating weight copies are timed with
+    CUDA events on `stream`."""
     import torch
 
-    inter = B.mxfp8_linear_intermediates(ws, wl.M, wl.K, wl.N)
-    a, w = inter["a"].clone(), inter["w"].clone()
-    y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=a.device)
-    for _ in range(3):
-        B.w8a8_mxfp8_linear_dequantized(a, w, y=y)
+    xc, xs = B.w8a8_mxfp8_quantize(x)
+    y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=x.device)
+    for i in range(3):
+        pk, s_ = copies[i % len(copies)]
+        B.w8a8_mxfp8_linear_prequant(xc, xs, pk, s_, y=y)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(steps):
-        B.w8a8_mxfp8_linear_dequantized(a, w, y=y)
+    for i in range(steps):
+        pk, s_ = copies[i % len(copies)]
+        B.w8a8_mxfp8_linear_prequant(xc, xs, pk, s_, y=y)
     e1.record(stream)
     torch.cuda.synchronize()
     B.w8a8_check_status()
@@ -588,12 +587,15 @@ MEASURED_TRAFFIC = {
     # 392.0 MB read + 3.6 MB written; prefill (T = 8192) 538.6 MB read + 88.7 MB written
     "qwen3-30b-a3b-decode": (391_984_896 + 3_580_160, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
     "qwen3-30b-a3b-prefill": (538_649_344 + 88_734_976, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
+    # the W4A8 GEMM launch of the 2048 x 2048 -> 6144 linear: 10.9 MB read (weights, scales, token
+    # codes once), nothing written back to DRAM within the launch (the 25 MB output stays in L2)
+    "qwen3-1.7b-mlp-w4a8": (10_933_760 + 0, "1b4b2dc7d15bec2e91ed021dfeeca923eb8d5b51"),
 }
 TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
     "w4a8": ("gemm.cuh", "gemm_w4a8.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
     "w8a8": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
-    "mxfp8": ("gemm.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
+    "mxfp8": ("elementwise.cuh", "gemm.cuh", "mxfp8.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
 }
 
 
@@ -635,7 +637,7 @@ def roofline_entry(ops: float, nbytes: float, seconds: float, peaks, peak_kind, 
     if t_ops >= t_bytes:
         roof = {"bound": "tensor", "achieved": tf["tops"], "peak": tf["peak_2x_measured_bf16"], "unit": "TOPS",
                 "frac": tf["frac_of_2x_measured_bf16"],
-                "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8:bf16 ratio)"}
+                "peak_source": f"{peak_kind} bf16 TFLOP/s x 2 (nominal int8 or fp8 : bf16 ratio)"}
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                 "peak_source": f"{peak_kind} HBM copy GB/s"}
@@ -677,50 +679,25 @@ def moe_result(wl, res, K, world, peaks, peak_kind):
     }
 
 
-def bf16_roofline_entry(ops: float, nbytes: float, seconds: float, peaks, peak_kind, traffic, kernel: str) -> dict:
-    """Roofline of a kind::f16 (bf16 operand) GEMM launch: tensor time at the measured bf16 rate
-    against HBM time at the measured copy bandwidth; the FP8 datasheet rate is given for context
-    (the rate of the block-scaled FP8 MMA that would run the same MXFP8 product natively)."""
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    tflops = ops / seconds / 1e12
-    gbs = nbytes / seconds / 1e9
-    tensor = {"tflops": tflops, "frac_of_measured_bf16": tflops / bf16, "peak_measured_bf16": bf16,
-              "frac_of_bf16_datasheet": tflops / BF16_DATASHEET_TFLOPS, "peak_bf16_datasheet": BF16_DATASHEET_TFLOPS,
-              "frac_of_fp8_datasheet": tflops / INT8_DATASHEET_TOPS, "peak_fp8_datasheet": INT8_DATASHEET_TOPS}
-    if ops / (bf16 * 1e12) >= nbytes / (hbm * 1e9):
-        roof = {"bound": "tensor", "achieved": tflops, "peak": bf16, "unit": "TFLOP/s", "frac": tflops / bf16,
-                "peak_source": f"{peak_kind} bf16 TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                "peak_source": f"{peak_kind} HBM copy GB/s"}
-    roof.update({"traffic": traffic, "traffic_unit": "bytes per launch", "kernel": kernel, "alg_ops": ops,
-                 "alg_bytes": nbytes, "launch_ms": seconds * 1e3, "tensor": tensor,
-                 "hbm": {"gbs": gbs, "frac": gbs / hbm, "peak": hbm}})
-    return roof
-
-
 def linear_result(wl, res, K, world, peaks, peak_kind):
     ms_step = res["ms"] / K
     ops = 2.0 * wl.M * wl.N * wl.K
     nbytes = res["weight_bytes"] + wl.M * wl.K * 2 + wl.M * wl.N * 2
     if wl.fmt == "mxfp8":
-        roof = bf16_roofline_entry(ops, nbytes, res["gemm_ms"] / 1e3, peaks, peak_kind,
-                                   measured_traffic(wl.name, "mxfp8"),
-                                   "MXFP8 GEMM (operands dequantised exactly to bf16, tcgen05 kind::f16, fp32 sums)")
-        step_tflops = ops / (ms_step / 1e3) / 1e12
-        bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        roof = roofline_entry(ops, nbytes, res["gemm_ms"] / 1e3, peaks, peak_kind, measured_traffic(wl.name, "mxfp8"),
+                              "MXFP8 GEMM (tcgen05 kind::mxf8f6f4 block-scaled FP8 MMA, E8M0 scales in TMEM)")
+        step_tf = tensor_fracs(ops, ms_step / 1e3, peaks)
         return {
             "value": whole_job_rate(world, wl.M, K, res["ms"]), "unit": UNIT, "ms_per_step": ms_step,
             "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "weights": "mxfp8 e4m3 + e8m0",
                        "block": 32},
             "roofline": roof,
-            "step": {"tflops": step_tflops, "tensor_frac_of_measured_bf16": step_tflops / bf16,
-                     "note": "step = MXFP8 quantisation of x (with its bf16 dequantisation), dequantisation of w, "
-                             "bf16 GEMM"},
+            "step": {"tops": step_tf["tops"], "tensor_frac_of_2x_measured_bf16": step_tf["frac_of_2x_measured_bf16"],
+                     "tensor_frac_of_datasheet": step_tf["frac_of_datasheet"],
+                     "note": "step = MXFP8 quantisation of x + block-scaled GEMM"},
             "e2e": {"value": whole_job_rate(world, wl.M, res["e2e_steps"], res["e2e_ms"]), "unit": UNIT,
                     "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"], "overlap": E2E_OVERLAP},
-            "gpu_launches": 3 * K,
+            "gpu_launches": 2 * K,
             "clocks": res["clocks"],
         }
     kind = "w4a8" if wl.fmt == "int4" else "w8a8"
@@ -894,7 +871,7 @@ def main():
     out = top_line(head, name, args, world)
     if name in synth.LINEAR_WORKLOADS:
         out["dtype"] = {"int4": "int8 (int4 weights unpacked to int8)", "int8": "int8",
-                        "mxfp8": "mxfp8 (e4m3 x e8m0, dequantised exactly to bf16)"}[wl.fmt]
+                        "mxfp8": "mxfp8 (e4m3 elements, e8m0 scales per 32)"}[wl.fmt]
     if subs:
         out["sub_results"] = subs
     if probe is not None:

@@ -283,23 +283,26 @@ int w8a8_mxfp8_quantize(const w8a8_bf16* x, int64_t R, int64_t K, uint8_t* codes
 size_t w8a8_mxfp8_linear_workspace_size(int64_t M, int64_t K, int64_t N);
 
 /* Defined by: the same row of the same table (MXFP8 A8W8: both operands in MXFP8).
- * Dense MXFP8 A8W8 linear: x is quantised to MXFP8 per token (w8a8_mxfp8_quantize), both
- * operands are dequantised to P * 2^E (exact in bf16) and multiplied on the tensor cores with fp32
- * accumulation: y[m, n] = bf16(sum_k A[m, k] W[n, k]), the sum of the exact products taken in the
- * tensor core's own order (so within (K - 1) * 2^-24 * sum_k |A W| of the exact sum before the
- * bf16 rounding).
- *   x bf16 [M, K]; w_codes uint8 [N, K] and w_scales uint8 [N, K/32] from w8a8_mxfp8_quantize;
- *   workspace of w8a8_mxfp8_linear_workspace_size() bytes (256-byte aligned; it receives x's
- *   codes at offset 0 and its scales after them, 256-byte aligned); y bf16 [M, N].
- * K % 64 == 0, N % 128 == 0 (else W8A8_ERR_UNSUPPORTED). */
+ * Dense MXFP8 A8W8 linear: x is quantised to MXFP8 per token (w8a8_mxfp8_quantize), then the
+ * block-scaled FP8 MMA of the tensor cores (tcgen05 kind::mxf8f6f4, one E8M0 scale per 32 values of
+ * K on both operands) sums the products of the dequantised values in fp32:
+ *   y[m, n] = bf16(sum_k (P_x[m,k] 2^Ex[m,k/32]) (P_w[n,k] 2^Ew[n,k/32])),
+ * in the tensor core's own summation order (within (K - 1) * 2^-24 * sum_k |products| of the exact
+ * sum before the bf16 rounding).
+ *   x bf16 [M, K] (16-byte aligned); w_codes uint8 [N, K] (16-byte aligned) and w_scales uint8
+ *   [N, K/32] (4-byte aligned) from w8a8_mxfp8_quantize; workspace of
+ *   w8a8_mxfp8_linear_workspace_size() bytes (256-byte aligned; it receives x's codes at offset 0
+ *   and its scales after them, 256-byte aligned); y bf16 [M, N].
+ * K % 128 == 0, N % 128 == 0 (else W8A8_ERR_UNSUPPORTED). */
 int w8a8_mxfp8_linear(const w8a8_bf16* x, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M, int64_t K,
                       int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y, w8a8_stream stream);
 
-/* The GEMM of w8a8_mxfp8_linear on operands already dequantised to bf16 (P * 2^E):
- *   a bf16 [M, K], w bf16 [N, K], y bf16 [M, N] = bf16(fp32 sum_k a[m, k] w[n, k]) on the tensor
- *   cores (kind::f16). Same shape rules as w8a8_mxfp8_linear; needs no workspace. */
-int w8a8_mxfp8_linear_dequantized(const w8a8_bf16* a, const w8a8_bf16* w, int64_t M, int64_t K, int64_t N,
-                                  w8a8_bf16* y, w8a8_stream stream);
+/* The GEMM of w8a8_mxfp8_linear on activations already in MXFP8 (for example from
+ * w8a8_mxfp8_quantize): x_codes uint8 [M, K] (16-byte aligned), x_scales uint8 [M, K/32] (4-byte
+ * aligned); the weights, y and the shape rules as w8a8_mxfp8_linear. Needs no workspace. */
+int w8a8_mxfp8_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, const uint8_t* w_codes,
+                               const uint8_t* w_scales, int64_t M, int64_t K, int64_t N, w8a8_bf16* y,
+                               w8a8_stream stream);
 
 /* Exact integer GEMM on the tensor cores: c[m, n] = sum_k a[m, k] * b[n, k] in int32: the
  * int8 x int8 product every W8A8 Linear of the group_0 scheme accumulates before its scales.

@@ -56,8 +56,8 @@ def test_workspace_queries_are_host_only(lib):
     assert B.w8a8_moe_workspace_size(64, 2048, 4, 8, 768) == 0  # k > E
     assert B.w8a8_linear_workspace_size(2048, 2048, 6144, 1, 64) == 0  # group != 128
     assert B.w8a8_linear_workspace_size(2048, 2048, 6144, 1, 128) > 0
-    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2048, 6144) >= 2048 * 2048 * (1 + 2) + 6144 * 2048 * 2
-    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2016, 6144) == 0  # K % 64
+    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2048, 6144) >= 2048 * 2048 + 2048 * 64
+    assert B.w8a8_mxfp8_linear_workspace_size(2048, 2112, 6144) == 0  # K % 128
     assert B.w8a8_mxfp8_linear_workspace_size(2048, 2048, 6100) == 0  # N % 128
 
 
@@ -82,8 +82,8 @@ def test_argument_checks_reject_before_any_launch(lib):
     assert lib.w8a8_mxfp8_quantize(None, 0, 64, None, None, None) == B.W8A8_OK  # empty
     assert lib.w8a8_mxfp8_linear(c(256), c(256), c(256), 8, 128, 256, c(256), 10, c(256), None) == \
         B.W8A8_ERR_WORKSPACE
-    assert lib.w8a8_mxfp8_linear(c(256), c(256), c(256), 8, 96, 256, c(256), 1 << 20, c(256), None) == \
-        B.W8A8_ERR_UNSUPPORTED  # K % 64
+    assert lib.w8a8_mxfp8_linear(c(256), c(256), c(256), 8, 192, 256, c(256), 1 << 20, c(256), None) == \
+        B.W8A8_ERR_UNSUPPORTED  # K % 128
     assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_debug_rcp_approx_ulp(0, 10, c(16), None) == B.W8A8_ERR_ARG  # not a normal input
     assert lib.w8a8_debug_rcp_approx_ulp(0x7E7FFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # reciprocal subnormal

@@ -75,7 +75,7 @@ SIGNATURES = {
     "w8a8_mxfp8_quantize": (_int, [_c_p, _i64, _i64, _c_p, _c_p, _c_p]),
     "w8a8_mxfp8_linear_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
     "w8a8_mxfp8_linear": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, ctypes.c_size_t, _c_p, _c_p]),
-    "w8a8_mxfp8_linear_dequantized": (_int, [_c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
+    "w8a8_mxfp8_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
     "w8a8_debug_rcp_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
     "w8a8_debug_ex2_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
@@ -398,29 +398,23 @@ def w8a8_mxfp8_linear(x, w_codes, w_scales, workspace=None, y=None, stream=None)
     return y
 
 
-def w8a8_mxfp8_linear_dequantized(a, w, y=None, stream=None):
-    """The GEMM of w8a8_mxfp8_linear on dequantised bf16 operands a [M, K], w [N, K]."""
-    _bf16(a), _bf16(w)
-    M, K = a.shape
-    N = w.shape[0]
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if y is None else y
-    _check(lib().w8a8_mxfp8_linear_dequantized(_ptr(a), _ptr(w), M, K, N, _ptr(y), _stream(stream)),
-           "w8a8_mxfp8_linear_dequantized")
+def w8a8_mxfp8_linear_prequant(x_codes, x_scales, w_codes, w_scales, y=None, stream=None):
+    """The GEMM of w8a8_mxfp8_linear on activations already in MXFP8 (codes [M, K], scales [M, K/32])."""
+    M, K = x_codes.shape
+    N = w_codes.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device) if y is None else y
+    _check(lib().w8a8_mxfp8_linear_prequant(_ptr(x_codes), _ptr(x_scales), _ptr(w_codes), _ptr(w_scales), M, K, N,
+                                            _ptr(y), _stream(stream)), "w8a8_mxfp8_linear_prequant")
     return y
 
 
-def mxfp8_linear_intermediates(workspace, M: int, K: int, N: int) -> dict:
-    """What w8a8_mxfp8_linear left in its workspace: x's MXFP8 codes [M, K] and scales [M, K/32],
-    and both dequantised operands, a bf16 [M, K] and w bf16 [N, K]."""
+def mxfp8_linear_intermediates(workspace, M: int, K: int) -> dict:
+    """x's MXFP8 codes [M, K] and scales [M, K/32] that w8a8_mxfp8_linear left in its workspace."""
     a256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
     codes = workspace[:M * K].view(M, K)
     off = a256(M * K)
     scales = workspace[off:off + M * (K // 32)].view(M, K // 32)
-    off += a256(M * (K // 32))
-    a = workspace[off:off + M * K * 2].view(torch.bfloat16).view(M, K)
-    off += a256(M * K * 2)
-    w = workspace[off:off + N * K * 2].view(torch.bfloat16).view(N, K)
-    return dict(codes=codes, scales=scales, a=a, w=w)
+    return dict(codes=codes, scales=scales)
 
 
 def w8a8_gemm_s8s8s32(a, b, c=None, stream=None):

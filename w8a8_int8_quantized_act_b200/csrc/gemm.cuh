@@ -30,7 +30,6 @@ enum EpiKind : int {
   kEpiGateUp = 2,   // int32 gate|up -> dequant, SiLU(gate)*up -> bf16 h
   kEpiDown = 3,     // int32 -> dequant -> bf16 o written to the assignment's slot row
   kEpiDense = 4,    // int32 -> dequant -> bf16 y (dense W8A8 linear)
-  kEpiDenseF32 = 5, // fp32 -> bf16 y (kind::f16 GEMM of dequantised MXFP8 operands)
 };
 
 constexpr int kBM = 128;            // MMA M (TMEM lanes)
@@ -298,24 +297,6 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
           uint16_t* o = out + size_t(orow[j]) * ldo;
           o[0] = uint16_t(v0[j]);
           if (second) o[kBM] = uint16_t(v1[j]);
-        }
-      }
-    }
-  } else if constexpr (EPI == kEpiDenseF32) {
-    // two 128-channel blocks of fp32 sums: y = bf16(acc), nothing else
-    const bool second = ch + kBM < p.n_channels;
-    uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
-    uint32_t r1[16];
-#pragma unroll 1
-    for (int j0 = half * 16; j0 < c.rows; j0 += 32) {
-      const int nj = min(16, c.rows - j0);
-      tmem_ld16x2(t_lane + j0, t_lane + NB + j0, r, r1);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j < nj) {
-          uint16_t* o = out + size_t(c.tok0 + j0 + j) * ldo;
-          o[0] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
-          if (second) o[kBM] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r1[j])));
         }
       }
     }

@@ -4,16 +4,13 @@
 //   E = floor(log2(max |v| over the block)) - 8, clamped to [-127, 127]; a block of zeros takes
 //       E = -127 (8 is the exponent of E4M3's largest binade, whose top value is 448);
 //   element = E4M3(v * 2^-E), nearest with ties to even, saturating at 448, sign kept at zero.
-// The dense MXFP8 linear multiplies the dequantised operands P * 2^E. Each of them is exact in
-// bf16 (at most 4 significant bits, and 2^E inside bf16's exponent range), and each product of two
-// is exact in fp32, so the tcgen05 kind::f16 MMA on the dequantised bf16 operands computes the MX
-// GEMM's sum of products with only its fp32 accumulation rounding; the block-scaled FP8 MMA would
-// compute the same sum at twice the rate.
+// The dense MXFP8 linear runs on the block-scaled FP8 MMA, which takes the codes and the E8M0
+// scales as they are and sums the products in fp32.
 #pragma once
-#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "elementwise.cuh"
+#include "gemm.cuh"
 
 namespace w8a8 {
 
@@ -33,35 +30,13 @@ __device__ __forceinline__ uint32_t e4m3_pair(float lo, float hi) {
   return uint32_t(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// 2^E as an fp32 value for E in [-127, 127] (2^-127 is the subnormal 0x00400000).
-__device__ __forceinline__ float pow2_f32(int E) {
-  return E >= -126 ? __int_as_float((E + 127) << 23) : __int_as_float(0x00400000);
-}
-
-// Eight elements of one block with the block's scale 2^E into bf16 values P * 2^E, packed. The
-// E4M3 -> fp16 conversion and the power-of-two product are exact.
-__device__ __forceinline__ uint4 mx_dequant8(uint2 codes, float scale) {
-  uint32_t out[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t w = (i < 2) ? codes.x : codes.y;
-    const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(__nv_fp8x2_storage_t((w >> ((i & 1) * 16)) & 0xFFFFu),
-                                                      __NV_E4M3);
-    const float2 f = __half22float2(__half2(h2));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(f.x, scale), __fmul_rn(f.y, scale));
-    out[i] = *reinterpret_cast<const uint32_t*>(&b);
-  }
-  return make_uint4(out[0], out[1], out[2], out[3]);
-}
-
-// codes [R, K] (E4M3 bytes), scales [R, K / 32] (E8M0 bytes) of the bf16 rows src [R, K], and,
-// when deq is not null, the dequantised values P * 2^E as bf16 [R, K]. K is a multiple of 32.
+// codes [R, K] (E4M3 bytes), scales [R, K / 32] (E8M0 bytes) of the bf16 rows src [R, K]. K is a
+// multiple of 32.
 // Lane l of a warp holds values 8l .. 8l+7 of its 256-value piece: block l / 4, four lanes each.
 __global__ void __launch_bounds__(kMxWarps * 32) mx_quant_rows_kernel(const uint16_t* __restrict__ src,
                                                                       int64_t R, int K,
                                                                       uint8_t* __restrict__ codes,
-                                                                      uint8_t* __restrict__ scales,
-                                                                      uint16_t* __restrict__ deq) {
+                                                                      uint8_t* __restrict__ scales) {
   pdl_wait();
   pdl_launch_dependents();
   const int pieces = (K + 255) / 256;
@@ -89,25 +64,262 @@ __global__ void __launch_bounds__(kMxWarps * 32) mx_quant_rows_kernel(const uint
   if (!valid) return;
   *reinterpret_cast<uint2*>(codes + r * K + k0) = make_uint2(c[0], c[1]);
   if ((lane & 3) == 0) scales[r * (K / kMxBlock) + k0 / kMxBlock] = uint8_t(E + 127);
-  if (deq != nullptr) *reinterpret_cast<uint4*>(deq + r * K + k0) = mx_dequant8(make_uint2(c[0], c[1]), pow2_f32(E));
 }
 
-// The dequantised bf16 values P * 2^(scale - 127) of MXFP8 rows (codes [R, K], scales [R, K / 32]).
-__global__ void __launch_bounds__(kMxWarps * 32) mx_dequant_rows_kernel(const uint8_t* __restrict__ codes,
-                                                                        const uint8_t* __restrict__ scales,
-                                                                        int64_t R, int K,
-                                                                        uint16_t* __restrict__ deq) {
-  pdl_wait();
+// ---------------------------------------------------------------- block-scaled MXFP8 GEMM
+// y[t, n] = bf16(sum_k (P_x[t,k] 2^Ex[t,k/32]) (P_w[n,k] 2^Ew[n,k/32])) with the block-scaled FP8
+// MMA (tcgen05.mma kind::mxf8f6f4.block_scale, scale_vec::1X: one E8M0 scale per 32 values of K
+// for every row of A and of B). Channels on the MMA's M side (128 weight rows), tokens on N (128).
+// A 128-byte K-block of FP8 codes is four MMAs of K = 32, i.e. four MX blocks, whose scales are
+// one 32-bit word per row: scales[r, 4kb .. 4kb+3], byte j for the j-th MMA.
+// Scale factors live in TMEM, per pipeline stage: SFA in 4 columns, SFB in 4 columns. Row
+// 32g + l of a 128-row operand sits in column g, at lane l of every lane quarter (each quarter of
+// the tensor core reads its own copy), byte j for K-block j of the four; the MMA names the byte
+// in the top two bits of the scale's TMEM address and in the instruction's scale-factor ids.
+// Roles per CTA (one per SM, 14 warps):
+//   warp 0      TMA producer: weight and token code blocks (128 rows x 128 bytes, 128-byte swizzle);
+//   warp 1      TMEM allocator and MMA issuer (one elected thread);
+//   warps 2-5   scale writers, one per TMEM lane quarter: each stage's scale words from global
+//               memory into the stage's scale columns of their quarter (tcgen05.st);
+//   warps 6-13  epilogue: fp32 sums -> bf16 y, two warps per lane quarter.
+// Every wait is bounded (ptx.cuh).
+struct MxGemmParams {
+  CUtensorMap tmA;     // weight codes [N, K] bytes, box 128 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap tmB;     // token codes [M, K] bytes, the same box
+  const uint32_t* sfa; // weight scales [N, K/32] bytes, read as words [N, K/128]
+  const uint32_t* sfb; // token scales [M, K/32] bytes, read as words [M, K/128]
+  int num_kb;          // K / 128
+  int n_cb;            // N / 128
+  int M;
+  int N;
+  uint16_t* y;         // [M, N] bf16
+  uint64_t timeout_ns;
+};
+
+constexpr int kMxNB = 128;                          // tokens per tile (MMA N)
+constexpr int kMxStages = 6;
+constexpr int kMxSfAhead = 4;                       // scale-word prefetch depth (stages)
+constexpr int kMxStageBytes = 2 * kBM * kKBlockBytes;  // weight block + token block
+constexpr int kMxAccCols = kMxNB;                   // one accumulator set
+constexpr uint32_t kMxSfCol0 = 2 * kMxAccCols;      // scale columns: 8 per stage after both sets
+constexpr int kMxTmemCols = 512;
+constexpr int kMxThreads = 32 * 14;
+constexpr size_t kMxSmemBytes = 1024 + size_t(kMxStages) * kMxStageBytes + 512;
+static_assert(kMxSfCol0 + 8 * kMxStages <= kMxTmemCols, "accumulators and scale columns fit in TMEM");
+
+// Instruction descriptor of the block-scaled MMA: A and B E4M3 (format 0), both K-major, fp32
+// accumulation, M = 128, N = n, E8M0 scales (bit 23), scale-factor ids of A (bits 29-30) and B
+// (bits 4-5) = j.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int n, uint32_t j) {
+  return (j << 4) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(128 >> 4) << 24) | (j << 29);
+}
+
+__device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 4 consecutive 32-bit TMEM columns of the warp's 32 lanes from registers (no wait).
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d));
+}
+
+__global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_constant__ MxGemmParams p) {
+  constexpr int S = kMxStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kMxStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* sfready = empty + S;
+  uint64_t* tfull = sfready + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const WaitCtx wc{abort_flag, p.timeout_ns};
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); mbar_init(sfready + s, 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, 8); }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+    tma_prefetch_map(&p.tmA);
+    tma_prefetch_map(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kMxTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();  // the token codes and scales come from the quantisation kernel launched just before
   pdl_launch_dependents();
-  const int pieces = (K + 255) / 256;
-  const int64_t item = int64_t(blockIdx.x) * kMxWarps + (threadIdx.x >> 5);
-  if (item >= R * pieces) return;
-  const int64_t r = item / pieces;
-  const int k0 = int(item - r * pieces) * 256 + (threadIdx.x & 31) * 8;
-  if (k0 >= K) return;
-  const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + r * K + k0));
-  const int E = int(__ldg(scales + r * (K / kMxBlock) + k0 / kMxBlock)) - 127;
-  *reinterpret_cast<uint4*>(deq + r * K + k0) = mx_dequant8(c, pow2_f32(E));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int m_tiles = (p.M + kMxNB - 1) / kMxNB;
+  const int total = m_tiles * p.n_cb;
+  const int nkb = p.num_kb;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, parity = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+        if (elect_one()) {
+          uint8_t* st = smem + stage * kMxStageBytes;
+          mbar_arrive_expect_tx(full + stage, uint32_t(kMxStageBytes));
+          tma_load_2d(st, &p.tmA, full + stage, kb * kKBlockBytes, cb * kBM);
+          tma_load_2d(st + kBM * kKBlockBytes, &p.tmB, full + stage, kb * kKBlockBytes, mt * kMxNB);  // rows past M: zeros
+        }
+        __syncwarp();
+        issued |= 1u << stage;
+        parity = (parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (lane == 0 && *abort_flag) {  // loads already issued land before the CTA exits
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, 100000000ull};
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) mbar_wait(full + s, (parity >> s) & 1u, dw);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint64_t adesc0 = sw128_kmajor_desc(smem_addr(smem));
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool issued_any = false, ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + uint32_t(acc * kMxAccCols);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_warp(full + stage, phase, wc)) { ok = false; break; }
+        if (!mbar_wait_warp(sfready + stage, phase, wc)) { ok = false; break; }
+        tc_fence_after();  // the scale columns written by the scale warps (tcgen05.st) precede
+        if (elect_one()) {
+          const uint64_t ad = adesc0 + uint64_t(stage * (kMxStageBytes >> 4));
+          const uint64_t bd = ad + uint64_t((kBM * kKBlockBytes) >> 4);
+          const uint32_t sf = tmem_base + kMxSfCol0 + uint32_t(8 * stage);
+#pragma unroll
+          for (uint32_t j = 0; j < 4; ++j)
+            tc_mma_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8(kMxNB, j), sf + (j << 30),
+                        sf + 4u + (j << 30), (kb | int(j)) != 0 ? 1u : 0u);
+          tc_commit(empty + stage);
+        }
+        __syncwarp();
+        issued_any = true;
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (elect_one()) tc_commit(tfull + acc);
+      __syncwarp();
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0 && *abort_flag && issued_any) {
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, 100000000ull};
+      mbar_wait(drain, 0, dw);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ scale writers (one per quarter)
+    // The scale words of a stage are loaded from global memory kMxSfAhead stages before they are
+    // written, so their latency overlaps the MMAs of the stages in between.
+    constexpr int D = kMxSfAhead;
+    const int q = warp & 3;
+    const uint32_t lane_off = uint32_t(q * 32) << 16;
+    const int wpr = nkb;  // scale words per row
+    const int my_tiles = int(blockIdx.x) < total ? (total - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    const int n = my_tiles * nkb;  // this CTA's (tile, K-block) items in order
+    // rows 32g + lane of A (channels) and of B (tokens) of item i; tokens past M take scale word 0
+    auto load = [&](int i, uint32_t (&a)[4], uint32_t (&b)[4]) {
+      const int tile = int(blockIdx.x) + (i / nkb) * int(gridDim.x), kb = i % nkb;
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      const int c0 = cb * kBM, t0 = mt * kMxNB;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        a[g] = __ldg(p.sfa + size_t(c0 + 32 * g + lane) * wpr + kb);
+        const int t = t0 + 32 * g + lane;
+        b[g] = t < p.M ? __ldg(p.sfb + size_t(t) * wpr + kb) : 0u;
+      }
+    };
+    uint32_t ra[D][4], rb[D][4];
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+      if (d < n) load(d, ra[d], rb[d]);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int i0 = 0; i0 < n && ok; i0 += D) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        const int i = i0 + d;
+        if (i >= n) break;
+        // the MMAs that read this stage's previous scales have completed
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+        const uint32_t col = tmem_base + lane_off + kMxSfCol0 + uint32_t(8 * stage);
+        tmem_st4(col, ra[d][0], ra[d][1], ra[d][2], ra[d][3]);
+        tmem_st4(col + 4u, rb[d][0], rb[d][1], rb[d][2], rb[d][3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sfready + stage);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+        if (i + D < n) load(i + D, ra[d], rb[d]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 6-13)
+    const int q = warp & 3;
+    const int half = (warp - 6) >> 2;  // token columns [64 half, 64 half + 64)
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      const int t0 = mt * kMxNB;
+      const int ch = cb * kBM + q * 32 + lane;  // this lane's output channel
+      if (!mbar_wait_warp(tfull + acc, acc_phase, wc)) break;
+      tc_fence_after();
+      const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kMxAccCols);
+      uint16_t* out = p.y + ch;
+#pragma unroll 1
+      for (int j0 = half * 64; j0 < half * 64 + 64; j0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(t_lane + uint32_t(j0), r);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (t0 + j0 + j < p.M)
+            out[size_t(t0 + j0 + j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kMxTmemCols);
+  }
 }
 
 }  // namespace w8a8

@@ -328,37 +328,34 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
 }
 
 // Launches quant_rows_kernel with the register depth that fits rows of K values.
-// MXFP8 rows: quantise src (codes, scales, and the dequantised bf16 values when deq is not null),
-// or, with src null, dequantise in_codes / in_scales into deq.
-int launch_mx_rows(const w8a8_bf16* src, const uint8_t* in_codes, const uint8_t* in_scales, int64_t R, int K,
-                   uint8_t* codes, uint8_t* scales, uint16_t* deq, cudaStream_t s) {
+// MXFP8 codes and scales of the bf16 rows src [R, K].
+int launch_mx_rows(const w8a8_bf16* src, int64_t R, int K, uint8_t* codes, uint8_t* scales, cudaStream_t s) {
   const int64_t items = R * ((K + 255) / 256);
   const dim3 grid(unsigned((items + kMxWarps - 1) / kMxWarps));
-  if (src != nullptr)
-    return launch_pdl(mx_quant_rows_kernel, grid, dim3(kMxWarps * 32), 0, s, reinterpret_cast<const uint16_t*>(src),
-                      R, K, codes, scales, deq);
-  return launch_pdl(mx_dequant_rows_kernel, grid, dim3(kMxWarps * 32), 0, s, in_codes, in_scales, R, K, deq);
+  return launch_pdl(mx_quant_rows_kernel, grid, dim3(kMxWarps * 32), 0, s, reinterpret_cast<const uint16_t*>(src), R,
+                    K, codes, scales);
 }
 
-// y [M, N] = bf16(a [M, K] . w [N, K]^T) for bf16 operands (the dequantised MXFP8 values): the
-// one-CTA tcgen05 GEMM with kind::f16, channels on the MMA's M side, fp32 accumulators.
-int mx_gemm(const uint16_t* a, const uint16_t* w, int64_t M, int64_t K, int64_t N, w8a8_bf16* y, cudaStream_t s) {
-  GemmParams p{};
-  if (!make_kmajor_map(&p.tmA, w, true, K, N, 128) || !make_kmajor_map(&p.tmB, a, true, K, M, kBBoxRows) ||
-      !make_kmajor_map(&p.tmB2, a, true, K, M, 128))
+// y [M, N] = the MXFP8 product of token codes / scales and weight codes / scales on the
+// block-scaled FP8 MMA (mx_gemm_kernel). K % 128 == 0, N % 128 == 0; checked by the callers.
+int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8_t* ws, int64_t M, int64_t K,
+            int64_t N, w8a8_bf16* y, cudaStream_t s) {
+  MxGemmParams p{};
+  if (!make_kmajor_map(&p.tmA, wc, false, K, N, 128) || !make_kmajor_map(&p.tmB, xc, false, K, M, 128))
     return W8A8_ERR_UNSUPPORTED;
-  p.num_kb = int(K / 64);  // 128-byte K-blocks of bf16
-  p.n_cb = int((N + 255) / 256);
-  p.n_channels = int(N);
-  p.num_groups = 1;
+  p.sfa = reinterpret_cast<const uint32_t*>(ws);
+  p.sfb = reinterpret_cast<const uint32_t*>(xs);
+  p.num_kb = int(K / 128);
+  p.n_cb = int(N / 128);
   p.M = int(M);
-  p.a_second_offset = 128;
-  p.a_cb_step = 256;
+  p.N = int(N);
+  p.y = reinterpret_cast<uint16_t*>(y);
   p.timeout_ns = wait_timeout_ns();
-  p.out = y;
-  p.ldo = int(N);
-  const int tiles = int((M + 127) / 128) * p.n_cb;
-  return launch_gemm<2, 128, kEpiDenseF32, kKindBF16>(p, tiles, s);
+  if (cudaFuncSetAttribute(mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMxSmemBytes)) !=
+      cudaSuccess)
+    return W8A8_ERR_LAUNCH;
+  const int tiles = int((M + kMxNB - 1) / kMxNB) * p.n_cb;
+  return launch_pdl(mx_gemm_kernel, dim3(max(1, min(num_sms(), tiles))), dim3(kMxThreads), kMxSmemBytes, s, p);
 }
 
 int launch_quant_rows(const uint16_t* src, int64_t R, int K, int8_t* q, float* scale, cudaStream_t s) {
@@ -1138,14 +1135,14 @@ int w8a8_mxfp8_quantize(const w8a8_bf16* x, int64_t R, int64_t K, uint8_t* codes
   if (R == 0) return W8A8_OK;
   if (!x || !codes || !scales) return W8A8_ERR_ARG;
   if (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 7u)) return W8A8_ERR_UNSUPPORTED;
-  return launch_mx_rows(x, nullptr, nullptr, R, int(K), codes, scales, nullptr, as_stream(stream));
+  return launch_mx_rows(x, R, int(K), codes, scales, as_stream(stream));
 }
 
 size_t w8a8_mxfp8_linear_workspace_size(int64_t M, int64_t K, int64_t N) {
-  if (M < 0 || K <= 0 || N <= 0 || K % 64 || N % 128) return 0;
+  if (M < 0 || K <= 0 || N <= 0 || K % 128 || N % 128) return 0;
   if (K > (int64_t(1) << 24) || N > (int64_t(1) << 24) || M >= (int64_t(1) << 30)) return 0;
   const size_t m = size_t(M > 0 ? M : 1);
-  return align256(m * K) + align256(m * K / kMxBlock) + align256(m * K * 2) + align256(size_t(N) * K * 2);
+  return align256(m * K) + align256(m * K / kMxBlock);
 }
 
 int w8a8_mxfp8_linear(const w8a8_bf16* x, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M, int64_t K,
@@ -1156,31 +1153,28 @@ int w8a8_mxfp8_linear(const w8a8_bf16* x, const uint8_t* w_codes, const uint8_t*
   if (M == 0) return W8A8_OK;
   if (!x || !w_codes || !w_scales || !y || !workspace) return W8A8_ERR_ARG;
   if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
-  if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(w_codes) & 7u) ||
+  if (!aligned16(x) || !aligned16(y) || !aligned16(w_codes) || (reinterpret_cast<uintptr_t>(w_scales) & 3u) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return W8A8_ERR_UNSUPPORTED;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* xc = ws;
+  uint8_t* xc = static_cast<uint8_t*>(workspace);
   uint8_t* xs = xc + align256(size_t(M) * K);
-  uint16_t* xd = reinterpret_cast<uint16_t*>(xs + align256(size_t(M) * K / kMxBlock));
-  uint16_t* wdq = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(xd) + align256(size_t(M) * K * 2));
   const cudaStream_t s = as_stream(stream);
-  int rc = launch_mx_rows(x, nullptr, nullptr, M, int(K), xc, xs, xd, s);  // x: codes, scales, P * 2^E
+  const int rc = launch_mx_rows(x, M, int(K), xc, xs, s);
   if (rc != W8A8_OK) return rc;
-  rc = launch_mx_rows(nullptr, w_codes, w_scales, N, int(K), nullptr, nullptr, wdq, s);  // w: P * 2^E
-  if (rc != W8A8_OK) return rc;
-  return mx_gemm(xd, wdq, M, K, N, y, s);
+  return mx_gemm(xc, xs, w_codes, w_scales, M, K, N, y, s);
 }
 
-int w8a8_mxfp8_linear_dequantized(const w8a8_bf16* a, const w8a8_bf16* w, int64_t M, int64_t K, int64_t N,
-                                  w8a8_bf16* y, w8a8_stream stream) {
+int w8a8_mxfp8_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, const uint8_t* w_codes,
+                               const uint8_t* w_scales, int64_t M, int64_t K, int64_t N, w8a8_bf16* y,
+                               w8a8_stream stream) {
   if (M < 0 || K <= 0 || N <= 0) return W8A8_ERR_ARG;
   if (w8a8_mxfp8_linear_workspace_size(M, K, N) == 0) return W8A8_ERR_UNSUPPORTED;
   if (M == 0) return W8A8_OK;
-  if (!a || !w || !y) return W8A8_ERR_ARG;
-  if (!aligned16(a) || !aligned16(w) || !aligned16(y)) return W8A8_ERR_UNSUPPORTED;
-  return mx_gemm(reinterpret_cast<const uint16_t*>(a), reinterpret_cast<const uint16_t*>(w), M, K, N, y,
-                 as_stream(stream));
+  if (!x_codes || !x_scales || !w_codes || !w_scales || !y) return W8A8_ERR_ARG;
+  if (!aligned16(x_codes) || !aligned16(w_codes) || !aligned16(y) || (reinterpret_cast<uintptr_t>(x_scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(w_scales) & 3u))
+    return W8A8_ERR_UNSUPPORTED;
+  return mx_gemm(x_codes, x_scales, w_codes, w_scales, M, K, N, y, as_stream(stream));
 }
 
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {
