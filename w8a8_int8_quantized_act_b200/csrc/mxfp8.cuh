@@ -97,7 +97,7 @@ struct MxGemmParams {
 };
 
 constexpr int kMxNB = 128;                          // tokens per tile (MMA N)
-constexpr int kMxStages = 6;
+constexpr int kMxStages = 7;
 constexpr int kMxSfAhead = 4;                       // scale-word prefetch depth (stages)
 constexpr int kMxStageBytes = 2 * kBM * kKBlockBytes;  // weight block + token block
 constexpr int kMxAccCols = kMxNB;                   // one accumulator set
