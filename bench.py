@@ -590,6 +590,9 @@ MEASURED_TRAFFIC = {
     # the W4A8 GEMM launch of the 2048 x 2048 -> 6144 linear: 10.9 MB read (weights, scales, token
     # codes once), nothing written back to DRAM within the launch (the 25 MB output stays in L2)
     "qwen3-1.7b-mlp-w4a8": (10_933_760 + 0, "1b4b2dc7d15bec2e91ed021dfeeca923eb8d5b51"),
+    # the block-scaled MXFP8 GEMM launch of the same shape: 17.3 MB read (FP8 weights and scales,
+    # token codes and scales, each once), 1.5 KB written back within the launch
+    "qwen3-1.7b-mlp-mxfp8": (17_346_304 + 1_536, "4a2b6e44df235a8e6e82bd6525612b372f14f632"),
 }
 TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
