@@ -11,6 +11,7 @@
 
 #include "elementwise.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 
 namespace w8a8 {
 
@@ -319,6 +320,283 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_con
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kMxTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- the same GEMM on CTA pairs
+// Tiles of 256 channels x 192 tokens on the two CTAs of a cluster with M = 256 block-scaled MMAs
+// (cta_group::2): rank r supplies its 128 weight rows and 96 of the token rows, and receives the
+// sums of its 128 channels for all 192 tokens, so per SM and K-block 16 + 12 KB of codes feed
+// 128 x 192 x 128 MACs (the one-CTA tile moves 32 KB for 128 x 128 x 128). Each rank keeps in its
+// TMEM, per stage and laid out like the one-CTA kernel's, the scales of its own 128 weight rows
+// (4 columns) and those of all 192 token rows of the tile (6 columns): each CTA's half of the
+// tensor core scales every column of its accumulators. (Holding only the 96 token rows a rank
+// supplies gives wrong sums for the other half of the columns.)
+struct MxPairParams {
+  CUtensorMap tmA;     // weight codes [N, K], box 128 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap tmB;     // token codes [M, K], box 96 rows x 128 bytes, 128-byte swizzle
+  const uint32_t* sfa; // weight scales as words [N, K/128]
+  const uint32_t* sfb; // token scales as words [M, K/128]
+  int num_kb;          // K / 128
+  int n_cb;            // N / 256
+  int M;
+  int N;
+  uint16_t* y;         // [M, N] bf16
+  uint64_t timeout_ns;
+};
+
+constexpr int kMxPairNB = 192;                 // tokens per tile (MMA N)
+constexpr int kMxPairHalf = kMxPairNB / 2;     // token rows each rank loads
+constexpr int kMxPairStages = 7;
+constexpr int kMxPairABytes = kBM * kKBlockBytes;
+constexpr int kMxPairBBytes = kMxPairHalf * kKBlockBytes;
+constexpr int kMxPairStageBytes = kMxPairABytes + kMxPairBBytes;
+constexpr uint32_t kMxPairSfCol0 = 2 * kMxPairNB;  // after both accumulator sets
+constexpr int kMxPairSfCols = 12;                  // per stage: SFA 4 + SFB 6 (+ 2 of padding)
+constexpr int kMxPairThreads = 32 * 14;
+constexpr size_t kMxPairSmemBytes = 1024 + size_t(kMxPairStages) * kMxPairStageBytes + 512;
+static_assert(kMxPairSfCol0 + kMxPairSfCols * kMxPairStages <= 512, "accumulators and scales fit in TMEM");
+static_assert(kMxPairBBytes % 1024 == 0, "128-byte swizzled token rows sit on 1 KB boundaries");
+
+__host__ __device__ constexpr uint32_t idesc_mxf8_m256(int n, uint32_t j) {
+  return (j << 4) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(256 >> 4) << 24) | (j << 29);
+}
+
+__device__ __forceinline__ void tc_mma_pair_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
+    mx_pair_kernel(const __grid_constant__ MxPairParams p) {
+  constexpr int S = kMxPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kMxPairStageBytes);  // used on rank 0
+  uint64_t* empty = full + S;                                                  // each rank
+  uint64_t* sfready = empty + S;                                               // used on rank 0
+  uint64_t* tfull = sfready + S;                                               // each rank, [2]
+  uint64_t* tempty = tfull + 2;                                                // used on rank 0, [2]
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = int(cluster_index());
+  const int nclusters = int(cluster_count());
+  const WaitCtx wc{abort_flag, p.timeout_ns};
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); mbar_init(sfready + s, 8); }
+    for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, 16); }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+    tma_prefetch_map(&p.tmA);
+    tma_prefetch_map(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  pdl_wait();  // the token codes and scales come from the quantisation kernel launched just before
+  pdl_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int m_tiles = (p.M + kMxPairNB - 1) / kMxPairNB;
+  const int total = m_tiles * p.n_cb;
+  const int nkb = p.num_kb;
+  const int my_tiles = cluster < total ? (total - cluster + nclusters - 1) / nclusters : 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both ranks)
+    const uint32_t full0 = map_to_rank(smem_addr(full), 0);
+    int stage = 0;
+    uint32_t phase = 0, issued = 0, parity = 0;
+    bool ok = true;
+    for (int tile = cluster; tile < total && ok; tile += nclusters) {
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+        if (elect_one()) {
+          uint8_t* st = smem + stage * kMxPairStageBytes;
+          const uint32_t bar = full0 + uint32_t(stage) * 8u;
+          if (leader) mbar_arrive_expect_tx(full + stage, 2u * uint32_t(kMxPairStageBytes));
+          tma_load_2d_pair(st, &p.tmA, bar, kb * kKBlockBytes, cb * 256 + int(rank) * 128);
+          tma_load_2d_pair(st + kMxPairABytes, &p.tmB, bar, kb * kKBlockBytes,
+                           mt * kMxPairNB + int(rank) * kMxPairHalf);  // rows past M: zeros
+        }
+        __syncwarp();
+        issued |= 1u << stage;
+        parity = (parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (ok) {
+      // every stage released by the MMAs (their completions reach this CTA) before exit
+      for (int i = 0; i < S; ++i) {
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) break;
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int no_abort = 0;
+      const WaitCtx dw{&no_abort, 100000000ull};
+      if (leader) {
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s)) mbar_wait(full + s, (parity >> s) & 1u, dw);
+      } else {
+        const uint64_t until = globaltimer_ns() + 1000000ull;
+        while (globaltimer_ns() < until) __nanosleep(10000);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (rank 0)
+    if (leader) {
+      const uint32_t empty_own = smem_addr(empty), empty_peer = map_to_rank(smem_addr(empty), 1);
+      const uint32_t tfull_own = smem_addr(tfull), tfull_peer = map_to_rank(smem_addr(tfull), 1);
+      const uint64_t adesc0 = sw128_kmajor_desc(smem_addr(smem));
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool issued_any = false, ok = true;
+      for (int t = 0; t < my_tiles && ok; ++t) {
+        if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(acc * kMxPairNB);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_warp(full + stage, phase, wc)) { ok = false; break; }
+          if (!mbar_wait_warp(sfready + stage, phase, wc)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
+            const uint64_t ad = adesc0 + uint64_t(stage * (kMxPairStageBytes >> 4));
+            const uint64_t bd = ad + uint64_t(kMxPairABytes >> 4);
+            const uint32_t sf = tmem_base + kMxPairSfCol0 + uint32_t(kMxPairSfCols * stage);
+#pragma unroll
+            for (uint32_t j = 0; j < 4; ++j)
+              tc_mma_pair_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8_m256(kMxPairNB, j),
+                               sf + (j << 30), sf + 4u + (j << 30), (kb | int(j)) != 0 ? 1u : 0u);
+            tc_commit_pair(empty_own + uint32_t(stage) * 8u);
+            tc_commit_pair(empty_peer + uint32_t(stage) * 8u);
+          }
+          __syncwarp();
+          issued_any = true;
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (elect_one()) {
+          tc_commit_pair(tfull_own + uint32_t(acc) * 8u);
+          tc_commit_pair(tfull_peer + uint32_t(acc) * 8u);
+        }
+        __syncwarp();
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (ok && !*abort_flag) {
+        for (int i = 0; i < 2; ++i) {
+          if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) break;
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+      }
+      if (lane == 0 && *abort_flag && issued_any) {
+        tc_commit_pair(smem_addr(drain));
+        volatile int no_abort = 0;
+        const WaitCtx dw{&no_abort, 100000000ull};
+        mbar_wait(drain, 0, dw);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ scale writers (both ranks)
+    constexpr int D = kMxSfAhead;
+    const int q = warp & 3;
+    const uint32_t lane_off = uint32_t(q * 32) << 16;
+    const uint32_t sfready0 = map_to_rank(smem_addr(sfready), 0);
+    const int wpr = nkb;
+    const int n = my_tiles * nkb;
+    auto load = [&](int i, uint32_t (&a)[4], uint32_t (&b)[6]) {
+      const int tile = cluster + (i / nkb) * nclusters, kb = i % nkb;
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      const int c0 = cb * 256 + int(rank) * 128, t0 = mt * kMxPairNB;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) a[g] = __ldg(p.sfa + size_t(c0 + 32 * g + lane) * wpr + kb);
+#pragma unroll
+      for (int g = 0; g < 6; ++g) {
+        const int t = t0 + 32 * g + lane;
+        b[g] = t < p.M ? __ldg(p.sfb + size_t(t) * wpr + kb) : 0u;
+      }
+    };
+    uint32_t ra[D][4], rb[D][6];
+#pragma unroll
+    for (int d = 0; d < D; ++d)
+      if (d < n) load(d, ra[d], rb[d]);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int i0 = 0; i0 < n && ok; i0 += D) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) {
+        const int i = i0 + d;
+        if (i >= n) break;
+        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
+        const uint32_t col = tmem_base + lane_off + kMxPairSfCol0 + uint32_t(kMxPairSfCols * stage);
+        tmem_st4(col, ra[d][0], ra[d][1], ra[d][2], ra[d][3]);
+        tmem_st4(col + 4u, rb[d][0], rb[d][1], rb[d][2], rb[d][3]);
+        tmem_st4(col + 8u, rb[d][4], rb[d][5], 0u, 0u);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(sfready0 + uint32_t(stage) * 8u);
+        if (++stage == S) { stage = 0; phase ^= 1u; }
+        if (i + D < n) load(i + D, ra[d], rb[d]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both ranks)
+    const int q = warp & 3;
+    const int half = (warp - 6) >> 2;  // token columns [96 half, 96 half + 96)
+    const uint32_t tempty0 = map_to_rank(smem_addr(tempty), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster; tile < total; tile += nclusters) {
+      const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
+      const int t0 = mt * kMxPairNB;
+      const int ch = cb * 256 + int(rank) * 128 + q * 32 + lane;
+      if (!mbar_wait_warp(tfull + acc, acc_phase, wc)) break;
+      tc_fence_after();
+      const uint32_t t_lane = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kMxPairNB);
+      uint16_t* out = p.y + ch;
+#pragma unroll 1
+      for (int j0 = half * kMxPairHalf; j0 < half * kMxPairHalf + kMxPairHalf; j0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(t_lane + uint32_t(j0), r);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (t0 + j0 + j < p.M)
+            out[size_t(t0 + j0 + j) * p.N] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[j])));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 

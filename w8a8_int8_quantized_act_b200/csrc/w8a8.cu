@@ -336,10 +336,32 @@ int launch_mx_rows(const w8a8_bf16* src, int64_t R, int K, uint8_t* codes, uint8
                     K, codes, scales);
 }
 
+// MXFP8 GEMMs with more token rows than this (and N a multiple of 256) run on CTA pairs.
+constexpr int64_t kMxPairMinRows = 192;
+
 // y [M, N] = the MXFP8 product of token codes / scales and weight codes / scales on the
 // block-scaled FP8 MMA (mx_gemm_kernel). K % 128 == 0, N % 128 == 0; checked by the callers.
 int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8_t* ws, int64_t M, int64_t K,
             int64_t N, w8a8_bf16* y, cudaStream_t s) {
+  if (M > kMxPairMinRows && N % 256 == 0) {
+    MxPairParams q{};
+    if (!make_kmajor_map(&q.tmA, wc, false, K, N, 128) || !make_kmajor_map(&q.tmB, xc, false, K, M, kMxPairHalf))
+      return W8A8_ERR_UNSUPPORTED;
+    q.sfa = reinterpret_cast<const uint32_t*>(ws);
+    q.sfb = reinterpret_cast<const uint32_t*>(xs);
+    q.num_kb = int(K / 128);
+    q.n_cb = int(N / 256);
+    q.M = int(M);
+    q.N = int(N);
+    q.y = reinterpret_cast<uint16_t*>(y);
+    q.timeout_ns = wait_timeout_ns();
+    auto kern = mx_pair_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMxPairSmemBytes)) != cudaSuccess)
+      return W8A8_ERR_LAUNCH;
+    const int tiles = int((M + kMxPairNB - 1) / kMxPairNB) * q.n_cb;
+    const int clusters = max(1, min(num_sms() / 2, tiles));
+    return launch_pdl(kern, dim3(2 * clusters), dim3(kMxPairThreads), kMxPairSmemBytes, s, q);
+  }
   MxGemmParams p{};
   if (!make_kmajor_map(&p.tmA, wc, false, K, N, 128) || !make_kmajor_map(&p.tmB, xc, false, K, M, 128))
     return W8A8_ERR_UNSUPPORTED;
