@@ -1,4 +1,4 @@
-"""CPU oracle for the W8A8 INT8 MoE expert-FFN forward and the dense W8A8/W4A8/MXFP8 linear.
+"""CPU oracle for the W8A8 INT8 MoE expert-FFN forward and the dense W8A8/W4A8/MXFP linears.
 
 TEST INFRASTRUCTURE. This module is the slow, plain statement of what the GPU path must
 compute. Only the test-suite, the smoke check and the CPU-baseline leg of the benchmark
@@ -56,6 +56,10 @@ Readings where the pages are silent (each one is fixed identically on the GPU si
   elements; E = floor(log2 amax) - 8, elements rounded to nearest even and saturated at 448. The
   layer's product is the exact sum of the dequantised products; the GPU's fp32 sum of the same
   products is checked within the summation bound (see ``linear_mxfp8``).
+* MXFP A8W4 (the same table's "MXFP A8w4" row): MXFP8 activations as above and MXFP4 weights, the
+  OCP format with E2M1 elements: E = floor(log2 amax) - 2, elements rounded to nearest even and
+  saturated at 6, two codes per byte with the even element in the low nibble (see
+  ``mx4_quantize_rows``).
 """
 from __future__ import annotations
 
@@ -604,6 +608,106 @@ def linear_mxfp8(x_bits, w_codes, w_scales) -> dict:
     xc, xs = mx_quantize_rows(x_bits)
     A = mx_dequantize(xc, xs)
     W = mx_dequantize(w_codes, w_scales)
+    y = A @ W.T
+    K = A.shape[1]
+    S = np.abs(A) @ np.abs(W).T
+    summ = (K - 1) * 2.0 ** -24 * S
+    bound = summ + 2.0 ** -8 * (np.abs(y) + summ)
+    return dict(codes=xc, scales=xs, y=y, bound=bound)
+
+
+# --------------------------------------------------------------------------------------
+# MXFP A8W4 (the "MXFP A8w4" row of the same accuracy table): MXFP8 activations, MXFP4 weights
+# --------------------------------------------------------------------------------------
+# Read, like the A8W8 row, as the OCP Microscaling formats: the activations exactly as above
+# (MXFP8, E4M3 elements), the weights as MXFP4: blocks of 32 consecutive values along K with one
+# E8M0 scale X = 2**E and FP4 E2M1 elements (1 sign, 2 exponent bits with bias 1, 1 mantissa bit;
+# exponent field 0 holds the subnormal 0.5; the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6; no
+# infinities or NaNs).
+#   E = floor(log2(max |v| over the block)) - 2 (2 is the exponent of E2M1's largest binade),
+#       clamped to [-127, 127]; a block of zeros takes E = -127;
+#   P = E2M1(v / 2**E), rounded to nearest with ties to the even mantissa, magnitudes above 6
+#       saturating to 6 (the block's largest element lands in [4, 8), so values in (6, 8) clip);
+#       the sign of a value that rounds to zero is kept (code 0x8).
+# Storage: two codes per byte, element 2i in the low nibble of byte i and element 2i + 1 in the
+# high nibble (a weight row of K values takes K / 2 bytes).
+# The product is y[t, n] = sum_k (P_x[t,k] X_x[t,k/32]) (P_w[n,k] X_w[n,k/32]), exact here, checked
+# on the GPU within the same fp32 summation bound as the A8W8 product.
+E2M1_MAX = 6.0
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """float64 value of each E2M1 code (the low four bits of each byte)."""
+    c = np.asarray(codes, np.uint8).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = (c & 1).astype(np.float64)
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.exp2(e.astype(np.float64) - 1.0))
+    return sign * mag
+
+
+# non-negative E2M1 values in increasing order; the code of each is its index
+_E2M1_POS_VALUES = e2m1_decode(np.arange(8, dtype=np.uint8))
+
+
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    """E2M1 code (0..15) of each finite float64 value: nearest representable magnitude, ties to the
+    even mantissa, saturating at 6; negative values (and -0) carry the sign bit 0x8."""
+    v = np.asarray(v, np.float64)
+    a = np.minimum(np.abs(v), E2M1_MAX)
+    # the quantum of the binade that holds a: 2**(e - 1) for e = floor(log2 a) >= 0; below 1 the
+    # subnormal quantum 0.5, the same as that of [1, 2)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = np.maximum(ex - 1, 0)
+    q = np.exp2(e.astype(np.float64) - 1.0)
+    n = np.rint(a / q)                        # a / q is exact; rint rounds halves to even
+    mag = np.minimum(n * q, E2M1_MAX)
+    idx = np.searchsorted(_E2M1_POS_VALUES, mag)
+    assert np.all(_E2M1_POS_VALUES[idx] == mag)
+    code = idx.astype(np.uint8)
+    return np.where(np.signbit(v), code | np.uint8(0x8), code).astype(np.uint8)
+
+
+def mx4_quantize_rows(v_bits: np.ndarray):
+    """MXFP4 weights of bf16 rows: packed E2M1 codes [R, K/2] (uint8) and E8M0 scales [R, K/32]."""
+    v = bf16_to_f32(v_bits).astype(np.float64)
+    R, K = v.shape
+    assert K % MX_BLOCK == 0
+    blocks = v.reshape(R, K // MX_BLOCK, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=2)
+    _, ex = np.frexp(np.where(amax > 0, amax, 1.0))      # amax in [2**(ex-1), 2**ex)
+    E = np.where(amax > 0, ex - 1 - 2, -127)
+    E = np.clip(E, -127, 127)
+    codes = e2m1_encode(blocks / np.exp2(E.astype(np.float64))[:, :, None]).reshape(R, K)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, (E + 127).astype(np.uint8)
+
+
+def mx4_unpack(packed: np.ndarray) -> np.ndarray:
+    """E2M1 codes [R, K] of packed MXFP4 rows [R, K/2]."""
+    p = np.asarray(packed, np.uint8)
+    codes = np.empty((p.shape[0], 2 * p.shape[1]), np.uint8)
+    codes[:, 0::2] = p & 0xF
+    codes[:, 1::2] = p >> 4
+    return codes
+
+
+def mx4_dequantize(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """float64 values P * 2**(scale - 127) of packed MXFP4 rows."""
+    codes = mx4_unpack(packed)
+    R, K = codes.shape
+    p = e2m1_decode(codes).reshape(R, K // MX_BLOCK, MX_BLOCK)
+    x = np.exp2(np.asarray(scales, np.float64) - 127.0)
+    return (p * x[:, :, None]).reshape(R, K)
+
+
+def linear_mxfp_a8w4(x_bits, w_packed, w_scales) -> dict:
+    """Dense MXFP A8W4 linear: x quantised per token to MXFP8, the weights in MXFP4, then
+    y = A . W^T exactly; returns the same fields as ``linear_mxfp8`` (token codes and scales, y,
+    and the bound of an fp32 summation in any order followed by one bf16 rounding)."""
+    xc, xs = mx_quantize_rows(x_bits)
+    A = mx_dequantize(xc, xs)
+    W = mx4_dequantize(w_packed, w_scales)
     y = A @ W.T
     K = A.shape[1]
     S = np.abs(A) @ np.abs(W).T
