@@ -51,7 +51,8 @@ HEADLINE = "qwen3-235b-a22b"
 SUB_MOE = ("qwen3-30b-a3b-decode", "qwen3-30b-a3b-prefill", "qwen3-30b-a3b-prefill-skewed",
            "qwen3-30b-a3b-prefill-shared")
 SUB_LINEAR = ("qwen3-1.7b-mlp-w4a8", "qwen3-1.7b-mlp-w8a8", "qwen3-30b-a3b-q-proj-w8a8",
-              "qwen3-30b-a3b-k-proj-w8a8", "qwen3-30b-a3b-o-proj-w8a8", "qwen3-1.7b-mlp-mxfp8")
+              "qwen3-30b-a3b-k-proj-w8a8", "qwen3-30b-a3b-o-proj-w8a8", "qwen3-1.7b-mlp-mxfp8",
+              "qwen3-1.7b-mlp-mxfp-a8w4")
 
 
 def parse():
@@ -177,6 +178,9 @@ def cpu_oracle_linear_rate(wl, n_tokens: int, min_seconds: float = 5.0, max_seco
     elif wl.fmt == "mxfp8":
         wc, ws = O.mx_quantize_rows(w)
         fwd = lambda: O.linear_mxfp8(x, wc, ws)  # noqa: E731
+    elif wl.fmt == "mxfp_a8w4":
+        wp, ws = O.mx4_quantize_rows(w)
+        fwd = lambda: O.linear_mxfp_a8w4(x, wp, ws)  # noqa: E731
     else:
         wq, sw = O.quantize_weight_per_channel(w)
         fwd = lambda: O.linear_w8a8(x, wq, sw)  # noqa: E731
@@ -447,12 +451,15 @@ def run_linear(args, wl, rank, dist, dev):
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).to(dev)  # noqa: E731
     x = bf(x_host)
     w = bf(synth.dense_weight(wl.N, wl.K, wl.seed))
-    mx = wl.fmt == "mxfp8"
+    mx = wl.fmt in ("mxfp8", "mxfp_a8w4")
     if wl.fmt == "int4":
         wq, sw = B.w8a8_quantize_weight_int4_per_group(w, wl.group)
         fmt, group = B.W8A8_W_INT4_PER_GROUP, wl.group
-    elif mx:
+    elif wl.fmt == "mxfp8":
         wq, sw = B.w8a8_mxfp8_quantize(w)  # E4M3 codes [N, K], E8M0 scales [N, K/32]
+        fmt, group = None, 32
+    elif wl.fmt == "mxfp_a8w4":
+        wq, sw = B.w8a8_mxfp4_quantize(w)  # packed E2M1 codes [N, K/2], E8M0 scales [N, K/32]
         fmt, group = None, 32
     else:
         wq, sw = B.w8a8_quantize_weight_per_channel(w)
@@ -463,8 +470,10 @@ def run_linear(args, wl, rank, dist, dev):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
     def linear(xd, pk, s_, wsp, yd, st=None):
-        if mx:
+        if wl.fmt == "mxfp8":
             B.w8a8_mxfp8_linear(xd, pk, s_, workspace=wsp, y=yd, stream=st)
+        elif wl.fmt == "mxfp_a8w4":
+            B.w8a8_mxfp_a8w4_linear(xd, pk, s_, workspace=wsp, y=yd, stream=st)
         else:
             B.w8a8_linear(xd, pk, s_, fmt, group, workspace=wsp, y=yd, stream=st)
 
@@ -531,22 +540,23 @@ def run_linear(args, wl, rank, dist, dev):
 
 
 def time_mxfp8_gemm(B, x, copies, wl, steps, stream):
-    """Mean duration (ms) of the MXFP8 linear's GEMM launch alone: x is quantised to MXFP8 once,
-    then K launches of w8a8_mxfp8_linear_prequant over the rotating weight copies are timed with
-    CUDA events on `stream`."""
+    """Mean duration (ms) of the MX linear's GEMM launch alone: x is quantised to MXFP8 once,
+    then K launches of w8a8_mxfp8_linear_prequant (or w8a8_mxfp_a8w4_linear_prequant) over the
+    rotating weight copies are timed with CUDA events on `stream`."""
     import torch
 
+    gemm = B.w8a8_mxfp_a8w4_linear_prequant if wl.fmt == "mxfp_a8w4" else B.w8a8_mxfp8_linear_prequant
     xc, xs = B.w8a8_mxfp8_quantize(x)
     y = torch.empty((wl.M, wl.N), dtype=torch.bfloat16, device=x.device)
     for i in range(3):
         pk, s_ = copies[i % len(copies)]
-        B.w8a8_mxfp8_linear_prequant(xc, xs, pk, s_, y=y)
+        gemm(xc, xs, pk, s_, y=y)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(stream)
     for i in range(steps):
         pk, s_ = copies[i % len(copies)]
-        B.w8a8_mxfp8_linear_prequant(xc, xs, pk, s_, y=y)
+        gemm(xc, xs, pk, s_, y=y)
     e1.record(stream)
     torch.cuda.synchronize()
     B.w8a8_check_status()
@@ -590,9 +600,12 @@ MEASURED_TRAFFIC = {
     # the W4A8 GEMM launch of the 2048 x 2048 -> 6144 linear: 10.9 MB read (weights, scales, token
     # codes once), nothing written back to DRAM within the launch (the 25 MB output stays in L2)
     "qwen3-1.7b-mlp-w4a8": (10_933_760 + 0, "1b4b2dc7d15bec2e91ed021dfeeca923eb8d5b51"),
-    # the block-scaled MXFP8 GEMM launch of the same shape: 17.3 MB read (FP8 weights and scales,
-    # token codes and scales, each once), 1.5 KB written back within the launch
-    "qwen3-1.7b-mlp-mxfp8": (17_346_304 + 1_536, "4a2b6e44df235a8e6e82bd6525612b372f14f632"),
+    # the block-scaled MXFP8 GEMM launch (CTA pairs) of the same shape: 17.4 MB read (FP8 weights
+    # and scales, token codes and scales, each once), nothing written back within the launch
+    "qwen3-1.7b-mlp-mxfp8": (17_357_824 + 0, "f19379502f764dd2f31a0291d0e550f9439368e2"),
+    # the MXFP A8W4 GEMM launch of the same shape: 11.1 MB read (6.3 MB of packed E2M1 weights, their
+    # scales, the token codes and scales, each once), nothing written back within the launch
+    "qwen3-1.7b-mlp-mxfp-a8w4": (11_066_368 + 0, "f19379502f764dd2f31a0291d0e550f9439368e2"),
 }
 TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
@@ -686,14 +699,18 @@ def linear_result(wl, res, K, world, peaks, peak_kind):
     ms_step = res["ms"] / K
     ops = 2.0 * wl.M * wl.N * wl.K
     nbytes = res["weight_bytes"] + wl.M * wl.K * 2 + wl.M * wl.N * 2
-    if wl.fmt == "mxfp8":
-        roof = roofline_entry(ops, nbytes, res["gemm_ms"] / 1e3, peaks, peak_kind, measured_traffic(wl.name, "mxfp8"),
-                              "MXFP8 GEMM (tcgen05 kind::mxf8f6f4 block-scaled FP8 MMA, E8M0 scales in TMEM)")
+    if wl.fmt in ("mxfp8", "mxfp_a8w4"):
+        a8w4 = wl.fmt == "mxfp_a8w4"
+        kernel = ("MXFP A8W4 GEMM (tcgen05 kind::mxf8f6f4 block-scaled MMA, E2M1 weights x E4M3 tokens, "
+                  "E8M0 scales in TMEM)" if a8w4 else
+                  "MXFP8 GEMM (tcgen05 kind::mxf8f6f4 block-scaled FP8 MMA, E8M0 scales in TMEM)")
+        roof = roofline_entry(ops, nbytes, res["gemm_ms"] / 1e3, peaks, peak_kind,
+                              measured_traffic(wl.name, "mxfp8"), kernel)
         step_tf = tensor_fracs(ops, ms_step / 1e3, peaks)
         return {
             "value": whole_job_rate(world, wl.M, K, res["ms"]), "unit": UNIT, "ms_per_step": ms_step,
-            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N, "weights": "mxfp8 e4m3 + e8m0",
-                       "block": 32},
+            "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N,
+                       "weights": "mxfp4 e2m1 + e8m0" if a8w4 else "mxfp8 e4m3 + e8m0", "block": 32},
             "roofline": roof,
             "step": {"tops": step_tf["tops"], "tensor_frac_of_2x_measured_bf16": step_tf["frac_of_2x_measured_bf16"],
                      "tensor_frac_of_datasheet": step_tf["frac_of_datasheet"],
@@ -874,7 +891,8 @@ def main():
     out = top_line(head, name, args, world)
     if name in synth.LINEAR_WORKLOADS:
         out["dtype"] = {"int4": "int8 (int4 weights unpacked to int8)", "int8": "int8",
-                        "mxfp8": "mxfp8 (e4m3 elements, e8m0 scales per 32)"}[wl.fmt]
+                        "mxfp8": "mxfp8 (e4m3 elements, e8m0 scales per 32)",
+                        "mxfp_a8w4": "mxfp8 x mxfp4 (e4m3 tokens, e2m1 weights, e8m0 scales per 32)"}[wl.fmt]
     if subs:
         out["sub_results"] = subs
     if probe is not None:

@@ -304,6 +304,39 @@ int w8a8_mxfp8_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, 
                                const uint8_t* w_scales, int64_t M, int64_t K, int64_t N, w8a8_bf16* y,
                                w8a8_stream stream);
 
+/* Defined by: the "MXFP A8w4" row of the same table (MXFP8 activations, MXFP4 weights), read as
+ * the OCP Microscaling FP4 format for the weights.
+ * MXFP4 quantisation of bf16 rows along K, for the weights of an MXFP A8W4 layer (once, per output
+ * channel): per block of 32 values E = floor(log2 max|v|) - 2 (clamped to [-127, 127], -127 for a
+ * zero block), scale byte E + 127 (E8M0), elements E2M1(v * 2^-E) rounded to nearest with ties to
+ * even and saturated at 6, the sign kept at zero; two codes per byte, element 2i in the low nibble.
+ *   w bf16 [R, K] (16-byte aligned), packed uint8 [R, K/2] (4-byte aligned), scales uint8 [R, K/32];
+ *   all device memory owned by the caller. K % 32 == 0 (else W8A8_ERR_UNSUPPORTED). */
+int w8a8_mxfp4_quantize(const w8a8_bf16* w, int64_t R, int64_t K, uint8_t* packed, uint8_t* scales,
+                        w8a8_stream stream);
+
+/* Defined by: the same row (MXFP A8W4).
+ * Dense MXFP A8W4 linear: x is quantised to MXFP8 per token (as in w8a8_mxfp8_linear), then the
+ * block-scaled MMA multiplies its E4M3 codes by the E2M1 weight codes, one E8M0 scale per 32
+ * values of K on both operands, summing in fp32:
+ *   y[m, n] = bf16(sum_k (P_x[m,k] 2^Ex[m,k/32]) (P_w[n,k] 2^Ew[n,k/32])),
+ * within the same summation bound as w8a8_mxfp8_linear.
+ *   x bf16 [M, K] (16-byte aligned); w_packed uint8 [N, K/2] (32-byte aligned) and w_scales uint8
+ *   [N, K/32] (4-byte aligned) from w8a8_mxfp4_quantize; workspace of
+ *   w8a8_mxfp8_linear_workspace_size() bytes (256-byte aligned; x's MXFP8 codes at offset 0 and
+ *   its scales after them, 256-byte aligned); y bf16 [M, N].
+ * K % 128 == 0, N % 128 == 0 (else W8A8_ERR_UNSUPPORTED). */
+int w8a8_mxfp_a8w4_linear(const w8a8_bf16* x, const uint8_t* w_packed, const uint8_t* w_scales, int64_t M,
+                          int64_t K, int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
+                          w8a8_stream stream);
+
+/* The GEMM of w8a8_mxfp_a8w4_linear on activations already in MXFP8: x_codes uint8 [M, K]
+ * (16-byte aligned), x_scales uint8 [M, K/32] (4-byte aligned); the weights, y and the shape rules
+ * as w8a8_mxfp_a8w4_linear. Needs no workspace. */
+int w8a8_mxfp_a8w4_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, const uint8_t* w_packed,
+                                   const uint8_t* w_scales, int64_t M, int64_t K, int64_t N, w8a8_bf16* y,
+                                   w8a8_stream stream);
+
 /* Exact integer GEMM on the tensor cores: c[m, n] = sum_k a[m, k] * b[n, k] in int32: the
  * int8 x int8 product every W8A8 Linear of the group_0 scheme accumulates before its scales.
  *   a int8 [M, K], b int8 [N, K], c int32 [M, N];  K % 128 == 0, N % 128 == 0. */

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.w8a8_version() == 210
+    assert lib.w8a8_version() == 220
     for st in range(-5, 1):
         assert B.status_string(st) not in ("", "unknown status")
 
@@ -84,6 +84,18 @@ def test_argument_checks_reject_before_any_launch(lib):
         B.W8A8_ERR_WORKSPACE
     assert lib.w8a8_mxfp8_linear(c(256), c(256), c(256), 8, 192, 256, c(256), 1 << 20, c(256), None) == \
         B.W8A8_ERR_UNSUPPORTED  # K % 128
+    assert lib.w8a8_mxfp4_quantize(c(16), 4, 48, c(16), c(16), None) == B.W8A8_ERR_UNSUPPORTED  # K % 32
+    assert lib.w8a8_mxfp4_quantize(None, 4, 64, None, None, None) == B.W8A8_ERR_ARG
+    assert lib.w8a8_mxfp4_quantize(None, 0, 64, None, None, None) == B.W8A8_OK  # empty
+    assert lib.w8a8_mxfp4_quantize(c(16), 4, 64, c(18), c(16), None) == B.W8A8_ERR_UNSUPPORTED  # packed alignment
+    assert lib.w8a8_mxfp_a8w4_linear(c(256), c(256), c(256), 8, 128, 256, c(256), 10, c(256), None) == \
+        B.W8A8_ERR_WORKSPACE
+    assert lib.w8a8_mxfp_a8w4_linear(c(256), c(256), c(256), 8, 192, 256, c(256), 1 << 20, c(256), None) == \
+        B.W8A8_ERR_UNSUPPORTED  # K % 128
+    assert lib.w8a8_mxfp_a8w4_linear(c(256), c(272), c(256), 8, 128, 256, c(256), 1 << 20, c(256), None) == \
+        B.W8A8_ERR_UNSUPPORTED  # packed weights not 32-byte aligned (the 4-bit TMA type needs it)
+    assert lib.w8a8_mxfp_a8w4_linear_prequant(c(256), c(256), c(256), c(256), 8, 128, 200, c(256), None) == \
+        B.W8A8_ERR_UNSUPPORTED  # N % 128
     assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_debug_rcp_approx_ulp(0, 10, c(16), None) == B.W8A8_ERR_ARG  # not a normal input
     assert lib.w8a8_debug_rcp_approx_ulp(0x7E7FFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # reciprocal subnormal

@@ -76,6 +76,9 @@ SIGNATURES = {
     "w8a8_mxfp8_linear_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64]),
     "w8a8_mxfp8_linear": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, ctypes.c_size_t, _c_p, _c_p]),
     "w8a8_mxfp8_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
+    "w8a8_mxfp4_quantize": (_int, [_c_p, _i64, _i64, _c_p, _c_p, _c_p]),
+    "w8a8_mxfp_a8w4_linear": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, ctypes.c_size_t, _c_p, _c_p]),
+    "w8a8_mxfp_a8w4_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
     "w8a8_debug_rcp_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
     "w8a8_debug_ex2_approx_ulp": (_int, [ctypes.c_uint32, ctypes.c_uint32, _c_p, _c_p]),
@@ -408,8 +411,47 @@ def w8a8_mxfp8_linear_prequant(x_codes, x_scales, w_codes, w_scales, y=None, str
     return y
 
 
+def w8a8_mxfp4_quantize(w: torch.Tensor, packed=None, scales=None, stream=None):
+    """w bf16 [R, K] -> (packed uint8 [R, K/2] (two E2M1 codes a byte, even element low),
+    scales uint8 [R, K/32] (E8M0))."""
+    _bf16(w)
+    R, K = w.shape
+    packed = torch.empty((R, max(K // 2, 1)), dtype=torch.uint8, device=w.device) if packed is None else packed
+    scales = torch.empty((R, max(K // 32, 1)), dtype=torch.uint8, device=w.device) if scales is None else scales
+    _check(lib().w8a8_mxfp4_quantize(_ptr(w), R, K, _ptr(packed), _ptr(scales), _stream(stream)),
+           "w8a8_mxfp4_quantize")
+    return packed, scales
+
+
+def w8a8_mxfp_a8w4_linear(x, w_packed, w_scales, workspace=None, y=None, stream=None):
+    """Dense MXFP A8W4 linear: y bf16 [M, N] = x [M, K] . W^T, x quantised to MXFP8 per token, W
+    given as MXFP4 (packed [N, K/2], scales [N, K/32]). The workspace is sized by
+    w8a8_mxfp8_linear_workspace_size and receives x's MXFP8 codes and scales."""
+    _bf16(x)
+    M, K = x.shape
+    N = w_packed.shape[0]
+    ws_bytes = w8a8_mxfp8_linear_workspace_size(M, K, N)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _check(lib().w8a8_mxfp_a8w4_linear(_ptr(x), _ptr(w_packed), _ptr(w_scales), M, K, N, _ptr(workspace),
+                                       workspace.numel(), _ptr(y), _stream(stream)), "w8a8_mxfp_a8w4_linear")
+    return y
+
+
+def w8a8_mxfp_a8w4_linear_prequant(x_codes, x_scales, w_packed, w_scales, y=None, stream=None):
+    """The GEMM of w8a8_mxfp_a8w4_linear on activations already in MXFP8."""
+    M, K = x_codes.shape
+    N = w_packed.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device) if y is None else y
+    _check(lib().w8a8_mxfp_a8w4_linear_prequant(_ptr(x_codes), _ptr(x_scales), _ptr(w_packed), _ptr(w_scales), M,
+                                                K, N, _ptr(y), _stream(stream)), "w8a8_mxfp_a8w4_linear_prequant")
+    return y
+
+
 def mxfp8_linear_intermediates(workspace, M: int, K: int) -> dict:
-    """x's MXFP8 codes [M, K] and scales [M, K/32] that w8a8_mxfp8_linear left in its workspace."""
+    """x's MXFP8 codes [M, K] and scales [M, K/32] that w8a8_mxfp8_linear (or
+    w8a8_mxfp_a8w4_linear) left in its workspace."""
     a256 = lambda v: (v + 255) // 256 * 256  # noqa: E731
     codes = workspace[:M * K].view(M, K)
     off = a256(M * K)

@@ -6,7 +6,17 @@
 //   element = E4M3(v * 2^-E), nearest with ties to even, saturating at 448, sign kept at zero.
 // The dense MXFP8 linear runs on the block-scaled FP8 MMA, which takes the codes and the E8M0
 // scales as they are and sums the products in fp32.
+// MXFP A8W4 (the "MXFP A8w4" row of the same table): the same MXFP8 activations against MXFP4
+// weights, the OCP format with FP4 E2M1 elements (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6):
+//   E = floor(log2(max |v| over the block)) - 2 (2 is the exponent of E2M1's largest binade);
+//   element = E2M1(v * 2^-E), nearest with ties to even, saturating at 6, sign kept at zero;
+//   two codes per byte, element 2i in the low nibble of byte i.
+// The GEMM kernels below take either weight format: E2M1 weights are loaded by TMA as packed
+// 4-bit data (the 16U4_ALIGN16B tensor-map type), which lands in shared memory as 8 bytes of 16
+// codes followed by 8 bytes of padding, the operand layout the MMA reads for 4-bit elements of
+// kind::mxf8f6f4; the MMA then multiplies E2M1 weights by E4M3 tokens directly.
 #pragma once
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "elementwise.cuh"
@@ -67,6 +77,46 @@ __global__ void __launch_bounds__(kMxWarps * 32) mx_quant_rows_kernel(const uint
   if ((lane & 3) == 0) scales[r * (K / kMxBlock) + k0 / kMxBlock] = uint8_t(E + 127);
 }
 
+// E2M1 codes of (lo, hi) in the low and high nibble of a byte: nearest, ties to even, saturating
+// at 6 (cvt.rn.satfinite.e2m1x2).
+__device__ __forceinline__ uint32_t e2m1_pair(float lo, float hi) {
+  return uint32_t(__nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest));
+}
+
+// MXFP4 weights of the bf16 rows src [R, K]: packed [R, K / 2] (two E2M1 codes per byte, the even
+// element low), scales [R, K / 32] (E8M0 bytes). K is a multiple of 32. The same split of the work
+// as mx_quant_rows_kernel: lane l holds values 8l .. 8l+7 of its warp's 256-value piece.
+__global__ void __launch_bounds__(kMxWarps * 32) mx4_quant_rows_kernel(const uint16_t* __restrict__ src,
+                                                                       int64_t R, int K,
+                                                                       uint8_t* __restrict__ packed,
+                                                                       uint8_t* __restrict__ scales) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int pieces = (K + 255) / 256;
+  const int64_t item = int64_t(blockIdx.x) * kMxWarps + (threadIdx.x >> 5);
+  if (item >= R * pieces) return;  // warp-uniform
+  const int64_t r = item / pieces;
+  const int lane = threadIdx.x & 31;
+  const int k0 = int(item - r * pieces) * 256 + lane * 8;
+  const bool valid = k0 < K;
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (valid) v = __ldg(reinterpret_cast<const uint4*>(src + r * K + k0));
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t mag = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mag = max(mag, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, 1));
+  mag = max(mag, __shfl_xor_sync(0xffffffffu, mag, 2));
+  const int E = mag == 0 ? -127 : min(127, max(-127, bf16_floor_log2(mag) - 2));
+  const float inv = __int_as_float((127 - E) << 23);  // 2^-E, a normal float (E <= 125 for bf16 input)
+  uint32_t c = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c |= e2m1_pair(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv)) << (8 * i);
+  if (!valid) return;
+  *reinterpret_cast<uint32_t*>(packed + r * (K / 2) + k0 / 2) = c;
+  if ((lane & 3) == 0) scales[r * (K / kMxBlock) + k0 / kMxBlock] = uint8_t(E + 127);
+}
+
 // ---------------------------------------------------------------- block-scaled MXFP8 GEMM
 // y[t, n] = bf16(sum_k (P_x[t,k] 2^Ex[t,k/32]) (P_w[n,k] 2^Ew[n,k/32])) with the block-scaled FP8
 // MMA (tcgen05.mma kind::mxf8f6f4.block_scale, scale_vec::1X: one E8M0 scale per 32 values of K
@@ -85,7 +135,8 @@ __global__ void __launch_bounds__(kMxWarps * 32) mx_quant_rows_kernel(const uint
 //   warps 6-13  epilogue: fp32 sums -> bf16 y, two warps per lane quarter.
 // Every wait is bounded (ptx.cuh).
 struct MxGemmParams {
-  CUtensorMap tmA;     // weight codes [N, K] bytes, box 128 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap tmA;     // weight codes: E4M3 [N, K] bytes, or E2M1 [N, K/2] packed bytes loaded as
+                       // 16U4_ALIGN16B; box 128 rows x 128 values, 128-byte swizzle
   CUtensorMap tmB;     // token codes [M, K] bytes, the same box
   const uint32_t* sfa; // weight scales [N, K/32] bytes, read as words [N, K/128]
   const uint32_t* sfb; // token scales [M, K/32] bytes, read as words [M, K/128]
@@ -108,11 +159,22 @@ constexpr int kMxThreads = 32 * 14;
 constexpr size_t kMxSmemBytes = 1024 + size_t(kMxStages) * kMxStageBytes + 512;
 static_assert(kMxSfCol0 + 8 * kMxStages <= kMxTmemCols, "accumulators and scale columns fit in TMEM");
 
-// Instruction descriptor of the block-scaled MMA: A and B E4M3 (format 0), both K-major, fp32
-// accumulation, M = 128, N = n, E8M0 scales (bit 23), scale-factor ids of A (bits 29-30) and B
-// (bits 4-5) = j.
+// Element formats of the block-scaled MMA's operands (its format fields): the weights are E4M3
+// or E2M1, the tokens always E4M3.
+constexpr int kMxE4M3 = 0;
+constexpr int kMxE2M1 = 5;
+// TMA bytes of one 128-row weight K-block (128 values a row): E2M1 rows are 64 bytes in global
+// memory (the transaction count of the 16U4_ALIGN16B load; it fills 128 bytes of shared memory).
+template <int WF>
+constexpr uint32_t kMxWeightTxBytes = WF == kMxE2M1 ? kBM * kKBlockBytes / 2 : kBM * kKBlockBytes;
+
+// Instruction descriptor of the block-scaled MMA: A (weights) in format WF (bits 7-9), B (tokens)
+// E4M3, both K-major, fp32 accumulation, M = 128, N = n, E8M0 scales (bit 23), scale-factor ids of
+// A (bits 29-30) and B (bits 4-5) = j.
+template <int WF>
 __host__ __device__ constexpr uint32_t idesc_mxf8(int n, uint32_t j) {
-  return (j << 4) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(128 >> 4) << 24) | (j << 29);
+  return (j << 4) | (uint32_t(WF) << 7) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(128 >> 4) << 24) |
+         (j << 29);
 }
 
 __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -131,6 +193,7 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b,
                "r"(d));
 }
 
+template <int WF>
 __global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_constant__ MxGemmParams p) {
   constexpr int S = kMxStages;
   extern __shared__ uint8_t smem_raw[];
@@ -181,7 +244,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_con
         if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
         if (elect_one()) {
           uint8_t* st = smem + stage * kMxStageBytes;
-          mbar_arrive_expect_tx(full + stage, uint32_t(kMxStageBytes));
+          mbar_arrive_expect_tx(full + stage, kMxWeightTxBytes<WF> + uint32_t(kMxNB * kKBlockBytes));
           tma_load_2d(st, &p.tmA, full + stage, kb * kKBlockBytes, cb * kBM);
           tma_load_2d(st + kBM * kKBlockBytes, &p.tmB, full + stage, kb * kKBlockBytes, mt * kMxNB);  // rows past M: zeros
         }
@@ -218,7 +281,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_con
           const uint32_t sf = tmem_base + kMxSfCol0 + uint32_t(8 * stage);
 #pragma unroll
           for (uint32_t j = 0; j < 4; ++j)
-            tc_mma_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8(kMxNB, j), sf + (j << 30),
+            tc_mma_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8<WF>(kMxNB, j), sf + (j << 30),
                         sf + 4u + (j << 30), (kb | int(j)) != 0 ? 1u : 0u);
           tc_commit(empty + stage);
         }
@@ -333,7 +396,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_con
 // tensor core scales every column of its accumulators. (Holding only the 96 token rows a rank
 // supplies gives wrong sums for the other half of the columns.)
 struct MxPairParams {
-  CUtensorMap tmA;     // weight codes [N, K], box 128 rows x 128 bytes, 128-byte swizzle
+  CUtensorMap tmA;     // weight codes (E4M3 or packed E2M1, as in MxGemmParams), box 128 rows x 128
+                       // values, 128-byte swizzle
   CUtensorMap tmB;     // token codes [M, K], box 96 rows x 128 bytes, 128-byte swizzle
   const uint32_t* sfa; // weight scales as words [N, K/128]
   const uint32_t* sfb; // token scales as words [M, K/128]
@@ -358,8 +422,10 @@ constexpr size_t kMxPairSmemBytes = 1024 + size_t(kMxPairStages) * kMxPairStageB
 static_assert(kMxPairSfCol0 + kMxPairSfCols * kMxPairStages <= 512, "accumulators and scales fit in TMEM");
 static_assert(kMxPairBBytes % 1024 == 0, "128-byte swizzled token rows sit on 1 KB boundaries");
 
+template <int WF>
 __host__ __device__ constexpr uint32_t idesc_mxf8_m256(int n, uint32_t j) {
-  return (j << 4) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(256 >> 4) << 24) | (j << 29);
+  return (j << 4) | (uint32_t(WF) << 7) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(256 >> 4) << 24) |
+         (j << 29);
 }
 
 __device__ __forceinline__ void tc_mma_pair_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -372,6 +438,7 @@ __device__ __forceinline__ void tc_mma_pair_mxf8(uint32_t d_tmem, uint64_t adesc
       : "memory");
 }
 
+template <int WF>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
     mx_pair_kernel(const __grid_constant__ MxPairParams p) {
   constexpr int S = kMxPairStages;
@@ -431,7 +498,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
         if (elect_one()) {
           uint8_t* st = smem + stage * kMxPairStageBytes;
           const uint32_t bar = full0 + uint32_t(stage) * 8u;
-          if (leader) mbar_arrive_expect_tx(full + stage, 2u * uint32_t(kMxPairStageBytes));
+          if (leader) mbar_arrive_expect_tx(full + stage, 2u * (kMxWeightTxBytes<WF> + uint32_t(kMxPairBBytes)));
           tma_load_2d_pair(st, &p.tmA, bar, kb * kKBlockBytes, cb * 256 + int(rank) * 128);
           tma_load_2d_pair(st + kMxPairABytes, &p.tmB, bar, kb * kKBlockBytes,
                            mt * kMxPairNB + int(rank) * kMxPairHalf);  // rows past M: zeros
@@ -484,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
             const uint32_t sf = tmem_base + kMxPairSfCol0 + uint32_t(kMxPairSfCols * stage);
 #pragma unroll
             for (uint32_t j = 0; j < 4; ++j)
-              tc_mma_pair_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8_m256(kMxPairNB, j),
+              tc_mma_pair_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8_m256<WF>(kMxPairNB, j),
                                sf + (j << 30), sf + 4u + (j << 30), (kb | int(j)) != 0 ? 1u : 0u);
             tc_commit_pair(empty_own + uint32_t(stage) * 8u);
             tc_commit_pair(empty_peer + uint32_t(stage) * 8u);

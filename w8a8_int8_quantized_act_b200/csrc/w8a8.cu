@@ -17,7 +17,7 @@
 namespace w8a8 {
 namespace {
 
-constexpr int kVersion = 210;  // 0.2.1
+constexpr int kVersion = 220;  // 0.2.2
 
 cudaStream_t as_stream(w8a8_stream s) { return static_cast<cudaStream_t>(s); }
 
@@ -74,6 +74,23 @@ bool make_kmajor_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D K-major map over packed 4-bit rows [rows, inner values] (inner / 2 bytes a row) with a
+// (box_rows x 128-value) box of the 16U4_ALIGN16B type: each 8 bytes of 16 codes land in 16
+// bytes of shared memory (the padded 4-bit operand layout of the block-scaled MMA), 128-byte
+// swizzle. The type needs a 32-byte aligned base, rows of a multiple of 32 bytes and inner a
+// multiple of 128 values.
+bool make_kmajor_map_e2m1(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || inner == 0 || inner % 128 || (reinterpret_cast<uintptr_t>(base) & 31u)) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner / 2};
+  const cuuint32_t box[2] = {128u, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2-D map over [rows, inner_bytes] bytes with an unswizzled (box_rows x box_bytes) box.
@@ -336,16 +353,33 @@ int launch_mx_rows(const w8a8_bf16* src, int64_t R, int K, uint8_t* codes, uint8
                     K, codes, scales);
 }
 
-// MXFP8 GEMMs with more token rows than this (and N a multiple of 256) run on CTA pairs.
+// MXFP4 weights (packed E2M1 codes and E8M0 scales) of the bf16 rows src [R, K].
+int launch_mx4_rows(const w8a8_bf16* src, int64_t R, int K, uint8_t* packed, uint8_t* scales, cudaStream_t s) {
+  const int64_t items = R * ((K + 255) / 256);
+  const dim3 grid(unsigned((items + kMxWarps - 1) / kMxWarps));
+  return launch_pdl(mx4_quant_rows_kernel, grid, dim3(kMxWarps * 32), 0, s, reinterpret_cast<const uint16_t*>(src),
+                    R, K, packed, scales);
+}
+
+// MX GEMMs with more token rows than this (and N a multiple of 256) run on CTA pairs.
 constexpr int64_t kMxPairMinRows = 192;
 
-// y [M, N] = the MXFP8 product of token codes / scales and weight codes / scales on the
-// block-scaled FP8 MMA (mx_gemm_kernel). K % 128 == 0, N % 128 == 0; checked by the callers.
+// Weight map of the MX GEMMs: E4M3 codes [N, K] or packed E2M1 codes [N, K/2], 128-row box.
+template <int WF>
+bool make_mx_weight_map(CUtensorMap* m, const uint8_t* wc, int64_t K, int64_t N) {
+  if constexpr (WF == kMxE2M1) return make_kmajor_map_e2m1(m, wc, uint64_t(K), uint64_t(N), 128);
+  return make_kmajor_map(m, wc, false, uint64_t(K), uint64_t(N), 128);
+}
+
+// y [M, N] = the MX product of token codes / scales (MXFP8) and weight codes / scales (MXFP8, or
+// MXFP4 for WF = kMxE2M1) on the block-scaled MMA. K % 128 == 0, N % 128 == 0; checked by the
+// callers.
+template <int WF>
 int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8_t* ws, int64_t M, int64_t K,
             int64_t N, w8a8_bf16* y, cudaStream_t s) {
   if (M > kMxPairMinRows && N % 256 == 0) {
     MxPairParams q{};
-    if (!make_kmajor_map(&q.tmA, wc, false, K, N, 128) || !make_kmajor_map(&q.tmB, xc, false, K, M, kMxPairHalf))
+    if (!make_mx_weight_map<WF>(&q.tmA, wc, K, N) || !make_kmajor_map(&q.tmB, xc, false, K, M, kMxPairHalf))
       return W8A8_ERR_UNSUPPORTED;
     q.sfa = reinterpret_cast<const uint32_t*>(ws);
     q.sfb = reinterpret_cast<const uint32_t*>(xs);
@@ -355,7 +389,7 @@ int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8
     q.N = int(N);
     q.y = reinterpret_cast<uint16_t*>(y);
     q.timeout_ns = wait_timeout_ns();
-    auto kern = mx_pair_kernel;
+    auto kern = mx_pair_kernel<WF>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMxPairSmemBytes)) != cudaSuccess)
       return W8A8_ERR_LAUNCH;
     const int tiles = int((M + kMxPairNB - 1) / kMxPairNB) * q.n_cb;
@@ -363,7 +397,7 @@ int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8
     return launch_pdl(kern, dim3(2 * clusters), dim3(kMxPairThreads), kMxPairSmemBytes, s, q);
   }
   MxGemmParams p{};
-  if (!make_kmajor_map(&p.tmA, wc, false, K, N, 128) || !make_kmajor_map(&p.tmB, xc, false, K, M, 128))
+  if (!make_mx_weight_map<WF>(&p.tmA, wc, K, N) || !make_kmajor_map(&p.tmB, xc, false, K, M, 128))
     return W8A8_ERR_UNSUPPORTED;
   p.sfa = reinterpret_cast<const uint32_t*>(ws);
   p.sfb = reinterpret_cast<const uint32_t*>(xs);
@@ -373,11 +407,11 @@ int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8
   p.N = int(N);
   p.y = reinterpret_cast<uint16_t*>(y);
   p.timeout_ns = wait_timeout_ns();
-  if (cudaFuncSetAttribute(mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMxSmemBytes)) !=
-      cudaSuccess)
+  auto kern = mx_gemm_kernel<WF>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMxSmemBytes)) != cudaSuccess)
     return W8A8_ERR_LAUNCH;
   const int tiles = int((M + kMxNB - 1) / kMxNB) * p.n_cb;
-  return launch_pdl(mx_gemm_kernel, dim3(max(1, min(num_sms(), tiles))), dim3(kMxThreads), kMxSmemBytes, s, p);
+  return launch_pdl(kern, dim3(max(1, min(num_sms(), tiles))), dim3(kMxThreads), kMxSmemBytes, s, p);
 }
 
 int launch_quant_rows(const uint16_t* src, int64_t R, int K, int8_t* q, float* scale, cudaStream_t s) {
@@ -1183,7 +1217,7 @@ int w8a8_mxfp8_linear(const w8a8_bf16* x, const uint8_t* w_codes, const uint8_t*
   const cudaStream_t s = as_stream(stream);
   const int rc = launch_mx_rows(x, M, int(K), xc, xs, s);
   if (rc != W8A8_OK) return rc;
-  return mx_gemm(xc, xs, w_codes, w_scales, M, K, N, y, s);
+  return mx_gemm<kMxE4M3>(xc, xs, w_codes, w_scales, M, K, N, y, s);
 }
 
 int w8a8_mxfp8_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, const uint8_t* w_codes,
@@ -1196,7 +1230,50 @@ int w8a8_mxfp8_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, 
   if (!aligned16(x_codes) || !aligned16(w_codes) || !aligned16(y) || (reinterpret_cast<uintptr_t>(x_scales) & 3u) ||
       (reinterpret_cast<uintptr_t>(w_scales) & 3u))
     return W8A8_ERR_UNSUPPORTED;
-  return mx_gemm(x_codes, x_scales, w_codes, w_scales, M, K, N, y, as_stream(stream));
+  return mx_gemm<kMxE4M3>(x_codes, x_scales, w_codes, w_scales, M, K, N, y, as_stream(stream));
+}
+
+int w8a8_mxfp4_quantize(const w8a8_bf16* w, int64_t R, int64_t K, uint8_t* packed, uint8_t* scales,
+                        w8a8_stream stream) {
+  if (R < 0 || K <= 0) return W8A8_ERR_ARG;
+  if (K % kMxBlock || K > (int64_t(1) << 30) || R >= (int64_t(1) << 31)) return W8A8_ERR_UNSUPPORTED;
+  if (R == 0) return W8A8_OK;
+  if (!w || !packed || !scales) return W8A8_ERR_ARG;
+  if (!aligned16(w) || (reinterpret_cast<uintptr_t>(packed) & 3u)) return W8A8_ERR_UNSUPPORTED;
+  return launch_mx4_rows(w, R, int(K), packed, scales, as_stream(stream));
+}
+
+int w8a8_mxfp_a8w4_linear(const w8a8_bf16* x, const uint8_t* w_packed, const uint8_t* w_scales, int64_t M,
+                          int64_t K, int64_t N, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
+                          w8a8_stream stream) {
+  if (M < 0 || K <= 0 || N <= 0) return W8A8_ERR_ARG;
+  const size_t need = w8a8_mxfp8_linear_workspace_size(M, K, N);
+  if (need == 0) return W8A8_ERR_UNSUPPORTED;
+  if (M == 0) return W8A8_OK;
+  if (!x || !w_packed || !w_scales || !y || !workspace) return W8A8_ERR_ARG;
+  if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(y) || (reinterpret_cast<uintptr_t>(w_packed) & 31u) ||
+      (reinterpret_cast<uintptr_t>(w_scales) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return W8A8_ERR_UNSUPPORTED;
+  uint8_t* xc = static_cast<uint8_t*>(workspace);
+  uint8_t* xs = xc + align256(size_t(M) * K);
+  const cudaStream_t s = as_stream(stream);
+  const int rc = launch_mx_rows(x, M, int(K), xc, xs, s);
+  if (rc != W8A8_OK) return rc;
+  return mx_gemm<kMxE2M1>(xc, xs, w_packed, w_scales, M, K, N, y, s);
+}
+
+int w8a8_mxfp_a8w4_linear_prequant(const uint8_t* x_codes, const uint8_t* x_scales, const uint8_t* w_packed,
+                                   const uint8_t* w_scales, int64_t M, int64_t K, int64_t N, w8a8_bf16* y,
+                                   w8a8_stream stream) {
+  if (M < 0 || K <= 0 || N <= 0) return W8A8_ERR_ARG;
+  if (w8a8_mxfp8_linear_workspace_size(M, K, N) == 0) return W8A8_ERR_UNSUPPORTED;
+  if (M == 0) return W8A8_OK;
+  if (!x_codes || !x_scales || !w_packed || !w_scales || !y) return W8A8_ERR_ARG;
+  if (!aligned16(x_codes) || (reinterpret_cast<uintptr_t>(w_packed) & 31u) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(x_scales) & 3u) || (reinterpret_cast<uintptr_t>(w_scales) & 3u))
+    return W8A8_ERR_UNSUPPORTED;
+  return mx_gemm<kMxE2M1>(x_codes, x_scales, w_packed, w_scales, M, K, N, y, as_stream(stream));
 }
 
 int w8a8_debug_wait_timeout(uint64_t timeout_ns, w8a8_stream stream) {

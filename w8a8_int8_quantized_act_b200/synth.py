@@ -62,8 +62,9 @@ class MoEWorkload:
 @dataclass(frozen=True)
 class LinearWorkload:
     """Dense linear workload: x [M, K] times W [N, K]^T; weights int4 in groups of ``group``
-    along K (``fmt`` "int4"), int8 per output channel (``fmt`` "int8"), or MXFP8 with both
-    operands in blocks of 32 along K (``fmt`` "mxfp8")."""
+    along K (``fmt`` "int4"), int8 per output channel (``fmt`` "int8"), MXFP8 with both
+    operands in blocks of 32 along K (``fmt`` "mxfp8"), or MXFP8 activations with MXFP4 weights
+    (``fmt`` "mxfp_a8w4")."""
 
     name: str
     M: int
@@ -104,6 +105,9 @@ LINEAR_WORKLOADS = {
         LinearWorkload("qwen3-30b-a3b-o-proj-w8a8", M=2048, K=4096, N=2048, group=0, n_outlier=41, fmt="int8"),
         # the MLP shape in MXFP8 A8W8 (E4M3 elements, one E8M0 scale per 32 values along K)
         LinearWorkload("qwen3-1.7b-mlp-mxfp8", M=2048, K=2048, N=6144, group=32, n_outlier=20, fmt="mxfp8"),
+        # and in MXFP A8W4 (MXFP8 activations, E2M1 weights with one E8M0 scale per 32 values)
+        LinearWorkload("qwen3-1.7b-mlp-mxfp-a8w4", M=2048, K=2048, N=6144, group=32, n_outlier=20,
+                       fmt="mxfp_a8w4"),
     )
 }
 
