@@ -392,9 +392,17 @@ __global__ void __launch_bounds__(kMxThreads, 1) mx_gemm_kernel(const __grid_con
 // sums of its 128 channels for all 192 tokens, so per SM and K-block 16 + 12 KB of codes feed
 // 128 x 192 x 128 MACs (the one-CTA tile moves 32 KB for 128 x 128 x 128). Each rank keeps in its
 // TMEM, per stage and laid out like the one-CTA kernel's, the scales of its own 128 weight rows
-// (4 columns) and those of all 192 token rows of the tile (6 columns): each CTA's half of the
-// tensor core scales every column of its accumulators. (Holding only the 96 token rows a rank
-// supplies gives wrong sums for the other half of the columns.)
+// (4 columns) and those of the tile's token rows (6 of 8 columns): each CTA's half of the tensor
+// core scales every column of its accumulators. (Holding only the 96 token rows a rank supplies
+// gives wrong sums for the other half of the columns.)
+// The scales reach TMEM through shared memory: the scale warps write each stage's words there in
+// the order one `tcgen05.cp.32x128b.warpx4` takes (32 rows of 16 bytes: row l holds the words of
+// rows l, 32 + l, 64 + l, 96 + l, copied to columns 0-3 of every lane quarter), and the MMA thread
+// issues the copies right before the stage's MMAs; copies and MMAs of one thread run in issue
+// order, so nothing waits on TMEM stores. (Scale warps storing into TMEM themselves with
+// tcgen05.st made every K-block wait for those stores: 45 us against 28 us without them.) The
+// token scales are copied as 8 groups of 32 rows from the 4-aligned group at or below the tile's
+// first (tiles start at group 6 mt), and the MMA's scale address skips the first 0 or 2 columns.
 struct MxPairParams {
   CUtensorMap tmA;     // weight codes (E4M3 or packed E2M1, as in MxGemmParams), box 128 rows x 128
                        // values, 128-byte swizzle
@@ -416,9 +424,11 @@ constexpr int kMxPairABytes = kBM * kKBlockBytes;
 constexpr int kMxPairBBytes = kMxPairHalf * kKBlockBytes;
 constexpr int kMxPairStageBytes = kMxPairABytes + kMxPairBBytes;
 constexpr uint32_t kMxPairSfCol0 = 2 * kMxPairNB;  // after both accumulator sets
-constexpr int kMxPairSfCols = 12;                  // per stage: SFA 4 + SFB 6 (+ 2 of padding)
+constexpr int kMxPairSfCols = 12;                  // per stage: SFA 4 + SFB 8 (token groups)
+constexpr int kMxPairSfBytes = 3 * 512;            // per stage in shared memory: SFA, SFB groups 0-3, 4-7
 constexpr int kMxPairThreads = 32 * 14;
-constexpr size_t kMxPairSmemBytes = 1024 + size_t(kMxPairStages) * kMxPairStageBytes + 512;
+constexpr size_t kMxPairSmemBytes =
+    1024 + size_t(kMxPairStages) * kMxPairStageBytes + 512 + size_t(kMxPairStages) * kMxPairSfBytes;
 static_assert(kMxPairSfCol0 + kMxPairSfCols * kMxPairStages <= 512, "accumulators and scales fit in TMEM");
 static_assert(kMxPairBBytes % 1024 == 0, "128-byte swizzled token rows sit on 1 KB boundaries");
 
@@ -426,6 +436,23 @@ template <int WF>
 __host__ __device__ constexpr uint32_t idesc_mxf8_m256(int n, uint32_t j) {
   return (j << 4) | (uint32_t(WF) << 7) | (uint32_t(n >> 3) << 17) | (1u << 23) | (uint32_t(256 >> 4) << 24) |
          (j << 29);
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte block for tcgen05.cp: no swizzle, rows 16 bytes
+// apart within 8-row core matrices, core matrices 128 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t sf_block_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t(1) << 16;          // leading byte offset (one 16-byte column: unused)
+  d |= uint64_t(128 >> 4) << 32;   // stride byte offset
+  d |= uint64_t(1) << 46;          // descriptor version
+  return d;                        // layout type 0: no swizzle
+}
+
+// Copies a 32-row x 128-bit block from shared memory into 4 TMEM columns of every lane quarter
+// (row l to lane l of each quarter), in both CTAs of the pair (each from its own shared memory).
+__device__ __forceinline__ void tc_cp_pair_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_pair_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -452,6 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* sf_smem = smem + S * kMxPairStageBytes + 512;  // [S][3][32 rows][16 bytes]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -461,7 +489,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
   const int nclusters = int(cluster_count());
   const WaitCtx wc{abort_flag, p.timeout_ns};
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); mbar_init(sfready + s, 8); }
+    for (int s = 0; s < S; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); mbar_init(sfready + s, 2); }
     for (int a = 0; a < 2; ++a) { mbar_init(tfull + a, 1); mbar_init(tempty + a, 16); }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -541,6 +569,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
         if (!mbar_wait_warp(tempty + acc, acc_phase ^ 1u, wc)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * kMxPairNB);
+        const int mt = (cluster + t * nclusters) / p.n_cb;
+        const uint32_t sfb_skip = uint32_t((6 * mt) & 3);  // the tile's first token group within the copied 8
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_warp(full + stage, phase, wc)) { ok = false; break; }
           if (!mbar_wait_warp(sfready + stage, phase, wc)) { ok = false; break; }
@@ -549,10 +579,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
             const uint64_t ad = adesc0 + uint64_t(stage * (kMxPairStageBytes >> 4));
             const uint64_t bd = ad + uint64_t(kMxPairABytes >> 4);
             const uint32_t sf = tmem_base + kMxPairSfCol0 + uint32_t(kMxPairSfCols * stage);
+            const uint32_t sfs = smem_addr(sf_smem + stage * kMxPairSfBytes);
+            tc_cp_pair_32x128b_x4(sf, sf_block_desc(sfs));                // weight rows: columns 0-3
+            tc_cp_pair_32x128b_x4(sf + 4u, sf_block_desc(sfs + 512u));    // token groups 0-3
+            tc_cp_pair_32x128b_x4(sf + 8u, sf_block_desc(sfs + 1024u));   // token groups 4-7
+            const uint32_t sfb = sf + 4u + sfb_skip;
 #pragma unroll
             for (uint32_t j = 0; j < 4; ++j)
               tc_mma_pair_mxf8(d, ad + uint64_t(2 * j), bd + uint64_t(2 * j), idesc_mxf8_m256<WF>(kMxPairNB, j),
-                               sf + (j << 30), sf + 4u + (j << 30), (kb | int(j)) != 0 ? 1u : 0u);
+                               sf + (j << 30), sfb + (j << 30), (kb | int(j)) != 0 ? 1u : 0u);
             tc_commit_pair(empty_own + uint32_t(stage) * 8u);
             tc_commit_pair(empty_peer + uint32_t(stage) * 8u);
           }
@@ -584,48 +619,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMxPairThreads, 1)
     __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------ scale writers (both ranks)
-    constexpr int D = kMxSfAhead;
-    const int q = warp & 3;
-    const uint32_t lane_off = uint32_t(q * 32) << 16;
+    // The four warps take the stages in turn (warp 2 + w the items w, w + 4, ...), so each has
+    // four K-blocks of time for one stage's loads, stores, proxy fence and remote arrival. Lane l
+    // writes row l of the three 32-row blocks: the words of weight rows l, 32 + l, 64 + l, 96 + l
+    // and of token groups 0-3 and 4-7 (row l of each), one 16-byte store per block.
+    const int w = warp - 2;
     const uint32_t sfready0 = map_to_rank(smem_addr(sfready), 0);
     const int wpr = nkb;
     const int n = my_tiles * nkb;
-    auto load = [&](int i, uint32_t (&a)[4], uint32_t (&b)[6]) {
+    auto load = [&](int i, uint32_t (&v)[12]) {
       const int tile = cluster + (i / nkb) * nclusters, kb = i % nkb;
       const int mt = tile / p.n_cb, cb = tile - mt * p.n_cb;
-      const int c0 = cb * 256 + int(rank) * 128, t0 = mt * kMxPairNB;
+      const int c0 = cb * 256 + int(rank) * 128 + lane;
+      const int t0 = 32 * ((6 * mt) & ~3) + lane;  // row l of the first copied token group
 #pragma unroll
-      for (int g = 0; g < 4; ++g) a[g] = __ldg(p.sfa + size_t(c0 + 32 * g + lane) * wpr + kb);
+      for (int g = 0; g < 4; ++g) v[g] = __ldg(p.sfa + size_t(c0 + 32 * g) * wpr + kb);
 #pragma unroll
-      for (int g = 0; g < 6; ++g) {
-        const int t = t0 + 32 * g + lane;
-        b[g] = t < p.M ? __ldg(p.sfb + size_t(t) * wpr + kb) : 0u;
+      for (int g = 0; g < 8; ++g) {
+        const int t = t0 + 32 * g;
+        v[4 + g] = t < p.M ? __ldg(p.sfb + size_t(t) * wpr + kb) : 0u;
       }
     };
-    uint32_t ra[D][4], rb[D][6];
-#pragma unroll
-    for (int d = 0; d < D; ++d)
-      if (d < n) load(d, ra[d], rb[d]);
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int i0 = 0; i0 < n && ok; i0 += D) {
-#pragma unroll
-      for (int d = 0; d < D; ++d) {
-        const int i = i0 + d;
-        if (i >= n) break;
-        if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
-        const uint32_t col = tmem_base + lane_off + kMxPairSfCol0 + uint32_t(kMxPairSfCols * stage);
-        tmem_st4(col, ra[d][0], ra[d][1], ra[d][2], ra[d][3]);
-        tmem_st4(col + 4u, rb[d][0], rb[d][1], rb[d][2], rb[d][3]);
-        tmem_st4(col + 8u, rb[d][4], rb[d][5], 0u, 0u);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(sfready0 + uint32_t(stage) * 8u);
-        if (++stage == S) { stage = 0; phase ^= 1u; }
-        if (i + D < n) load(i + D, ra[d], rb[d]);
-      }
+    uint32_t v[12];
+    if (w < n) load(w, v);
+    for (int i = w; i < n; i += 4) {
+      const int stage = i % S;
+      const uint32_t phase = uint32_t(i / S) & 1u;
+      // the stage's previous copies have completed (they precede the MMAs whose commit this is)
+      if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) break;
+      uint4* blk = reinterpret_cast<uint4*>(sf_smem + stage * kMxPairSfBytes) + lane;
+      blk[0] = make_uint4(v[0], v[1], v[2], v[3]);
+      blk[32] = make_uint4(v[4], v[5], v[6], v[7]);
+      blk[64] = make_uint4(v[8], v[9], v[10], v[11]);
+      fence_proxy_async_smem();  // generic-proxy writes become visible to tcgen05.cp
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(sfready0 + uint32_t(stage) * 8u);
+      if (i + 4 < n) load(i + 4, v);
     }
   } else {
     // ------------------------------------------------------------ epilogue (both ranks)
