@@ -304,9 +304,11 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
                int renorm, int* ids, float* w, int* counts, int64_t count_stride, float* logits,
                cudaStream_t stream) {
   const int nb = router_bn(E);
-  // 64 tokens per tile: the top-k epilogue, the larger part of the kernel, spreads over twice
-  // as many CTAs (64 -> 128 of them for 8192 tokens)
-  constexpr int kRouterRows = 64;
+  // 64 tokens per tile (the top-k epilogue spreads over twice as many CTAs as with 128: 128 of
+  // them for 8192 tokens), or 32 where that still fits the SMs in one wave (4096 tokens: 128
+  // CTAs instead of 64; each CTA streams all of W_gate, so fewer tokens per CTA leave the bytes
+  // per CTA nearly unchanged but use twice the SMs)
+  const int kRouterRows = (T + 31) / 32 <= num_sms() ? 32 : 64;
   GemmParams p{};
   if (!make_kmajor_map(&p.tmA, x, true, H, T, kRouterRows) || !make_kmajor_map(&p.tmB, wg, true, H, E, kBBoxRows) ||
       !make_kmajor_map(&p.tmB2, wg, true, H, E, uint32_t(nb)))
