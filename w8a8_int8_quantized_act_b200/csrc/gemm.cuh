@@ -70,7 +70,7 @@ struct GemmParams {
   float* topk_w;
   int* tile_counts;            // expert histogram rows (nullptr: none); zeroed before the launch
   int tile_count_stride;       // elements between the rows of consecutive 128-token chunks (0: one row)
-  int router_rows;             // router: tokens per tile (64 or 128; the A map's box height)
+  int router_rows;             // router: tokens per tile (32 or 64; the A map's box height)
   // down with the requantisation of h fused into the B operand (template QKB > 0): the bf16 rows
   // of h [rows, K] the CTA quantises itself, and where the tiles of channel block 0 leave the
   // codes and scales (hq [rows, K], s_h [rows])
@@ -81,16 +81,22 @@ struct GemmParams {
 
 // QKB > 0 (down GEMM of short token lists): the B operand of a tile is not loaded by TMA but made
 // by the CTA itself from bf16 h, QKB K-blocks at most, into one of two resident buffers.
+// Router tiles hold at most this many tokens (the A rows its TMA loads per K-block); its MMA keeps
+// M = 128 and reads the stage's next bytes as rows 64-127, whose results nobody reads.
+constexpr int kRouterMaxRows = 64;
+constexpr int kRouterPitch = kRouterMaxRows + 1;  // floats per expert row of the transposed logits
+
 template <int NA, int NB, int EPI, int QKB = 0>
 struct GemmCfg {
-  static constexpr int kABytes = kBM * kKBlockBytes;
+  static constexpr int kABytes = (EPI == kEpiRouter ? kRouterMaxRows : kBM) * kKBlockBytes;
   static constexpr int kBBytes = NB * kKBlockBytes;
   static constexpr int kStageBytes = NA * kABytes + (QKB > 0 ? 0 : kBBytes);
-  // router: logits of one tile transposed to [expert][token] (row pitch 129 floats, so both the
+  // router: logits of one tile transposed to [expert][token] (row pitch 65 floats, so both the
   // per-token writes and the per-expert reads are free of bank conflicts); resident B: two
   // buffers of QKB 128-byte-swizzled K-blocks of NB rows, then their row scales
   static constexpr int kQBBufBytes = QKB * NB * kKBlockBytes;
-  static constexpr int kXBytes = (EPI == kEpiRouter) ? NB * 129 * 4 : (QKB > 0 ? 2 * kQBBufBytes + 2 * NB * 4 : 0);
+  static constexpr int kXBytes =
+      (EPI == kEpiRouter) ? NB * kRouterPitch * 4 : (QKB > 0 ? 2 * kQBBufBytes + 2 * NB * 4 : 0);
   static_assert(QKB == 0 || (NB * kKBlockBytes) % 1024 == 0, "resident K-blocks sit on 1 KB boundaries");
   static constexpr int kStagesRaw = (196 * 1024 - kXBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
@@ -346,7 +352,7 @@ __device__ __forceinline__ void epilogue_router(const GemmParams& p, const Tile&
       uint32_t r[16];
       tmem_ld16(t_lane + c0 + c16, r);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xs[(c0 + c16 + i) * 129 + lane_row] = __uint_as_float(r[i]);
+      for (int i = 0; i < 16; ++i) xs[(c0 + c16 + i) * kRouterPitch + lane_row] = __uint_as_float(r[i]);
     }
   }
   mbar_arrive(xbar);
@@ -359,7 +365,7 @@ __device__ __forceinline__ void epilogue_router(const GemmParams& p, const Tile&
   for (int tb = ew; tb < c.rows; tb += kEpiWarps * NT) {
     const int nt = min(NT, (c.rows - tb + kEpiWarps - 1) / kEpiWarps);
     const int row = c.tok0 + tb;
-    warp_topk_tokens<PER, NT>([&](int u, int e) { return xs[e * 129 + tb + u * kEpiWarps]; }, nt, E, k,
+    warp_topk_tokens<PER, NT>([&](int u, int e) { return xs[e * kRouterPitch + tb + u * kEpiWarps]; }, nt, E, k,
                               p.renorm != 0, bias, static_cast<int*>(p.out) + size_t(row) * k,
                               p.topk_w + size_t(row) * k, kEpiWarps * k, counts);
   }
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_tc_kernel(const __grid_c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* mt_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + Cfg::kBarBytes);
   int* goff = mt_prefix + (kMaxGroups + 1);
-  float* xs = reinterpret_cast<float*>(goff + (kMaxGroups + 1));  // router: [NB][129] logits
+  float* xs = reinterpret_cast<float*>(goff + (kMaxGroups + 1));  // router: [NB][65] logits
   uint64_t* xbar = drain + 1;  // router: all epilogue threads, two phases per tile
   uint64_t* bready = drain + 2;  // QKB: resident B buffer [2] written (all epilogue threads)
   uint64_t* bfree = drain + 4;   // QKB: resident B buffer [2] read by the tile's MMAs (commit)

@@ -308,7 +308,7 @@ int run_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t
   // them for 8192 tokens), or 32 where that still fits the SMs in one wave (4096 tokens: 128
   // CTAs instead of 64; each CTA streams all of W_gate, so fewer tokens per CTA leave the bytes
   // per CTA nearly unchanged but use twice the SMs)
-  const int kRouterRows = (T + 31) / 32 <= num_sms() ? 32 : 64;
+  const int kRouterRows = (T + 31) / 32 <= num_sms() ? 32 : kRouterMaxRows;
   GemmParams p{};
   if (!make_kmajor_map(&p.tmA, x, true, H, T, kRouterRows) || !make_kmajor_map(&p.tmB, wg, true, H, E, kBBoxRows) ||
       !make_kmajor_map(&p.tmB2, wg, true, H, E, uint32_t(nb)))
