@@ -129,7 +129,9 @@ def test_quantize_int4_exact(N, K):
 @pytest.mark.parametrize("T,H,E,k,renorm,skew", [
     (64, 256, 8, 2, True, False), (64, 2048, 128, 8, True, False), (1, 2048, 128, 8, True, False),
     (300, 1024, 100, 6, False, False), (8192, 2048, 128, 8, True, True), (129, 4096, 128, 8, True, False),
-    (50, 512, 16, 16, True, False), (40, 256, 256, 4, False, False), (33, 128, 1, 1, True, False)])
+    (50, 512, 16, 16, True, False), (40, 256, 256, 4, False, False), (33, 128, 1, 1, True, False),
+    # tensor-core router with 32-token tiles (one wave), a ragged last tile, and at the 235B shape
+    (1000, 2048, 128, 8, True, False), (4096, 4096, 128, 8, True, False)])
 def test_route(T, H, E, k, renorm, skew):
     x = synth.activations(T, H, max(1, H // 100), seed=T)
     wg = synth.router_weight(E, H, seed=E)
