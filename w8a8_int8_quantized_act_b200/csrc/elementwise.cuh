@@ -25,6 +25,50 @@ __global__ void __launch_bounds__(kRowWarps * 32) quant_rows_kernel(const uint16
   if ((threadIdx.x & 31) == 0) scale[r] = s;
 }
 
+// The same quantisation (U > 0) with a grid of resident CTAs: each warp walks rows r, r + stride,
+// ... and loads its next row while it quantises the current one, so every warp keeps a row's
+// loads in flight instead of waiting for them once per row.
+template <int U>
+__device__ __forceinline__ void load_row8(const uint16_t* __restrict__ src, int64_t R, int K, int64_t r, int lane,
+                                          uint4 (&v)[U]) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int i = lane * 8 + u * 256;
+    v[u] = (r < R && i < K) ? __ldg(reinterpret_cast<const uint4*>(src + r * K + i)) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int U>
+__global__ void __launch_bounds__(kRowWarps * 32) quant_rows_stream_kernel(const uint16_t* __restrict__ src,
+                                                                           int64_t R, int K, int8_t* __restrict__ q,
+                                                                           float* __restrict__ scale) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = int64_t(gridDim.x) * kRowWarps;
+  int64_t r = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  uint4 cur[U], nxt[U];
+  load_row8<U>(src, R, K, r, lane, cur);
+  for (; r < R; r += stride) {
+    load_row8<U>(src, R, K, r + stride, lane, nxt);
+    float amax = 0.0f;
+#pragma unroll
+    for (int u = 0; u < U; ++u) amax = fmaxf(amax, amax8(cur[u]));
+    amax = warp_max(amax);
+    const float s = sym_scale(amax, kQMaxInt8);
+    const float inv = __frcp_rn(s);
+    int8_t* dst = q + r * K;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = lane * 8 + u * 256;
+      if (i < K) *reinterpret_cast<uint2*>(dst + i) = quant8(cur[u], s, inv);
+    }
+    if (lane == 0) scale[r] = s;
+#pragma unroll
+    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+  }
+}
+
 // Symmetric int4 per group of 128 along K: one warp per (row, group), 4 values per lane.
 // Byte i of a row holds code 2i (low nibble) and code 2i+1 (high nibble).
 __global__ void __launch_bounds__(kRowWarps * 32) quant_int4_group128_kernel(

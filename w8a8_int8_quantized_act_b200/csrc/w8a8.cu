@@ -416,15 +416,40 @@ int mx_gemm(const uint8_t* xc, const uint8_t* xs, const uint8_t* wc, const uint8
   return launch_pdl(kern, dim3(max(1, min(num_sms(), tiles))), dim3(kMxThreads), kMxSmemBytes, s, p);
 }
 
+// quant_rows_stream_kernel<U> over R rows: as many CTAs as are resident at once (cached per U),
+// fewer for short inputs.
+template <int U>
+int launch_quant_rows_stream(const uint16_t* src, int64_t R, int K, int8_t* q, float* scale, cudaStream_t s) {
+  static const int per_sm = [] {
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, quant_rows_stream_kernel<U>, kRowWarps * 32, 0) !=
+            cudaSuccess ||
+        b < 1)
+      b = 1;
+    return b;
+  }();
+  const int64_t want = (R + kRowWarps - 1) / kRowWarps;
+  const int64_t resident = int64_t(num_sms()) * per_sm;
+  const dim3 grid(unsigned(want < resident ? want : resident)), blk(kRowWarps * 32);
+  return launch_pdl(quant_rows_stream_kernel<U>, grid, blk, 0, s, src, R, K, q, scale);
+}
+
 int launch_quant_rows(const uint16_t* src, int64_t R, int K, int8_t* q, float* scale, cudaStream_t s) {
-  const dim3 grid(unsigned((R + kRowWarps - 1) / kRowWarps)), blk(kRowWarps * 32);
+  // rows of 768 and 1536 values (the h rows of the 30B- and 235B-shaped layers) hold exactly 3
+  // and 6 vectors a lane, which leaves room for more resident warps than 4 and 8
+  const int u = (K + 255) / 256;
+  if (u == 3) return launch_quant_rows_stream<3>(src, R, K, q, scale, s);
+  if (u == 5 || u == 6) return launch_quant_rows_stream<6>(src, R, K, q, scale, s);
   switch (row_units(K)) {
-    case 1: return launch_pdl(quant_rows_kernel<1>, grid, blk, 0, s, src, R, K, q, scale);
-    case 2: return launch_pdl(quant_rows_kernel<2>, grid, blk, 0, s, src, R, K, q, scale);
-    case 4: return launch_pdl(quant_rows_kernel<4>, grid, blk, 0, s, src, R, K, q, scale);
-    case 8: return launch_pdl(quant_rows_kernel<8>, grid, blk, 0, s, src, R, K, q, scale);
-    case 16: return launch_pdl(quant_rows_kernel<16>, grid, blk, 0, s, src, R, K, q, scale);
-    default: return launch_pdl(quant_rows_kernel<0>, grid, blk, 0, s, src, R, K, q, scale);
+    case 1: return launch_quant_rows_stream<1>(src, R, K, q, scale, s);
+    case 2: return launch_quant_rows_stream<2>(src, R, K, q, scale, s);
+    case 4: return launch_quant_rows_stream<4>(src, R, K, q, scale, s);
+    case 8: return launch_quant_rows_stream<8>(src, R, K, q, scale, s);
+    case 16: return launch_quant_rows_stream<16>(src, R, K, q, scale, s);
+    default: {
+      const dim3 grid(unsigned((R + kRowWarps - 1) / kRowWarps)), blk(kRowWarps * 32);
+      return launch_pdl(quant_rows_kernel<0>, grid, blk, 0, s, src, R, K, q, scale);
+    }
   }
 }
 
