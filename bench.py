@@ -591,21 +591,21 @@ def time_linear_gemm(B, x, copies, fmt, group, wl, steps, stream):
 # the kernel). Keys: workload name.
 MEASURED_TRAFFIC = {
     # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum on the gate_up launch of the
-    # Qwen3-235B-A22B-shaped layer (1 pass, full workload): 1905.0 MB read + 97.5 MB written
-    "qwen3-235b-a22b": (1_905_008_128 + 97_517_312, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
+    # Qwen3-235B-A22B-shaped layer (1 pass, full workload): 1906.3 MB read + 97.3 MB written
+    "qwen3-235b-a22b": (1_906_306_560 + 97_287_424, "43cc740bc128bff5c184ea5be0154d9b92498849"),
     # the same two metrics on the gate_up launch of the 30B-shaped layers: decode (T = 64)
-    # 392.0 MB read + 3.6 MB written; prefill (T = 8192) 538.6 MB read + 88.7 MB written
-    "qwen3-30b-a3b-decode": (391_984_896 + 3_580_160, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
-    "qwen3-30b-a3b-prefill": (538_649_344 + 88_734_976, "7cd9696ca59c5723202a4fc4c61ad9433431d5aa"),
+    # 392.0 MB read + 3.9 MB written; prefill (T = 8192) 538.7 MB read + 88.7 MB written
+    "qwen3-30b-a3b-decode": (391_971_072 + 3_937_280, "43cc740bc128bff5c184ea5be0154d9b92498849"),
+    "qwen3-30b-a3b-prefill": (538_654_208 + 88_660_224, "43cc740bc128bff5c184ea5be0154d9b92498849"),
     # the W4A8 GEMM launch of the 2048 x 2048 -> 6144 linear: 10.9 MB read (weights, scales, token
     # codes once), nothing written back to DRAM within the launch (the 25 MB output stays in L2)
-    "qwen3-1.7b-mlp-w4a8": (10_933_760 + 0, "1b4b2dc7d15bec2e91ed021dfeeca923eb8d5b51"),
+    "qwen3-1.7b-mlp-w4a8": (10_932_992 + 0, "3d048a51e1c8030a8b0a8441792e2ca2d2309450"),
     # the block-scaled MXFP8 GEMM launch (CTA pairs) of the same shape: 17.3 MB read (FP8 weights
-    # and scales, token codes and scales, each once), 10 KB written back within the launch
-    "qwen3-1.7b-mlp-mxfp8": (17_344_000 + 9_728, "1b6af13e5f0c640ee94589284d53110f6163846a"),
+    # and scales, token codes and scales, each once), nothing written back within the launch
+    "qwen3-1.7b-mlp-mxfp8": (17_344_000 + 0, "06a20b9f7bcec6397d7ecc1af2a1ebdc06f40292"),
     # the MXFP A8W4 GEMM launch of the same shape: 11.1 MB read (6.3 MB of packed E2M1 weights, their
     # scales, the token codes and scales, each once), nothing written back within the launch
-    "qwen3-1.7b-mlp-mxfp-a8w4": (11_052_544 + 0, "1b6af13e5f0c640ee94589284d53110f6163846a"),
+    "qwen3-1.7b-mlp-mxfp-a8w4": (11_052_544 + 0, "06a20b9f7bcec6397d7ecc1af2a1ebdc06f40292"),
 }
 TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),
