@@ -161,6 +161,54 @@ int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
                      int k, int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
                      w8a8_stream stream);
 
+/* ---- Expert parallelism: the forward split at its two exchange points ----------------------
+ * Defined by: "Qwen3-235B-A22B-quantized.w8a8" file-structure explainer, the model table (128
+ * experts, 8 per token) and the shard index section (the weights are sharded so that several cards
+ * load and serve the model together). Read as expert parallelism: rank r of W holds experts
+ * [r E/W, (r+1) E/W); each rank routes its own tokens, sends every assignment's int8 row and fp32
+ * scale to the rank of its expert, runs the expert FFN on what it receives, and gets the bf16
+ * expert outputs back for its ordered combine. Every step is row-wise, so the result equals
+ * w8a8_moe_forward on the same tokens bit for bit. The exchanges themselves are the caller's
+ * (the package's ep.py uses torch.distributed all-to-all); these entries are the compute between.
+ *
+ * w8a8_moe_route_group: steps 1 and 2 of w8a8_moe_forward on T local tokens (router, softmax,
+ * top-k, grouping by global expert, per-token int8 quantisation into the sorted rows). The
+ * workspace has the layout w8a8_moe_workspace_layout(T, H, E, k, 128, .) gives and at least its
+ * total; the call fills topk_ids, topk_w, offsets (sorted rows of each global expert; with experts
+ * in contiguous blocks per rank, the rows for each destination rank are consecutive), perm, sx,
+ * sx_sorted and xq. Shape rules and errors as w8a8_moe_forward. */
+int w8a8_moe_route_group(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
+                         int k, int renorm, void* workspace, size_t workspace_bytes, w8a8_stream stream);
+
+/* Workspace bytes of w8a8_moe_experts for A rows in G groups (0 if rejected: H or I not a
+ * multiple of 128, G outside [1, 1024]). */
+size_t w8a8_moe_experts_workspace_size(int64_t A, int64_t H, int64_t I, int64_t G);
+
+/* Steps 3-5 of w8a8_moe_forward on A received rows: grouped gate_up GEMM with dequant and
+ * SiLU(gate)*up, per-row requantisation of h, grouped down GEMM with dequant, o [A, H] bf16 in
+ * row order.
+ *   xq int8 [round_up(A, 128), H] (16-byte aligned; rows past A are read, not used) and sx fp32 [A]:
+ *   the rows and their per-token scales; group_offsets_host: HOST array [G+1], offsets[0] = 0,
+ *   non-decreasing, offsets[G] = A (else W8A8_ERR_ARG), group g = rows [offsets[g], offsets[g+1]);
+ *   group g uses expert g % weight_groups of the Ew experts in wgu [Ew, 2I, H] / s_gu [Ew, 2I] /
+ *   wd [Ew, H, I] / s_d [Ew, H] (weight_groups 0: expert g, G <= Ew) -- with W source ranks and
+ *   E/W local experts, G = W * E/W groups in source-major order and weight_groups = E/W;
+ *   workspace of w8a8_moe_experts_workspace_size(A, H, I, G) bytes (256-byte aligned).
+ *   Ew <= 256. All device memory except group_offsets_host owned by the caller. */
+int w8a8_moe_experts(const int8_t* xq, const float* sx, const int* group_offsets_host, int64_t G,
+                     int64_t weight_groups, int64_t A, int64_t H, int64_t I, int64_t Ew, const int8_t* wgu,
+                     const float* s_gu, const int8_t* wd, const float* s_d, void* workspace, size_t workspace_bytes,
+                     w8a8_bf16* o, w8a8_stream stream);
+
+/* Step 6 of w8a8_moe_forward from expert outputs in sorted-row order: o_sorted [T*k, H] bf16 (row
+ * r = sorted row r, as w8a8_moe_route_group ordered them), perm and topk_w from the same call;
+ * o_slots [T*k, H] bf16 is scratch (receives the rows in slot order t*k + j); y [T, H] bf16 =
+ * bf16(fma chain over j = 0..k-1 of topk_w[t, j] * o[t, j, :]). A perm entry outside [0, T*k) sets
+ * the device error word (W8A8_ERR_DEVICE at the next w8a8_check_status) and its row is skipped.
+ * H % 128 == 0, k <= 16. */
+int w8a8_moe_combine_sorted(const w8a8_bf16* o_sorted, const int* perm, const float* topk_w, int64_t T, int64_t H,
+                            int k, w8a8_bf16* o_slots, w8a8_bf16* y, w8a8_stream stream);
+
 /* Workspace of w8a8_moe_forward_shared: the routed layer's regions (as w8a8_moe_ws_layout gives
  * them for the same T, H, E, k, I) followed by the shared expert's (every region 256-byte aligned):
  *   xq int8 [T, H] and sx fp32 [T] (per-token codes and scales of x, token order);

@@ -96,6 +96,24 @@ def test_argument_checks_reject_before_any_launch(lib):
         B.W8A8_ERR_UNSUPPORTED  # packed weights not 32-byte aligned (the 4-bit TMA type needs it)
     assert lib.w8a8_mxfp_a8w4_linear_prequant(c(256), c(256), c(256), c(256), 8, 128, 200, c(256), None) == \
         B.W8A8_ERR_UNSUPPORTED  # N % 128
+    # expert-parallel entries: shapes, offsets and pointers are checked on the host
+    assert lib.w8a8_moe_route_group(None, None, None, 8, 200, 8, 2, 1, None, 0, None) == B.W8A8_ERR_UNSUPPORTED
+    assert lib.w8a8_moe_route_group(None, None, None, 0, 256, 8, 2, 1, None, 0, None) == B.W8A8_OK  # empty
+    assert lib.w8a8_moe_route_group(c(256), c(256), None, 8, 256, 8, 2, 1, c(256), 10, None) == B.W8A8_ERR_WORKSPACE
+    assert B.w8a8_moe_experts_workspace_size(100, 256, 128, 8) > 0
+    assert B.w8a8_moe_experts_workspace_size(100, 200, 128, 8) == 0  # H % 128
+    assert B.w8a8_moe_experts_workspace_size(100, 256, 128, 1025) == 0  # more than 1024 groups
+    offs = (ctypes.c_int * 3)(0, 4, 3)
+    assert lib.w8a8_moe_experts(c(256), c(256), offs, 2, 2, 3, 256, 128, 2, c(256), c(256), c(256), c(256),
+                                c(256), 1 << 20, c(256), None) == B.W8A8_ERR_ARG  # decreasing offsets
+    offs = (ctypes.c_int * 3)(0, 4, 9)
+    assert lib.w8a8_moe_experts(c(256), c(256), offs, 2, 3, 9, 256, 128, 2, c(256), c(256), c(256), c(256),
+                                c(256), 1 << 20, c(256), None) == B.W8A8_ERR_ARG  # weight_groups > Ew
+    assert lib.w8a8_moe_experts(c(256), c(256), offs, 2, 2, 9, 256, 128, 2, c(256), c(256), c(256), c(256),
+                                c(256), 10, c(256), None) == B.W8A8_ERR_WORKSPACE
+    assert lib.w8a8_moe_combine_sorted(c(256), c(256), c(256), 4, 200, 2, c(256), c(256), None) == \
+        B.W8A8_ERR_UNSUPPORTED  # H % 128
+    assert lib.w8a8_moe_combine_sorted(None, None, None, 4, 256, 2, None, None, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_debug_wait_timeout(0, None) == B.W8A8_ERR_ARG
     assert lib.w8a8_debug_rcp_approx_ulp(0, 10, c(16), None) == B.W8A8_ERR_ARG  # not a normal input
     assert lib.w8a8_debug_rcp_approx_ulp(0x7E7FFFFF, 2, c(16), None) == B.W8A8_ERR_ARG  # reciprocal subnormal

@@ -77,6 +77,11 @@ SIGNATURES = {
     "w8a8_mxfp8_linear": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, ctypes.c_size_t, _c_p, _c_p]),
     "w8a8_mxfp8_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_mxfp4_quantize": (_int, [_c_p, _i64, _i64, _c_p, _c_p, _c_p]),
+    "w8a8_moe_route_group": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _int, _int, _c_p, ctypes.c_size_t, _c_p]),
+    "w8a8_moe_experts_workspace_size": (ctypes.c_size_t, [_i64, _i64, _i64, _i64]),
+    "w8a8_moe_experts": (_int, [_c_p, _c_p, ctypes.POINTER(ctypes.c_int), _i64, _i64, _i64, _i64, _i64, _i64, _c_p,
+                                _c_p, _c_p, _c_p, _c_p, ctypes.c_size_t, _c_p, _c_p]),
+    "w8a8_moe_combine_sorted": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _int, _c_p, _c_p, _c_p]),
     "w8a8_mxfp_a8w4_linear": (_int, [_c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, ctypes.c_size_t, _c_p, _c_p]),
     "w8a8_mxfp_a8w4_linear_prequant": (_int, [_c_p, _c_p, _c_p, _c_p, _i64, _i64, _i64, _c_p, _c_p]),
     "w8a8_debug_wait_timeout": (_int, [ctypes.c_uint64, _c_p]),
@@ -313,6 +318,56 @@ def w8a8_moe_forward_profiled(x, wg, wgu, s_gu, wd, s_d, k: int, events, renorm:
                                            _ptr(s_d), T, H, E, k, I, int(renorm), _ptr(workspace),
                                            workspace.numel(), _ptr(y), _stream(stream), arr),
            "w8a8_moe_forward_profiled")
+    return y
+
+
+def w8a8_moe_route_group(x, wg, E: int, k: int, renorm: bool = True, bias=None, workspace=None, stream=None):
+    """Steps 1-2 of the forward on local tokens; returns the workspace (the layout of
+    w8a8_moe_workspace_layout(T, H, E, k, 128)) whose topk_ids, topk_w, offsets, perm, sx_sorted and
+    xq moe_intermediates(workspace, T, H, E, k, 128) views."""
+    _bf16(x), _bf16(wg)
+    T, H = x.shape
+    ws_bytes = w8a8_moe_workspace_size(T, H, E, k, 128)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=x.device)
+    _check(lib().w8a8_moe_route_group(_ptr(x), _ptr(wg), _ptr(bias), T, H, E, k, int(renorm), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "w8a8_moe_route_group")
+    return workspace
+
+
+def w8a8_moe_experts_workspace_size(A: int, H: int, I: int, G: int) -> int:
+    return int(lib().w8a8_moe_experts_workspace_size(A, H, I, G))
+
+
+def w8a8_moe_experts(xq, sx, group_offsets, wgu, s_gu, wd, s_d, weight_groups: int = 0, A: int = None,
+                     workspace=None, o=None, stream=None):
+    """Steps 3-5 on received rows: xq int8 [>= round_up(A, 128), H], sx fp32 [A], group_offsets a
+    host sequence of G+1 ints; group g uses expert g % weight_groups (0: g). Returns o bf16 [A, H]."""
+    H = xq.shape[1]
+    Ew, twoI, _ = wgu.shape
+    I = twoI // 2
+    offs = [int(v) for v in group_offsets]
+    G = len(offs) - 1
+    A = offs[-1] if A is None else A
+    need = w8a8_moe_experts_workspace_size(A, H, I, G)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=xq.device)
+    o = torch.empty((A, H), dtype=torch.bfloat16, device=xq.device) if o is None else o
+    arr = (ctypes.c_int * (G + 1))(*offs)
+    _check(lib().w8a8_moe_experts(_ptr(xq), _ptr(sx), arr, G, weight_groups, A, H, I, Ew, _ptr(wgu), _ptr(s_gu),
+                                  _ptr(wd), _ptr(s_d), _ptr(workspace), workspace.numel(), _ptr(o),
+                                  _stream(stream)), "w8a8_moe_experts")
+    return o
+
+
+def w8a8_moe_combine_sorted(o_sorted, perm, topk_w, k: int, o_slots=None, y=None, stream=None):
+    """Step 6 from expert outputs in sorted-row order: y bf16 [T, H]."""
+    A, H = o_sorted.shape
+    T = A // k
+    o_slots = torch.empty_like(o_sorted) if o_slots is None else o_slots
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=o_sorted.device) if y is None else y
+    _check(lib().w8a8_moe_combine_sorted(_ptr(o_sorted), _ptr(perm), _ptr(topk_w), T, H, k, _ptr(o_slots), _ptr(y),
+                                         _stream(stream)), "w8a8_moe_combine_sorted")
     return y
 
 

@@ -205,6 +205,27 @@ __global__ void __launch_bounds__(kPermThreads) group_quant_kernel(
   }
 }
 
+// dst[map[r], :] = src[r, :] for r < R, rows of `row_bytes` bytes (a multiple of 16, both buffers
+// 16-byte aligned): one warp per row. A map value outside [0, dst_rows) sets the bad-index bit of
+// the device error word and the row is skipped.
+__global__ void __launch_bounds__(kRowWarps * 32) scatter_rows_kernel(const uint8_t* __restrict__ src,
+                                                                      const int* __restrict__ map, int64_t R,
+                                                                      int row_bytes, uint8_t* __restrict__ dst,
+                                                                      int64_t dst_rows) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t r = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (r >= R) return;
+  const int d = __ldg(map + r);
+  if (d < 0 || d >= dst_rows) {
+    if ((threadIdx.x & 31) == 0) atomicOr(&g_error_word, kErrBadIndex);
+    return;
+  }
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + r * row_bytes);
+  uint4* d4 = reinterpret_cast<uint4*>(dst + int64_t(d) * row_bytes);
+  for (int i = threadIdx.x & 31; i < row_bytes / 16; i += 32) d4[i] = __ldg(s4 + i);
+}
+
 // y[t, :] = bf16(sum_j w[t, j] * o[t, j, :]): fp32 fused multiply-adds in slot order from 0.
 // With a shared expert (o_shared != nullptr) one more fused multiply-add follows the k slots:
 // acc = fma(g[t], o_shared[t, :], acc).

@@ -694,6 +694,182 @@ int dense_gate_up(const int8_t* xq, const float* sx, const int8_t* wgu, const fl
   return launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, int((T + 31) / 32) * p.n_cb, s);
 }
 
+// Steps 1 and 2 of the forward: routing, the grouping of the T*k assignments by expert and the
+// per-token quantisation into the sorted rows, into the workspace regions of L.
+int route_group_stage(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
+                      int k, int renorm, uint8_t* ws, const w8a8_moe_ws_layout& L, cudaStream_t s,
+                      void* const* ev) {
+  int* ids = reinterpret_cast<int*>(ws + L.topk_ids);
+  float* w = reinterpret_cast<float*>(ws + L.topk_w);
+  int* tile_counts = reinterpret_cast<int*>(ws + L.tile_counts);
+  int* offsets = reinterpret_cast<int*>(ws + L.offsets);
+  int* perm = reinterpret_cast<int*>(ws + L.perm);
+  float* sx = reinterpret_cast<float*>(ws + L.sx);
+  float* sx_sorted = reinterpret_cast<float*>(ws + L.sx_sorted);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
+  const int C = int((T + kChunk - 1) / kChunk);
+  int rc;
+  if (T <= kFrontMaxT && H <= kFrontMaxH) {
+    // short batch: routing, grouping and quantisation in one cooperative launch
+    mark(ev, 0, s);
+    unsigned* sync = reinterpret_cast<unsigned*>(ws + L.sync);
+    if (cudaMemsetAsync(sync, 0, sizeof(unsigned), s) != cudaSuccess) return W8A8_ERR_LAUNCH;
+    rc = launch_front_small(x, wg, bias, int(T), int(H), int(E), k, renorm, reinterpret_cast<float*>(ws + L.logits),
+                            sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
+    if (rc != W8A8_OK) return rc;
+    mark(ev, 1, s);
+    return W8A8_OK;
+  }
+  // 1. router (bf16 tcgen05 GEMM + softmax / top-k epilogue, per-chunk expert histogram)
+  mark(ev, 0, s);
+  rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E, reinterpret_cast<float*>(ws + L.logits),
+                  s);
+  if (rc != W8A8_OK) return rc;
+  // 2. group assignments by expert and quantise every token once into its sorted rows
+  const size_t gq_smem = sizeof(int) * (2 * E + 2 * kChunk * k + 4 * E);
+  mark(ev, 1, s);
+  return launch_group_quant(dim3(C, group_quant_splits()), gq_smem, s, x, ids, tile_counts, int(T), int(H), int(E),
+                            k, offsets, perm, sx, sx_sorted, xq);
+}
+
+// Operands of the grouped expert FFN: A sorted token rows xq [round_up(A, 128), H] with their
+// scales, G groups of consecutive rows (offsets [G+1] on the device), the intermediates h, s_h, hq
+// (round_up(A, 128) rows) and the output o; row_map sends sorted row r to output row row_map[r]
+// (nullptr: row r).
+struct ExpertRows {
+  const int8_t* xq;
+  const float* sx;
+  const int* offsets;
+  uint16_t* h;
+  float* s_h;
+  int8_t* hq;
+  uint16_t* o;
+  const int* row_map;
+};
+
+// Steps 3-5 of the forward: grouped gate_up with dequant + SiLU(gate)*up, the requantisation of h,
+// grouped down with dequant. Group g uses the weights and scales of expert g % weight_groups
+// (weight_groups 0: expert g); Ew experts are held in wgu [Ew, 2I, H] / wd [Ew, H, I].
+int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t weight_groups, int64_t Ew, int64_t H, int64_t I,
+                  const int8_t* wgu, const float* s_gu, const int8_t* wd, const float* s_d, cudaStream_t s,
+                  void* const* ev) {
+  const int64_t Ap = round_up(A > 0 ? A : 1, 128);
+  int rc;
+  // Few rows per group (decode): the expert GEMMs run one CTA per tile of <= 32 sorted rows;
+  // otherwise CTA pairs on tiles of <= 256 rows.
+  const bool small = small_token_blocks(A, G);
+
+  // 3. grouped gate_up GEMM (weights on M, tokens on N) with the dequant + SiLU(gate)*up
+  //    epilogue -> h
+  if (small) {
+    GemmParams p{};
+    if (!make_kmajor_map(&p.tmA, wgu, false, H, uint64_t(Ew) * 2 * I, 128) ||
+        !make_kmajor_map(&p.tmB, b.xq, false, H, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, b.xq, false, H, Ap, 32))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(H / 128);
+    p.n_cb = int(I / 128);
+    p.num_groups = int(G);
+    p.group_offsets = b.offsets;
+    p.weight_groups = int(weight_groups);
+    p.a_rows_per_group = int(2 * I);
+    p.a_second_offset = int(I);
+    p.a_cb_step = 128;
+    p.timeout_ns = wait_timeout_ns();
+    p.out = b.h;
+    p.ldo = int(I);
+    p.row_scale = b.sx;
+    p.col_scale = s_gu;
+    p.col_scale_stride = int(2 * I);
+    p.up_offset = int(I);
+    const int tiles = max_token_blocks(A, G, 32) * p.n_cb;
+    mark(ev, 2, s);
+    if ((rc = launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, tiles, s)) != W8A8_OK) return rc;
+  } else {
+    PairParams p{};
+    if (!make_gate_up_pair_map(&p.tmA, wgu, H, I, Ew) || !make_pair_b_maps(&p, b.xq, H, Ap))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(H / 128);
+    p.n_cb = int(I / 128);
+    p.num_groups = int(G);
+    p.group_offsets = b.offsets;
+    p.weight_groups = int(weight_groups);
+    p.a_rows_per_group = int(2 * I);
+    p.n_channels = int(I);
+    p.timeout_ns = wait_timeout_ns();
+    p.out = b.h;
+    p.ldo = int(I);
+    p.row_scale = b.sx;
+    p.col_scale = s_gu;
+    p.col_scale_stride = int(2 * I);
+    p.up_offset = int(I);
+    const int tiles = max_token_blocks(A, G, kPairNB) * p.n_cb;
+    mark(ev, 2, s);
+    if ((rc = launch_pair<kEpiGateUp>(p, tiles, s)) != W8A8_OK) return rc;
+  }
+
+  // 4. per-row requantisation of h: inside the down GEMM for short token lists with rows of up
+  //    to 1024 values (each CTA quantises its tile's rows into shared memory), else a launch of
+  //    its own
+  const bool rq_in_down = small && I <= 1024;
+  mark(ev, 3, s);
+  if (!rq_in_down && (rc = launch_quant_rows(b.h, A, int(I), b.hq, b.s_h, s)) != W8A8_OK) return rc;
+
+  // 5. grouped down GEMM with the dequant epilogue -> o (rows through row_map)
+  if (small) {
+    GemmParams p{};
+    if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(Ew) * H, 128) ||
+        !make_kmajor_map(&p.tmB, b.hq, false, I, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, b.hq, false, I, Ap, 32))
+      return W8A8_ERR_UNSUPPORTED;
+    p.num_kb = int(I / 128);
+    p.n_cb = int((H + 255) / 256);
+    p.n_channels = int(H);
+    p.num_groups = int(G);
+    p.group_offsets = b.offsets;
+    p.weight_groups = int(weight_groups);
+    p.a_rows_per_group = int(H);
+    p.a_second_offset = 128;
+    p.a_cb_step = 256;
+    p.timeout_ns = wait_timeout_ns();
+    p.out = b.o;
+    p.ldo = int(H);
+    p.row_scale = b.s_h;
+    p.col_scale = s_d;
+    p.col_scale_stride = int(H);
+    p.row_map = b.row_map;
+    const int tiles = max_token_blocks(A, G, 32) * p.n_cb;
+    mark(ev, 4, s);
+    if (rq_in_down) {
+      p.qb_h = b.h;
+      p.qb_hq = b.hq;
+      p.qb_s = b.s_h;
+      rc = launch_gemm<2, 32, kEpiDown, kKindI8, 8>(p, tiles, s);
+    } else {
+      rc = launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s);
+    }
+    return rc;
+  }
+  PairParams p{};
+  if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(Ew) * H, 128) || !make_pair_b_maps(&p, b.hq, I, Ap))
+    return W8A8_ERR_UNSUPPORTED;
+  p.num_kb = int(I / 128);
+  p.n_cb = int((H + 255) / 256);
+  p.n_channels = int(H);
+  p.num_groups = int(G);
+  p.group_offsets = b.offsets;
+  p.weight_groups = int(weight_groups);
+  p.a_rows_per_group = int(H);
+  p.timeout_ns = wait_timeout_ns();
+  p.out = b.o;
+  p.ldo = int(H);
+  p.row_scale = b.s_h;
+  p.col_scale = s_d;
+  p.col_scale_stride = int(H);
+  p.row_map = b.row_map;
+  const int tiles = max_token_blocks(A, G, kPairNB) * p.n_cb;
+  mark(ev, 4, s);
+  return launch_pair<kEpiDown>(p, tiles, s);
+}
+
 int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, const int8_t* wgu,
                      const float* s_gu, const int8_t* wd, const float* s_d, int64_t T, int64_t H, int64_t E, int k,
                      int64_t I, int renorm, void* workspace, size_t workspace_bytes, w8a8_bf16* y,
@@ -715,12 +891,9 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   const w8a8_moe_ws_layout& L = SL.routed;
   if (workspace_bytes < (sh != nullptr ? SL.total : L.total)) return W8A8_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int* ids = reinterpret_cast<int*>(ws + L.topk_ids);
   float* w = reinterpret_cast<float*>(ws + L.topk_w);
-  int* tile_counts = reinterpret_cast<int*>(ws + L.tile_counts);
   int* offsets = reinterpret_cast<int*>(ws + L.offsets);
   int* perm = reinterpret_cast<int*>(ws + L.perm);
-  float* sx = reinterpret_cast<float*>(ws + L.sx);
   float* sx_sorted = reinterpret_cast<float*>(ws + L.sx_sorted);
   int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
   uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
@@ -729,143 +902,10 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   uint16_t* o = reinterpret_cast<uint16_t*>(ws + L.o);
   cudaStream_t s = as_stream(stream);
   const int64_t A = T * k;
-  const int64_t Ap = round_up(A, 128);
-  const int C = int((T + kChunk - 1) / kChunk);
-  int rc;
-
-  // Few rows per expert (decode): the expert GEMMs run one CTA per tile of <= 32 sorted rows;
-  // otherwise CTA pairs on tiles of <= 256 rows.
-  const bool small = small_token_blocks(A, E);
-  if (T <= kFrontMaxT && H <= kFrontMaxH) {
-    // 1+2. short batch: routing, grouping and quantisation in one cooperative launch
-    mark(ev, 0, s);
-    unsigned* sync = reinterpret_cast<unsigned*>(ws + L.sync);
-    if (cudaMemsetAsync(sync, 0, sizeof(unsigned), s) != cudaSuccess) return W8A8_ERR_LAUNCH;
-    rc = launch_front_small(x, wg, bias, int(T), int(H), int(E), k, renorm, reinterpret_cast<float*>(ws + L.logits),
-                            sync, ids, w, tile_counts, offsets, perm, sx, sx_sorted, xq, s);
-    if (rc != W8A8_OK) return rc;
-    mark(ev, 1, s);
-  } else {
-    // 1. router (bf16 tcgen05 GEMM + softmax / top-k epilogue, per-chunk expert histogram)
-    mark(ev, 0, s);
-    rc = run_router(x, wg, bias, T, H, E, k, renorm, ids, w, tile_counts, E,
-                    reinterpret_cast<float*>(ws + L.logits), s);
-    if (rc != W8A8_OK) return rc;
-
-    // 2. group assignments by expert and quantise every token once into its sorted rows
-    const size_t gq_smem = sizeof(int) * (2 * E + 2 * kChunk * k + 4 * E);
-    mark(ev, 1, s);
-    rc = launch_group_quant(dim3(C, group_quant_splits()), gq_smem, s, x, ids, tile_counts, int(T), int(H),
-                            int(E), k, offsets, perm, sx, sx_sorted, xq);
-    if (rc != W8A8_OK) return rc;
-  }
-
-  // 3. grouped gate_up GEMM (weights on M, tokens on N) with the dequant + SiLU(gate)*up
-  //    epilogue -> h
-  if (small) {
-    GemmParams p{};
-    if (!make_kmajor_map(&p.tmA, wgu, false, H, uint64_t(E) * 2 * I, 128) ||
-        !make_kmajor_map(&p.tmB, xq, false, H, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, xq, false, H, Ap, 32))
-      return W8A8_ERR_UNSUPPORTED;
-    p.num_kb = int(H / 128);
-    p.n_cb = int(I / 128);
-    p.num_groups = int(E);
-    p.group_offsets = offsets;
-    p.a_rows_per_group = int(2 * I);
-    p.a_second_offset = int(I);
-    p.a_cb_step = 128;
-    p.timeout_ns = wait_timeout_ns();
-    p.out = h;
-    p.ldo = int(I);
-    p.row_scale = sx_sorted;
-    p.col_scale = s_gu;
-    p.col_scale_stride = int(2 * I);
-    p.up_offset = int(I);
-    const int tiles = max_token_blocks(A, E, 32) * p.n_cb;
-    mark(ev, 2, s);
-    if ((rc = launch_gemm<2, 32, kEpiGateUp, kKindI8>(p, tiles, s)) != W8A8_OK) return rc;
-  } else {
-    PairParams p{};
-    if (!make_gate_up_pair_map(&p.tmA, wgu, H, I, E) || !make_pair_b_maps(&p, xq, H, Ap))
-      return W8A8_ERR_UNSUPPORTED;
-    p.num_kb = int(H / 128);
-    p.n_cb = int(I / 128);
-    p.num_groups = int(E);
-    p.group_offsets = offsets;
-    p.a_rows_per_group = int(2 * I);
-    p.n_channels = int(I);
-    p.timeout_ns = wait_timeout_ns();
-    p.out = h;
-    p.ldo = int(I);
-    p.row_scale = sx_sorted;
-    p.col_scale = s_gu;
-    p.col_scale_stride = int(2 * I);
-    p.up_offset = int(I);
-    const int tiles = max_token_blocks(A, E, kPairNB) * p.n_cb;
-    mark(ev, 2, s);
-    if ((rc = launch_pair<kEpiGateUp>(p, tiles, s)) != W8A8_OK) return rc;
-  }
-
-  // 4. per-row requantisation of h: inside the down GEMM for short token lists with rows of up
-  //    to 1024 values (each CTA quantises its tile's rows into shared memory), else a launch of
-  //    its own
-  const bool rq_in_down = small && I <= 1024;
-  mark(ev, 3, s);
-  if (!rq_in_down && (rc = launch_quant_rows(h, A, int(I), hq, s_h, s)) != W8A8_OK) return rc;
-
-  // 5. grouped down GEMM with the dequant epilogue -> o in slot order
-  if (small) {
-    GemmParams p{};
-    if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(E) * H, 128) ||
-        !make_kmajor_map(&p.tmB, hq, false, I, Ap, kBBoxRows) || !make_kmajor_map(&p.tmB2, hq, false, I, Ap, 32))
-      return W8A8_ERR_UNSUPPORTED;
-    p.num_kb = int(I / 128);
-    p.n_cb = int((H + 255) / 256);
-    p.n_channels = int(H);
-    p.num_groups = int(E);
-    p.group_offsets = offsets;
-    p.a_rows_per_group = int(H);
-    p.a_second_offset = 128;
-    p.a_cb_step = 256;
-    p.timeout_ns = wait_timeout_ns();
-    p.out = o;
-    p.ldo = int(H);
-    p.row_scale = s_h;
-    p.col_scale = s_d;
-    p.col_scale_stride = int(H);
-    p.row_map = perm;
-    const int tiles = max_token_blocks(A, E, 32) * p.n_cb;
-    mark(ev, 4, s);
-    if (rq_in_down) {
-      p.qb_h = h;
-      p.qb_hq = hq;
-      p.qb_s = s_h;
-      rc = launch_gemm<2, 32, kEpiDown, kKindI8, 8>(p, tiles, s);
-    } else {
-      rc = launch_gemm<2, 32, kEpiDown, kKindI8>(p, tiles, s);
-    }
-    if (rc != W8A8_OK) return rc;
-  } else {
-    PairParams p{};
-    if (!make_kmajor_map(&p.tmA, wd, false, I, uint64_t(E) * H, 128) || !make_pair_b_maps(&p, hq, I, Ap))
-      return W8A8_ERR_UNSUPPORTED;
-    p.num_kb = int(I / 128);
-    p.n_cb = int((H + 255) / 256);
-    p.n_channels = int(H);
-    p.num_groups = int(E);
-    p.group_offsets = offsets;
-    p.a_rows_per_group = int(H);
-    p.timeout_ns = wait_timeout_ns();
-    p.out = o;
-    p.ldo = int(H);
-    p.row_scale = s_h;
-    p.col_scale = s_d;
-    p.col_scale_stride = int(H);
-    p.row_map = perm;
-    const int tiles = max_token_blocks(A, E, kPairNB) * p.n_cb;
-    mark(ev, 4, s);
-    if ((rc = launch_pair<kEpiDown>(p, tiles, s)) != W8A8_OK) return rc;
-  }
+  int rc = route_group_stage(x, wg, bias, T, H, E, k, renorm, ws, L, s, ev);
+  if (rc != W8A8_OK) return rc;
+  ExpertRows b{xq, sx_sorted, offsets, h, s_h, hq, o, perm};
+  if ((rc = experts_stage(b, A, E, 0, E, H, I, wgu, s_gu, wd, s_d, s, ev)) != W8A8_OK) return rc;
 
   // 5b. the shared expert (every token): its bf16 gate, per-token int8 x, the dense gate_up GEMM
   //     with the SiLU*up epilogue, the requantisation of its h, the dense down GEMM
@@ -934,6 +974,80 @@ int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
                      w8a8_stream stream) {
   return moe_forward_impl(x, wg, bias, wgu, s_gu, wd, s_d, T, H, E, k, I, renorm, workspace, workspace_bytes, y,
                           stream, nullptr);
+}
+
+// ------------------------------------------------------------------ expert-parallel building blocks
+int w8a8_moe_route_group(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
+                         int k, int renorm, void* workspace, size_t workspace_bytes, w8a8_stream stream) {
+  const int st = check_moe_shape(T, H, E, k, 128);
+  if (st != W8A8_OK) return st;
+  if (T == 0) return W8A8_OK;
+  if (!x || !wg || !workspace) return W8A8_ERR_ARG;
+  if (!aligned16(x) || !aligned16(wg) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return W8A8_ERR_UNSUPPORTED;
+  w8a8_moe_ws_layout L;
+  fill_layout(T, H, E, k, 128, &L);
+  if (workspace_bytes < L.total) return W8A8_ERR_WORKSPACE;  // the forward's layout with I = 128
+  return route_group_stage(x, wg, bias, T, H, E, k, renorm, static_cast<uint8_t*>(workspace), L,
+                           as_stream(stream), nullptr);
+}
+
+size_t w8a8_moe_experts_workspace_size(int64_t A, int64_t H, int64_t I, int64_t G) {
+  if (A < 0 || H <= 0 || I <= 0 || G <= 0 || H % 128 || I % 128 || G > kMaxGroups) return 0;
+  if (A >= (int64_t(1) << 30)) return 0;
+  const size_t Ap = size_t(round_up(A > 0 ? A : 1, 128));
+  return align256(sizeof(int) * size_t(G + 1)) + align256(Ap * I * 2) + align256(sizeof(float) * Ap) +
+         align256(Ap * I);
+}
+
+int w8a8_moe_experts(const int8_t* xq, const float* sx, const int* group_offsets_host, int64_t G,
+                     int64_t weight_groups, int64_t A, int64_t H, int64_t I, int64_t Ew, const int8_t* wgu,
+                     const float* s_gu, const int8_t* wd, const float* s_d, void* workspace, size_t workspace_bytes,
+                     w8a8_bf16* o, w8a8_stream stream) {
+  if (A < 0 || H <= 0 || I <= 0 || G <= 0 || Ew <= 0 || weight_groups < 0) return W8A8_ERR_ARG;
+  const size_t need = w8a8_moe_experts_workspace_size(A, H, I, G);
+  if (need == 0 || Ew > 256 || Ew * 2 * I >= (int64_t(1) << 31) || Ew * H >= (int64_t(1) << 31))
+    return W8A8_ERR_UNSUPPORTED;
+  if (weight_groups > Ew || (weight_groups == 0 && G > Ew)) return W8A8_ERR_ARG;
+  if (!group_offsets_host) return W8A8_ERR_ARG;
+  if (group_offsets_host[0] != 0 || group_offsets_host[G] != A) return W8A8_ERR_ARG;
+  for (int64_t g = 0; g < G; ++g)
+    if (group_offsets_host[g + 1] < group_offsets_host[g]) return W8A8_ERR_ARG;
+  if (A == 0) return W8A8_OK;
+  if (!xq || !sx || !wgu || !s_gu || !wd || !s_d || !workspace || !o) return W8A8_ERR_ARG;
+  if (workspace_bytes < need) return W8A8_ERR_WORKSPACE;
+  if (!aligned16(xq) || !aligned16(wgu) || !aligned16(wd) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return W8A8_ERR_UNSUPPORTED;
+  const size_t Ap = size_t(round_up(A, 128));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* offsets = reinterpret_cast<int*>(ws);
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + align256(sizeof(int) * size_t(G + 1)));
+  float* s_h = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(h) + align256(Ap * I * 2));
+  int8_t* hq = reinterpret_cast<int8_t*>(reinterpret_cast<uint8_t*>(s_h) + align256(sizeof(float) * Ap));
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(offsets, group_offsets_host, sizeof(int) * size_t(G + 1), cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return W8A8_ERR_LAUNCH;
+  ExpertRows b{xq, sx, offsets, h, s_h, hq, reinterpret_cast<uint16_t*>(o), nullptr};
+  return experts_stage(b, A, G, weight_groups, Ew, H, I, wgu, s_gu, wd, s_d, s, nullptr);
+}
+
+int w8a8_moe_combine_sorted(const w8a8_bf16* o_sorted, const int* perm, const float* topk_w, int64_t T, int64_t H,
+                            int k, w8a8_bf16* o_slots, w8a8_bf16* y, w8a8_stream stream) {
+  if (T < 0 || H <= 0 || k <= 0) return W8A8_ERR_ARG;
+  if (H % 128 || k > kMaxTopK || T * k >= (int64_t(1) << 31) / 2) return W8A8_ERR_UNSUPPORTED;
+  if (T == 0) return W8A8_OK;
+  if (!o_sorted || !perm || !topk_w || !o_slots || !y) return W8A8_ERR_ARG;
+  if (!aligned16(o_sorted) || !aligned16(o_slots) || !aligned16(y)) return W8A8_ERR_UNSUPPORTED;
+  const int64_t A = T * k;
+  cudaStream_t s = as_stream(stream);
+  int rc = launch_pdl(scatter_rows_kernel, dim3(unsigned((A + kRowWarps - 1) / kRowWarps)), dim3(kRowWarps * 32), 0,
+                      s, reinterpret_cast<const uint8_t*>(o_sorted), perm, A, int(H * 2),
+                      reinterpret_cast<uint8_t*>(o_slots), A);
+  if (rc != W8A8_OK) return rc;
+  return launch_pdl(combine_kernel, dim3(unsigned(T)), dim3(256), 0, s, reinterpret_cast<const uint16_t*>(o_slots),
+                    topk_w, int(T), int(H), k, reinterpret_cast<uint16_t*>(y), static_cast<const uint16_t*>(nullptr),
+                    static_cast<const float*>(nullptr));
 }
 
 // ------------------------------------------------------------------ allocation-free variant
