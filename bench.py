@@ -602,10 +602,10 @@ MEASURED_TRAFFIC = {
     "qwen3-1.7b-mlp-w4a8": (10_932_992 + 0, "3d048a51e1c8030a8b0a8441792e2ca2d2309450"),
     # the block-scaled MXFP8 GEMM launch (CTA pairs) of the same shape: 17.3 MB read (FP8 weights
     # and scales, token codes and scales, each once), nothing written back within the launch
-    "qwen3-1.7b-mlp-mxfp8": (17_344_000 + 0, "06a20b9f7bcec6397d7ecc1af2a1ebdc06f40292"),
+    "qwen3-1.7b-mlp-mxfp8": (17_344_256 + 0, "6f75f15e5f7becc17f8027677e0192c83257eacd"),
     # the MXFP A8W4 GEMM launch of the same shape: 11.1 MB read (6.3 MB of packed E2M1 weights, their
     # scales, the token codes and scales, each once), nothing written back within the launch
-    "qwen3-1.7b-mlp-mxfp-a8w4": (11_052_544 + 0, "06a20b9f7bcec6397d7ecc1af2a1ebdc06f40292"),
+    "qwen3-1.7b-mlp-mxfp-a8w4": (11_052_544 + 0, "6f75f15e5f7becc17f8027677e0192c83257eacd"),
 }
 TRAFFIC_SOURCES = {  # device-code files each dominant kernel is built from
     "gate_up": ("gemm.cuh", "gemm_pair.cuh", "numerics.cuh", "ptx.cuh", "routing.cuh"),

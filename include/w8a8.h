@@ -180,21 +180,24 @@ int w8a8_moe_forward(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
 int w8a8_moe_route_group(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias, int64_t T, int64_t H, int64_t E,
                          int k, int renorm, void* workspace, size_t workspace_bytes, w8a8_stream stream);
 
-/* Workspace bytes of w8a8_moe_experts for A rows in G groups (0 if rejected: H or I not a
- * multiple of 128, G outside [1, 1024]). */
-size_t w8a8_moe_experts_workspace_size(int64_t A, int64_t H, int64_t I, int64_t G);
+/* Workspace bytes of w8a8_moe_experts for A rows and Ew experts (0 if rejected: H or I not a
+ * multiple of 128, Ew outside [1, 256]). */
+size_t w8a8_moe_experts_workspace_size(int64_t A, int64_t H, int64_t I, int64_t Ew);
 
 /* Steps 3-5 of w8a8_moe_forward on A received rows: grouped gate_up GEMM with dequant and
- * SiLU(gate)*up, per-row requantisation of h, grouped down GEMM with dequant, o [A, H] bf16 in
- * row order.
- *   xq int8 [round_up(A, 128), H] (16-byte aligned; rows past A are read, not used) and sx fp32 [A]:
- *   the rows and their per-token scales; group_offsets_host: HOST array [G+1], offsets[0] = 0,
- *   non-decreasing, offsets[G] = A (else W8A8_ERR_ARG), group g = rows [offsets[g], offsets[g+1]);
- *   group g uses expert g % weight_groups of the Ew experts in wgu [Ew, 2I, H] / s_gu [Ew, 2I] /
- *   wd [Ew, H, I] / s_d [Ew, H] (weight_groups 0: expert g, G <= Ew) -- with W source ranks and
- *   E/W local experts, G = W * E/W groups in source-major order and weight_groups = E/W;
- *   workspace of w8a8_moe_experts_workspace_size(A, H, I, G) bytes (256-byte aligned).
- *   Ew <= 256. All device memory except group_offsets_host owned by the caller. */
+ * SiLU(gate)*up, per-row requantisation of h, grouped down GEMM with dequant; o [A, H] bf16, row r
+ * the output of input row r.
+ *   xq int8 [A, H] (16-byte aligned) and sx fp32 [A]: the rows and their per-token scales;
+ *   group_offsets_host: HOST array [G+1], offsets[0] = 0, non-decreasing, offsets[G] = A (else
+ *   W8A8_ERR_ARG), group g = rows [offsets[g], offsets[g+1]); group g uses expert g % weight_groups
+ *   of the Ew experts in wgu [Ew, 2I, H] / s_gu [Ew, 2I] / wd [Ew, H, I] / s_d [Ew, H]
+ *   (weight_groups 0: expert g, G <= Ew) -- with W source ranks and E/W local experts, G = W * E/W
+ *   groups in source-major order and weight_groups = E/W; G <= 1024;
+ *   workspace of w8a8_moe_experts_workspace_size(A, H, I, Ew) bytes (256-byte aligned).
+ * The call regroups the rows by expert (a row gather into the workspace, the map built on the
+ * host and copied), runs the grouped GEMMs on the experts' row blocks, and the down GEMM writes
+ * each output row back at its input position. All device memory except group_offsets_host owned
+ * by the caller. */
 int w8a8_moe_experts(const int8_t* xq, const float* sx, const int* group_offsets_host, int64_t G,
                      int64_t weight_groups, int64_t A, int64_t H, int64_t I, int64_t Ew, const int8_t* wgu,
                      const float* s_gu, const int8_t* wd, const float* s_d, void* workspace, size_t workspace_bytes,

@@ -335,21 +335,21 @@ def w8a8_moe_route_group(x, wg, E: int, k: int, renorm: bool = True, bias=None, 
     return workspace
 
 
-def w8a8_moe_experts_workspace_size(A: int, H: int, I: int, G: int) -> int:
-    return int(lib().w8a8_moe_experts_workspace_size(A, H, I, G))
+def w8a8_moe_experts_workspace_size(A: int, H: int, I: int, Ew: int) -> int:
+    return int(lib().w8a8_moe_experts_workspace_size(A, H, I, Ew))
 
 
 def w8a8_moe_experts(xq, sx, group_offsets, wgu, s_gu, wd, s_d, weight_groups: int = 0, A: int = None,
                      workspace=None, o=None, stream=None):
-    """Steps 3-5 on received rows: xq int8 [>= round_up(A, 128), H], sx fp32 [A], group_offsets a
-    host sequence of G+1 ints; group g uses expert g % weight_groups (0: g). Returns o bf16 [A, H]."""
+    """Steps 3-5 on received rows: xq int8 [A, H], sx fp32 [A], group_offsets a host sequence of
+    G+1 ints; group g uses expert g % weight_groups (0: g). Returns o bf16 [A, H] in input row order."""
     H = xq.shape[1]
     Ew, twoI, _ = wgu.shape
     I = twoI // 2
     offs = [int(v) for v in group_offsets]
     G = len(offs) - 1
     A = offs[-1] if A is None else A
-    need = w8a8_moe_experts_workspace_size(A, H, I, G)
+    need = w8a8_moe_experts_workspace_size(A, H, I, Ew)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=xq.device)
     o = torch.empty((A, H), dtype=torch.bfloat16, device=xq.device) if o is None else o

@@ -226,6 +226,30 @@ __global__ void __launch_bounds__(kRowWarps * 32) scatter_rows_kernel(const uint
   for (int i = threadIdx.x & 31; i < row_bytes / 16; i += 32) d4[i] = __ldg(s4 + i);
 }
 
+// dst[r, :] = src[map[r], :] for r < R, rows of `row_bytes` bytes (a multiple of 16, both buffers
+// 16-byte aligned), and dst_s[r] = src_s[map[r]] (one fp32 per row): one warp per row. A map
+// value outside [0, src_rows) sets the bad-index bit of the device error word and the row is left.
+__global__ void __launch_bounds__(kRowWarps * 32) gather_rows_kernel(const uint8_t* __restrict__ src,
+                                                                     const float* __restrict__ src_s,
+                                                                     const int* __restrict__ map, int64_t R,
+                                                                     int row_bytes, int64_t src_rows,
+                                                                     uint8_t* __restrict__ dst,
+                                                                     float* __restrict__ dst_s) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t r = int64_t(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (r >= R) return;
+  const int m = __ldg(map + r);
+  if (m < 0 || m >= src_rows) {
+    if ((threadIdx.x & 31) == 0) atomicOr(&g_error_word, kErrBadIndex);
+    return;
+  }
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + int64_t(m) * row_bytes);
+  uint4* d4 = reinterpret_cast<uint4*>(dst + r * row_bytes);
+  for (int i = threadIdx.x & 31; i < row_bytes / 16; i += 32) d4[i] = __ldg(s4 + i);
+  if ((threadIdx.x & 31) == 0) dst_s[r] = __ldg(src_s + m);
+}
+
 // y[t, :] = bf16(sum_j w[t, j] * o[t, j, :]): fp32 fused multiply-adds in slot order from 0.
 // With a shared expert (o_shared != nullptr) one more fused multiply-add follows the k slots:
 // acc = fma(g[t], o_shared[t, :], acc).

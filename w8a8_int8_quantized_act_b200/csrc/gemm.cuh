@@ -62,8 +62,7 @@ struct GemmParams {
   const float* col_scale;      // per channel scale, group-major
   int col_scale_stride;        // per group
   int up_offset;               // gate_up: offset of the up scales inside a group's scales
-  const int* row_map;          // down: sorted row -> slot row (t*k + j); nullptr: the sorted row
-  int weight_groups;           // > 0: group g uses the weights and scales of group g % weight_groups
+  const int* row_map;          // down: sorted row -> slot row (t*k + j)
   // router
   const float* bias;
   int topk;
@@ -126,8 +125,7 @@ __device__ __forceinline__ int find_group(const int* prefix, int G, int mt) {
 }
 
 struct Tile {
-  int g;       // group (token rows)
-  int wg;      // weight group (expert): g, or g % weight_groups
+  int g;       // group (expert)
   int cb;      // channel block (router: 0)
   int tok0;    // first token row of the tile
   int rows;    // valid token rows
@@ -144,7 +142,6 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* mt_p
     // router_rows tokens per tile (the MMA keeps M = 128: lanes past them compute values that
     // nobody reads); the histogram row is the tile's 128-token chunk
     c.g = 0;
-    c.wg = 0;
     c.cb = 0;
     c.tok0 = tile * p.router_rows;
     c.tt = c.tok0 / kBM;
@@ -168,10 +165,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* mt_p
       cnt = goff[c.g + 1] - off;
       blk = mt - mt_prefix[c.g];
     }
-    c.wg = p.weight_groups > 0 ? c.g % p.weight_groups : c.g;
     c.tok0 = off + blk * NB;
     c.rows = min(NB, cnt - blk * NB);
-    c.a_row = c.wg * p.a_rows_per_group + c.cb * p.a_cb_step;
+    c.a_row = c.g * p.a_rows_per_group + c.cb * p.a_cb_step;
     c.b_row = c.tok0;
     c.nb = (c.rows + 15) & ~15;
   }
@@ -237,8 +233,8 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
   const float* __restrict__ row_scale = p.row_scale;
   uint32_t r[16];
   if constexpr (EPI == kEpiGateUp) {
-    const float sg = __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + ch);
-    const float su = __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + p.up_offset + ch);
+    const float sg = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+    const float su = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + p.up_offset + ch);
     uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
     uint32_t ru[16];
 #pragma unroll 1
@@ -278,8 +274,8 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
   } else if constexpr (EPI == kEpiDown || EPI == kEpiDense) {
     // two 128-channel blocks: accumulator columns [0, NB) and [NB, 2NB)
     const bool second = ch + kBM < p.n_channels;
-    const float sc0 = __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + ch);
-    const float sc1 = second ? __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + ch + kBM) : 0.0f;
+    const float sc0 = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+    const float sc1 = second ? __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch + kBM) : 0.0f;
     const int* __restrict__ row_map = p.row_map;
     uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
     uint32_t r1[16];
@@ -292,7 +288,7 @@ __device__ __forceinline__ void epilogue_channels(const GemmParams& p, const Til
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         srow[j] = (j < nj) ? (tile_scale != nullptr ? tile_scale[j0 + j] : __ldg(row_scale + row0 + j)) : 0.0f;
-        orow[j] = (EPI == kEpiDown && row_map != nullptr) ? ((j < nj) ? __ldg(row_map + row0 + j) : 0) : row0 + j;
+        orow[j] = (EPI == kEpiDown) ? ((j < nj) ? __ldg(row_map + row0 + j) : 0) : row0 + j;
       }
       tmem_ld16x2(t_lane + j0, t_lane + NB + j0, r, r1);
       uint32_t v0[16], v1[16];

@@ -46,8 +46,7 @@ struct PairParams {
   const float* col_scale;
   int col_scale_stride;
   int up_offset;
-  const int* row_map;        // down: sorted row -> output row; nullptr: the sorted row
-  int weight_groups;         // > 0: group g uses the weights and scales of group g % weight_groups
+  const int* row_map;
 };
 
 // Epilogue warps per CTA: several per TMEM lane quarter, so that while one waits on a TMEM or
@@ -75,7 +74,7 @@ struct PairCfg {
 };
 
 struct PairTile {
-  int g, wg, cb, tok0, rows, n;  // wg: weight group (g, or g % weight_groups); n: MMA N = rows rounded up to 16
+  int g, cb, tok0, rows, n;  // n: MMA N = rows rounded up to 16
 };
 
 // Decodes tile (mt, cb). `g_hint` is the group of an earlier token block (0 at first): every
@@ -99,7 +98,6 @@ __device__ __forceinline__ PairTile pair_tile(const PairParams& p, const int* mt
     cnt = goff[g + 1] - off;
     blk = mt - mt_prefix[g];
   }
-  c.wg = p.weight_groups > 0 ? c.g % p.weight_groups : c.g;
   c.tok0 = off + blk * kPairNB;
   c.rows = min(kPairNB, cnt - blk * kPairNB);
   c.n = (c.rows + 15) & ~15;
@@ -155,8 +153,8 @@ struct PairTileIter {
 template <int W>
 __device__ __forceinline__ void pair_epilogue_gate_up(const PairParams& p, const PairTile& c, uint32_t t_lane,
                                                       int ch, bool is_up, int wq, const float* srow) {
-  const float sg = __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + ch);
-  const float su = __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + p.up_offset + ch);
+  const float sg = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch);
+  const float su = __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + p.up_offset + ch);
   uint16_t* out = static_cast<uint16_t*>(p.out) + ch;
   const size_t ldo = size_t(p.ldo);
   const int my0 = is_up ? 8 : 0;  // first token of the chunk this lane computes
@@ -224,7 +222,7 @@ __device__ __forceinline__ void pair_epilogue_channels(const PairParams& p, cons
   } else {
     // bf16 values go through this warp's 16 x 32 shared-memory block: lane = channel on the way
     // in, then four lanes per token row (8 channels = 16 bytes each) on the way out
-    const float s_col = valid ? __ldg(p.col_scale + size_t(c.wg) * p.col_scale_stride + ch) : 0.0f;
+    const float s_col = valid ? __ldg(p.col_scale + size_t(c.g) * p.col_scale_stride + ch) : 0.0f;
     const int lane = threadIdx.x & 31;
     const int ch0 = ch - lane;                      // first channel of the warp's 32
     const int jr = lane >> 2, cc = (lane & 3) * 8;  // token row (and row + 8), channel piece
@@ -354,7 +352,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
       const uint32_t bytes = uint32_t(Cfg::kABytes + hn * kKBlockBytes);
       const int b_row = c.tok0 + int(rank) * hn;
       const int a_y = (EPI == kEpiGateUp) ? (c.cb * 128 + int(rank) * 64) / 16
-                                          : c.wg * p.a_rows_per_group + c.cb * 256 + int(rank) * 128;
+                                          : c.g * p.a_rows_per_group + c.cb * 256 + int(rank) * 128;
       for (int kb = 0; kb < p.num_kb; ++kb) {
         if (!mbar_wait_warp(empty + stage, phase ^ 1u, wc)) { ok = false; break; }
         if (elect_one()) {
@@ -365,7 +363,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
           const int x = kb * kKBlockBytes;
           if constexpr (EPI == kEpiGateUp) {
             // 4 x (16 gate rows, 16 up rows) of channels cb*128 + 64*rank + [0, 64), one copy
-            tma_load_5d_pair(sa, &p.tmA, bar, x, 0, 0, a_y, c.wg);
+            tma_load_5d_pair(sa, &p.tmA, bar, x, 0, 0, a_y, c.g);
           } else {
             tma_load_2d_pair(sa, &p.tmA, bar, x, a_y);
           }
@@ -484,7 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI>::kThrea
     auto load_rows = [&](const PairTile& t) {
       const bool in = et < t.rows;
       if constexpr (EPI != kEpiRawS32) pre_s = in ? __ldg(p.row_scale + t.tok0 + et) : 0.0f;
-      if constexpr (EPI == kEpiDown) pre_m = in ? (p.row_map ? __ldg(p.row_map + t.tok0 + et) : t.tok0 + et) : 0;
+      if constexpr (EPI == kEpiDown) pre_m = in ? __ldg(p.row_map + t.tok0 + et) : 0;
     };
     PairTileIter it(cluster, nclusters, p.n_cb);
     PairTile c{};

@@ -5,6 +5,7 @@
 #include <stdlib.h>
 
 #include <mutex>
+#include <vector>
 
 #include "../../include/w8a8.h"
 #include "elementwise.cuh"
@@ -733,9 +734,9 @@ int route_group_stage(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias
 }
 
 // Operands of the grouped expert FFN: A sorted token rows xq [round_up(A, 128), H] with their
-// scales, G groups of consecutive rows (offsets [G+1] on the device), the intermediates h, s_h, hq
-// (round_up(A, 128) rows) and the output o; row_map sends sorted row r to output row row_map[r]
-// (nullptr: row r).
+// scales, G groups of consecutive rows (offsets [G+1] on the device; group g uses expert g), the
+// intermediates h, s_h, hq (round_up(A, 128) rows) and the output o; row_map sends sorted row r
+// to output row row_map[r].
 struct ExpertRows {
   const int8_t* xq;
   const float* sx;
@@ -748,9 +749,8 @@ struct ExpertRows {
 };
 
 // Steps 3-5 of the forward: grouped gate_up with dequant + SiLU(gate)*up, the requantisation of h,
-// grouped down with dequant. Group g uses the weights and scales of expert g % weight_groups
-// (weight_groups 0: expert g); Ew experts are held in wgu [Ew, 2I, H] / wd [Ew, H, I].
-int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t weight_groups, int64_t Ew, int64_t H, int64_t I,
+// grouped down with dequant; the G = Ew experts are held in wgu [Ew, 2I, H] / wd [Ew, H, I].
+int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t Ew, int64_t H, int64_t I,
                   const int8_t* wgu, const float* s_gu, const int8_t* wd, const float* s_d, cudaStream_t s,
                   void* const* ev) {
   const int64_t Ap = round_up(A > 0 ? A : 1, 128);
@@ -770,7 +770,6 @@ int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t weight_grou
     p.n_cb = int(I / 128);
     p.num_groups = int(G);
     p.group_offsets = b.offsets;
-    p.weight_groups = int(weight_groups);
     p.a_rows_per_group = int(2 * I);
     p.a_second_offset = int(I);
     p.a_cb_step = 128;
@@ -792,7 +791,6 @@ int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t weight_grou
     p.n_cb = int(I / 128);
     p.num_groups = int(G);
     p.group_offsets = b.offsets;
-    p.weight_groups = int(weight_groups);
     p.a_rows_per_group = int(2 * I);
     p.n_channels = int(I);
     p.timeout_ns = wait_timeout_ns();
@@ -825,7 +823,6 @@ int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t weight_grou
     p.n_channels = int(H);
     p.num_groups = int(G);
     p.group_offsets = b.offsets;
-    p.weight_groups = int(weight_groups);
     p.a_rows_per_group = int(H);
     p.a_second_offset = 128;
     p.a_cb_step = 256;
@@ -856,7 +853,6 @@ int experts_stage(const ExpertRows& b, int64_t A, int64_t G, int64_t weight_grou
   p.n_channels = int(H);
   p.num_groups = int(G);
   p.group_offsets = b.offsets;
-  p.weight_groups = int(weight_groups);
   p.a_rows_per_group = int(H);
   p.timeout_ns = wait_timeout_ns();
   p.out = b.o;
@@ -905,7 +901,7 @@ int moe_forward_impl(const w8a8_bf16* x, const w8a8_bf16* wg, const float* bias,
   int rc = route_group_stage(x, wg, bias, T, H, E, k, renorm, ws, L, s, ev);
   if (rc != W8A8_OK) return rc;
   ExpertRows b{xq, sx_sorted, offsets, h, s_h, hq, o, perm};
-  if ((rc = experts_stage(b, A, E, 0, E, H, I, wgu, s_gu, wd, s_d, s, ev)) != W8A8_OK) return rc;
+  if ((rc = experts_stage(b, A, E, E, H, I, wgu, s_gu, wd, s_d, s, ev)) != W8A8_OK) return rc;
 
   // 5b. the shared expert (every token): its bf16 gate, per-token int8 x, the dense gate_up GEMM
   //     with the SiLU*up epilogue, the requantisation of its h, the dense down GEMM
@@ -991,12 +987,36 @@ int w8a8_moe_route_group(const w8a8_bf16* x, const w8a8_bf16* wg, const float* b
                            as_stream(stream), nullptr);
 }
 
-size_t w8a8_moe_experts_workspace_size(int64_t A, int64_t H, int64_t I, int64_t G) {
-  if (A < 0 || H <= 0 || I <= 0 || G <= 0 || H % 128 || I % 128 || G > kMaxGroups) return 0;
-  if (A >= (int64_t(1) << 30)) return 0;
+// Workspace of w8a8_moe_experts: the experts' row offsets and the row map (device copies of what
+// the host builds), the rows and scales regrouped by expert, then h, s_h and hq.
+struct ExpertsWs {
+  size_t offsets, map, xq, sx, h, s_h, hq, total;
+};
+
+ExpertsWs experts_ws(int64_t A, int64_t H, int64_t I, int64_t Ew) {
   const size_t Ap = size_t(round_up(A > 0 ? A : 1, 128));
-  return align256(sizeof(int) * size_t(G + 1)) + align256(Ap * I * 2) + align256(sizeof(float) * Ap) +
-         align256(Ap * I);
+  ExpertsWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  w.offsets = take(sizeof(int) * size_t(Ew + 1));
+  w.map = take(sizeof(int) * Ap);
+  w.xq = take(Ap * size_t(H));
+  w.sx = take(sizeof(float) * Ap);
+  w.h = take(Ap * size_t(I) * 2);
+  w.s_h = take(sizeof(float) * Ap);
+  w.hq = take(Ap * size_t(I));
+  w.total = off;
+  return w;
+}
+
+size_t w8a8_moe_experts_workspace_size(int64_t A, int64_t H, int64_t I, int64_t Ew) {
+  if (A < 0 || H <= 0 || I <= 0 || Ew <= 0 || H % 128 || I % 128 || Ew > 256) return 0;
+  if (A >= (int64_t(1) << 30)) return 0;
+  return experts_ws(A, H, I, Ew).total;
 }
 
 int w8a8_moe_experts(const int8_t* xq, const float* sx, const int* group_offsets_host, int64_t G,
@@ -1004,8 +1024,8 @@ int w8a8_moe_experts(const int8_t* xq, const float* sx, const int* group_offsets
                      const float* s_gu, const int8_t* wd, const float* s_d, void* workspace, size_t workspace_bytes,
                      w8a8_bf16* o, w8a8_stream stream) {
   if (A < 0 || H <= 0 || I <= 0 || G <= 0 || Ew <= 0 || weight_groups < 0) return W8A8_ERR_ARG;
-  const size_t need = w8a8_moe_experts_workspace_size(A, H, I, G);
-  if (need == 0 || Ew > 256 || Ew * 2 * I >= (int64_t(1) << 31) || Ew * H >= (int64_t(1) << 31))
+  const size_t need = w8a8_moe_experts_workspace_size(A, H, I, Ew);
+  if (need == 0 || G > kMaxGroups || Ew * 2 * I >= (int64_t(1) << 31) || Ew * H >= (int64_t(1) << 31))
     return W8A8_ERR_UNSUPPORTED;
   if (weight_groups > Ew || (weight_groups == 0 && G > Ew)) return W8A8_ERR_ARG;
   if (!group_offsets_host) return W8A8_ERR_ARG;
@@ -1018,18 +1038,40 @@ int w8a8_moe_experts(const int8_t* xq, const float* sx, const int* group_offsets
   if (!aligned16(xq) || !aligned16(wgu) || !aligned16(wd) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return W8A8_ERR_UNSUPPORTED;
-  const size_t Ap = size_t(round_up(A, 128));
+  // rows regrouped by expert: expert e takes the groups g with g % weight_groups == e (or g == e)
+  // in increasing g; map[r] = the input row placed at regrouped row r, which is also where the
+  // down GEMM writes that row's output
+  std::vector<int> exp_off(static_cast<size_t>(Ew + 1), 0);
+  std::vector<int> map(static_cast<size_t>(A), 0);
+  int next = 0;
+  for (int64_t e = 0; e < Ew; ++e) {
+    exp_off[size_t(e)] = next;
+    for (int64_t g = 0; g < G; ++g) {
+      if ((weight_groups > 0 ? g % weight_groups : g) != e) continue;
+      for (int i = group_offsets_host[g]; i < group_offsets_host[g + 1]; ++i) map[size_t(next++)] = i;
+    }
+  }
+  exp_off[size_t(Ew)] = next;
+  if (next != A) return W8A8_ERR_ARG;  // groups past Ew experts (weight_groups 0)
+  const ExpertsWs L = experts_ws(A, H, I, Ew);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int* offsets = reinterpret_cast<int*>(ws);
-  uint16_t* h = reinterpret_cast<uint16_t*>(ws + align256(sizeof(int) * size_t(G + 1)));
-  float* s_h = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(h) + align256(Ap * I * 2));
-  int8_t* hq = reinterpret_cast<int8_t*>(reinterpret_cast<uint8_t*>(s_h) + align256(sizeof(float) * Ap));
+  int* d_off = reinterpret_cast<int*>(ws + L.offsets);
+  int* d_map = reinterpret_cast<int*>(ws + L.map);
+  int8_t* xq_g = reinterpret_cast<int8_t*>(ws + L.xq);
+  float* sx_g = reinterpret_cast<float*>(ws + L.sx);
   cudaStream_t s = as_stream(stream);
-  if (cudaMemcpyAsync(offsets, group_offsets_host, sizeof(int) * size_t(G + 1), cudaMemcpyHostToDevice, s) !=
-      cudaSuccess)
+  // pageable host sources: the copies have read them when the calls return
+  if (cudaMemcpyAsync(d_off, exp_off.data(), sizeof(int) * exp_off.size(), cudaMemcpyHostToDevice, s) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(d_map, map.data(), sizeof(int) * map.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return W8A8_ERR_LAUNCH;
-  ExpertRows b{xq, sx, offsets, h, s_h, hq, reinterpret_cast<uint16_t*>(o), nullptr};
-  return experts_stage(b, A, G, weight_groups, Ew, H, I, wgu, s_gu, wd, s_d, s, nullptr);
+  int rc = launch_pdl(gather_rows_kernel, dim3(unsigned((A + kRowWarps - 1) / kRowWarps)), dim3(kRowWarps * 32), 0,
+                      s, reinterpret_cast<const uint8_t*>(xq), sx, static_cast<const int*>(d_map), A, int(H), A,
+                      reinterpret_cast<uint8_t*>(xq_g), sx_g);
+  if (rc != W8A8_OK) return rc;
+  ExpertRows b{xq_g, sx_g, d_off, reinterpret_cast<uint16_t*>(ws + L.h), reinterpret_cast<float*>(ws + L.s_h),
+               reinterpret_cast<int8_t*>(ws + L.hq), reinterpret_cast<uint16_t*>(o), d_map};
+  return experts_stage(b, A, Ew, Ew, H, I, wgu, s_gu, wd, s_d, s, nullptr);
 }
 
 int w8a8_moe_combine_sorted(const w8a8_bf16* o_sorted, const int* perm, const float* topk_w, int64_t T, int64_t H,

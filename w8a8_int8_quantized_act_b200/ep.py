@@ -8,8 +8,9 @@ explainer: 128 experts, 8 per token, weights sharded so that several cards serve
      per-token int8 rows (sorted, so the rows for each destination rank are consecutive);
   2. dispatch: the per-(destination, local expert) row counts, then the int8 rows and their fp32
      scales, by all-to-all;
-  3. experts: the grouped gate_up / requantisation / down on the received rows, in groups of
-     (source rank, local expert), source-major, each using its local expert's weights;
+  3. experts: the grouped gate_up / requantisation / down on the received rows, given as groups
+     of (source rank, local expert), source-major (regrouped by expert inside the call, the
+     outputs written back in received order);
   4. return: the bf16 expert outputs, by all-to-all in the reverse direction;
   5. combine: the outputs back in slot order and the ordered fma chain over the k slots.
 
@@ -61,13 +62,11 @@ class GpuSteps:
                       topk_w=v["topk_w"], xq=v["xq"][:A], sx=v["sx_sorted"][:A])
 
     def alloc_rows(self, A: int, H: int, device) -> torch.Tensor:
-        # the expert GEMMs read rows up to round_up(A, 128): received rows land in a padded buffer
-        Ap = max(1, -(-A // 128)) * 128
-        return torch.zeros((Ap, H), dtype=torch.int8, device=device)
+        return torch.empty((A, H), dtype=torch.int8, device=device)
 
-    def experts(self, xq_padded, sx, offsets: list, weights, weight_groups: int) -> torch.Tensor:
+    def experts(self, xq, sx, offsets: list, weights, weight_groups: int) -> torch.Tensor:
         wgu, s_gu, wd, s_d = weights
-        return self.B.w8a8_moe_experts(xq_padded, sx, offsets, wgu, s_gu, wd, s_d, weight_groups=weight_groups)
+        return self.B.w8a8_moe_experts(xq, sx, offsets, wgu, s_gu, wd, s_d, weight_groups=weight_groups)
 
     def combine(self, o_sorted, perm, topk_w, k: int) -> torch.Tensor:
         return self.B.w8a8_moe_combine_sorted(o_sorted, perm, topk_w, k)
