@@ -1,9 +1,9 @@
-"""Expert parallelism (w8a8_int8_quantized_act_b200/ep.py) across two ``gloo`` ranks on CPU.
+"""Expert parallelism (w8a8_int8_quantized_act_b200/ep.py) across two and four ``gloo`` ranks on CPU.
 
 The exchange logic of ExpertParallelMoE runs as it does on GPUs (all-to-alls of the counts, the
 int8 rows, their fp32 scales and the bf16 outputs, the (source rank, local expert) groups of the
 received rows); its three compute steps are given here by the oracle, so that the result can be
-checked without a GPU. Each rank holds half the experts and its own tokens; y of every rank must
+checked without a GPU. Each rank holds its share of the experts and its own tokens; y of every rank must
 equal, bit for bit, the single-process oracle forward of all ranks' tokens with the same routing
 ("Qwen3-235B-A22B-quantized.w8a8" file-structure explainer: 128 experts, 8 per token, weights
 sharded over cards; every step of the forward is row-wise, so the split changes no bit).
@@ -16,7 +16,7 @@ import sys
 import numpy as np
 import pytest
 
-WORLD = 2
+WORLD = 2  # the default; one case below runs four ranks
 
 
 def _free_port() -> int:
@@ -88,7 +88,7 @@ class OracleSteps:
         return _bf16_tensor(O.combine(slots.reshape(A // k, k, H), topk_w.numpy()))
 
 
-def _worker(rank, world, port, root, tokens, k):
+def _worker(rank, world, port, root, tokens, k, E=8):
     if root not in sys.path:
         sys.path.insert(0, root)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -101,7 +101,7 @@ def _worker(rank, world, port, root, tokens, k):
 
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        wl = synth.MoEWorkload("ep", T=sum(tokens), H=256, E=8, k=k, I=128, n_outlier=2, seed=5)
+        wl = synth.MoEWorkload("ep", T=sum(tokens), H=256, E=E, k=k, I=128, n_outlier=2, seed=5)
         inp = synth.moe_inputs(wl)
         wgu_q, s_gu, wd_q, s_d = O.quantize_experts(inp.wgu, inp.wd)
         # every rank builds the same global batch and takes its own slice of tokens
@@ -128,6 +128,17 @@ def test_expert_parallel_two_gloo_ranks(tokens, k):
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     mp.start_processes(_worker, args=(WORLD, _free_port(), root, tokens, k), nprocs=WORLD, join=True,
+                       start_method="spawn")
+
+
+def test_expert_parallel_four_gloo_ranks():
+    # four sources per destination, uneven token counts and one rank without tokens: the
+    # (source, local expert) groups of the received rows in source-major order
+    import torch.multiprocessing as mp
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    tokens = (31, 0, 70, 16)
+    mp.start_processes(_worker, args=(4, _free_port(), root, tokens, 3, 16), nprocs=4, join=True,
                        start_method="spawn")
 
 
