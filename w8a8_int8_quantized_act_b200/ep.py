@@ -77,8 +77,10 @@ class ExpertParallelMoE:
 
     wg [E, H] bf16 (replicated), local expert weights wgu [E/W, 2I, H] int8, s_gu [E/W, 2I],
     wd [E/W, H, I] int8, s_d [E/W, H]; forward(x [T_local, H] bf16) -> y [T_local, H] bf16.
-    Every rank takes the same collective steps in the same order (two all-to-alls of counts,
-    rows and scales out, rows back), also when it has no tokens.
+    Every rank takes the same collective steps in the same order (the counts, then rows and
+    scales out, then rows back), also when it has no tokens. A rank that raises between the
+    exchanges leaves the others in their next all-to-all until the process group's timeout ends it
+    with an error, so give the group a short timeout.
     """
 
     def __init__(self, wg, wgu, s_gu, wd, s_d, E: int, k: int, renorm: bool = True, bias=None, group=None,
